@@ -1,0 +1,174 @@
+"""CPU oracle for ``y = x @ dequant(W_q)``.
+
+TEST INFRASTRUCTURE: only ``tests/``, ``__graft_entry__.smoke()`` and the
+bench's CPU-baseline / reference arm may import this package.  The product
+(``gemm_wq_gemv_b200``) never imports it and never falls back to it.
+
+Two independent restatements of the same plain definition live here:
+
+* ``wq_oracle.c`` (plain C, fp64, loaded with ctypes) -- the oracle proper;
+* ``numpy_oracle`` (NumPy, fp64) -- a twin written separately, used to
+  cross-check the C file on small shapes.
+
+Both follow ``dashq_kernel.py`` (module docstring, ``_pack_kmajor``,
+``_unpack_kmajor``, ``TritonQuantLinear.__init__``, ``dequantize_weight``,
+``forward``) and the "GPTQModel-Compatible Triton Kernel" README (sections
+"API Reference", "Dequantization Formula", "Group Quantization").
+
+Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
+(hand-derived golden words and products, closed forms, brute force, library
+special cases); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from pathlib import Path
+
+import numpy as np
+
+from . import numpy_oracle  # noqa: F401  (re-exported twin)
+
+_HERE = Path(__file__).resolve().parent
+_SRC = _HERE / "wq_oracle.c"
+_LIB = _HERE / "liboracle.so"
+_lib = None
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def build(force: bool = False) -> Path:
+    """Compile ``wq_oracle.c`` into ``liboracle.so`` (gcc -O2, OpenMP, no fast-math)."""
+    if force or not _LIB.exists() or _LIB.stat().st_mtime < _SRC.stat().st_mtime:
+        tmp = _LIB.with_suffix(f".so.tmp{os.getpid()}")
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-Wall",
+               "-o", str(tmp), str(_SRC), "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(str(_LIB))
+        p = ctypes.c_void_p
+        i = ctypes.c_int
+        L.orc_threads.restype = i
+        L.orc_half_to_double.argtypes = [ctypes.c_uint16]
+        L.orc_half_to_double.restype = ctypes.c_double
+        L.orc_pack_kmajor.argtypes = [p, i, i, i, p, p]
+        L.orc_unpack_kmajor.argtypes = [p, p, i, i, i, p]
+        L.orc_dequant.argtypes = [p, p, p, p, i, i, i, i, p]
+        L.orc_matmul.argtypes = [p, p, i, i, i, p, p]
+        L.orc_wq_matmul.argtypes = [p, p, p, p, p, i, i, i, i, i, p, p]
+        L.orc_wq_matmul_sampled.argtypes = [p, p, p, p, p, i, i, i, i, i, p, p, i, p, p]
+        for f in ("orc_pack_kmajor", "orc_unpack_kmajor", "orc_dequant", "orc_matmul",
+                  "orc_wq_matmul", "orc_wq_matmul_sampled"):
+            getattr(L, f).restype = i
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise OracleError(f"{what} failed with code {rc}")
+
+
+def words_shape(K: int, N: int, bits: int):
+    """Shapes of the packed planes: (hi/only plane, lo plane or None)."""
+    if bits == 3:
+        return (K // 16, N), (K // 32, N)
+    return (K // (32 // bits), N), None
+
+
+def threads() -> int:
+    return int(lib().orc_threads())
+
+
+def half_to_double(h: int) -> float:
+    return float(lib().orc_half_to_double(int(h) & 0xFFFF))
+
+
+def pack(codes_kn: np.ndarray, bits: int):
+    """``(K, N)`` uint8 codes -> ``(wq, wlo)`` uint32 words (``wlo`` is None unless 3-bit)."""
+    codes = np.ascontiguousarray(codes_kn, dtype=np.uint8)
+    K, N = codes.shape
+    hs, ls = words_shape(K, N, bits)
+    wq = np.zeros(hs, dtype=np.uint32)
+    wlo = np.zeros(ls, dtype=np.uint32) if ls else None
+    _check(lib().orc_pack_kmajor(_ptr(codes), K, N, bits, _ptr(wq), _ptr(wlo)), "pack")
+    return wq, wlo
+
+
+def unpack(wq: np.ndarray, wlo, K: int, N: int, bits: int) -> np.ndarray:
+    wq = np.ascontiguousarray(wq, dtype=np.uint32)
+    wlo = None if wlo is None else np.ascontiguousarray(wlo, dtype=np.uint32)
+    out = np.zeros((K, N), dtype=np.uint8)
+    _check(lib().orc_unpack_kmajor(_ptr(wq), _ptr(wlo), K, N, bits, _ptr(out)), "unpack")
+    return out
+
+
+def dequant(wq, wlo, scales, zeros, K: int, N: int, bits: int, group_size: int) -> np.ndarray:
+    wq = np.ascontiguousarray(wq, dtype=np.uint32)
+    wlo = None if wlo is None else np.ascontiguousarray(wlo, dtype=np.uint32)
+    s = np.ascontiguousarray(scales, dtype=np.float16).view(np.uint16)
+    z = np.ascontiguousarray(zeros, dtype=np.float16).view(np.uint16)
+    w = np.zeros((K, N), dtype=np.float64)
+    _check(lib().orc_dequant(_ptr(wq), _ptr(wlo), _ptr(s), _ptr(z), K, N, bits, group_size,
+                             _ptr(w)), "dequant")
+    return w
+
+
+def matmul(x, w_kn):
+    x = np.ascontiguousarray(x, dtype=np.float16).view(np.uint16)
+    w = np.ascontiguousarray(w_kn, dtype=np.float64)
+    M, K = x.shape
+    N = w.shape[1]
+    y = np.zeros((M, N), dtype=np.float64)
+    b = np.zeros((M, N), dtype=np.float64)
+    _check(lib().orc_matmul(_ptr(x), _ptr(w), M, K, N, _ptr(y), _ptr(b)), "matmul")
+    return y, b
+
+
+def wq_matmul(x, wq, wlo, scales, zeros, bits: int, group_size: int, N: int | None = None):
+    """``(y_ref, bound)`` in fp64 for the packed problem (unpack, dequant, matmul)."""
+    x = np.ascontiguousarray(x, dtype=np.float16).view(np.uint16)
+    M, K = x.shape
+    wq = np.ascontiguousarray(wq, dtype=np.uint32)
+    N = wq.shape[1] if N is None else N
+    wlo = None if wlo is None else np.ascontiguousarray(wlo, dtype=np.uint32)
+    s = np.ascontiguousarray(scales, dtype=np.float16).view(np.uint16)
+    z = np.ascontiguousarray(zeros, dtype=np.float16).view(np.uint16)
+    y = np.zeros((M, N), dtype=np.float64)
+    b = np.zeros((M, N), dtype=np.float64)
+    _check(lib().orc_wq_matmul(_ptr(x), _ptr(wq), _ptr(wlo), _ptr(s), _ptr(z), M, K, N, bits,
+                               group_size, _ptr(y), _ptr(b)), "wq_matmul")
+    return y, b
+
+
+def wq_matmul_sampled(x, wq, wlo, scales, zeros, bits: int, group_size: int, ms, ns):
+    """``(y_ref, bound)`` for the single outputs ``(ms[i], ns[i])``."""
+    x = np.ascontiguousarray(x, dtype=np.float16).view(np.uint16)
+    M, K = x.shape
+    wq = np.ascontiguousarray(wq, dtype=np.uint32)
+    N = wq.shape[1]
+    wlo = None if wlo is None else np.ascontiguousarray(wlo, dtype=np.uint32)
+    s = np.ascontiguousarray(scales, dtype=np.float16).view(np.uint16)
+    z = np.ascontiguousarray(zeros, dtype=np.float16).view(np.uint16)
+    ms = np.ascontiguousarray(ms, dtype=np.int32)
+    ns = np.ascontiguousarray(ns, dtype=np.int32)
+    y = np.zeros(len(ms), dtype=np.float64)
+    b = np.zeros(len(ms), dtype=np.float64)
+    _check(lib().orc_wq_matmul_sampled(_ptr(x), _ptr(wq), _ptr(wlo), _ptr(s), _ptr(z), M, K, N,
+                                       bits, group_size, _ptr(ms), _ptr(ns), len(ms), _ptr(y),
+                                       _ptr(b)), "wq_matmul_sampled")
+    return y, b

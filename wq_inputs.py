@@ -1,0 +1,94 @@
+"""Seeded synthetic inputs for the weight-only quantized matrix product.
+
+This module draws random numbers and nothing else: it holds none of the
+method's arithmetic (no packing, no dequantisation, no product).  Both the CPU
+oracle (through the tests) and the CUDA path (through the tests and the bench)
+take their inputs from here, so the two sides see byte-identical data.
+
+Shapes and distributions follow the workloads the method is described on
+(``dashq_kernel.py``: K-major codes ``(K, N)``, per-group ``s, z`` of shape
+``(K // group_size, N)``; "GPTQModel-Compatible Triton Kernel" README, section
+"API Reference": ``x`` of shape ``(M, K)``, ``group_size = -1`` meaning one
+group per output channel).
+
+Recipe (one ``numpy.random.default_rng(seed)`` stream, PCG64, drawn in this
+order): ``x`` ~ N(0, 1) rounded to fp16; codes uniform integers in
+``[0, 2**bits - 1]``; scales uniform in ``[s_lo, s_hi]`` rounded to fp16;
+zeros uniform integers in ``[0, 2**bits - 1]`` stored as fp16.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One synthetic problem: ``y (M, N) = x (M, K) @ dequant(codes (K, N))``."""
+
+    name: str
+    M: int
+    K: int
+    N: int
+    bits: int
+    group_size: int  # -1: one group spanning all of K
+    s_lo: float = 0.005
+    s_hi: float = 0.02
+
+    @property
+    def groups(self) -> int:
+        return 1 if self.group_size == -1 else self.K // self.group_size
+
+
+@dataclass
+class Case:
+    """Host arrays of one drawn problem (numpy, C-contiguous)."""
+
+    wl: Workload
+    x: np.ndarray        # (M, K) float16
+    codes: np.ndarray    # (K, N) uint8, values in [0, 2**bits - 1]
+    scales: np.ndarray   # (groups, N) float16
+    zeros: np.ndarray    # (groups, N) float16, integer-valued
+    seed: int = 0
+    extra: dict = field(default_factory=dict)
+
+
+# The named workloads: the small parity case, the decode GEMV at three token
+# counts, the 3-bit two-plane GEMV, the bit-width sweep and the batched GEMM.
+WORKLOADS = {
+    "tiny_gemv": Workload("tiny_gemv", 1, 512, 256, 4, 128),
+    "decode_gemv_m1": Workload("decode_gemv_m1", 1, 4096, 4096, 4, 128),
+    "decode_gemv_m4": Workload("decode_gemv_m4", 4, 4096, 4096, 4, 128),
+    "decode_gemv_m16": Workload("decode_gemv_m16", 16, 4096, 4096, 4, 128),
+    "gemv_3bit": Workload("gemv_3bit", 1, 4096, 11008, 3, 128, 0.01, 0.04),
+    "sweep_1bit": Workload("sweep_1bit", 1, 8192, 8192, 1, 128),
+    "sweep_2bit": Workload("sweep_2bit", 1, 8192, 8192, 2, 128),
+    "sweep_8bit": Workload("sweep_8bit", 1, 8192, 8192, 8, 128),
+    "sweep_8bit_perchannel": Workload("sweep_8bit_perchannel", 1, 8192, 8192, 8, -1),
+    "prefill_gemm": Workload("prefill_gemm", 512, 4096, 2048, 4, 128),
+}
+
+
+def draw(wl: Workload, seed: int = 0) -> Case:
+    """Draw one problem for workload ``wl`` from ``default_rng(seed)``."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((wl.M, wl.K)).astype(np.float16)
+    qmax = (1 << wl.bits) - 1
+    codes = rng.integers(0, qmax + 1, size=(wl.K, wl.N), dtype=np.int64).astype(np.uint8)
+    scales = rng.uniform(wl.s_lo, wl.s_hi, size=(wl.groups, wl.N)).astype(np.float16)
+    zeros = rng.integers(0, qmax + 1, size=(wl.groups, wl.N), dtype=np.int64).astype(np.float16)
+    return Case(wl, np.ascontiguousarray(x), np.ascontiguousarray(codes),
+                np.ascontiguousarray(scales), np.ascontiguousarray(zeros), seed)
+
+
+def custom(M: int, K: int, N: int, bits: int, group_size: int, seed: int = 0,
+           s_lo: float = 0.005, s_hi: float = 0.02, name: str = "custom") -> Case:
+    """Draw a problem of arbitrary shape with the same distributions."""
+    return draw(Workload(name, M, K, N, bits, group_size, s_lo, s_hi), seed)
+
+
+def x_batch(M: int, K: int, seed: int) -> np.ndarray:
+    """A fresh fp16 ``(M, K)`` activation block ~ N(0, 1)."""
+    rng = np.random.default_rng(seed)
+    return np.ascontiguousarray(rng.standard_normal((M, K)).astype(np.float16))
