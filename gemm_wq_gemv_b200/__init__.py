@@ -1,0 +1,177 @@
+"""Python binding of ``libwq.so`` (the C ABI declared in ``include/wq.h``).
+
+Argument marshalling only: every step of the product runs in the library's
+sm_100a kernels.  Tensors must already live on the current CUDA device; calls
+are enqueued on ``torch.cuda.current_stream()``.  There is no CPU path: if the
+library is missing or the device is not an sm_100 GPU, the calls raise.
+
+Entry points (same names as the C ABI, without the ``wq_`` prefix):
+
+* ``pack_kmajor(codes_kn, bits) -> (w_q, w_lo)``
+* ``unpack_kmajor(w_q, w_lo, K, bits) -> codes_kn``
+* ``gemv(x, w_q, w_lo, scales, zeros, bits, group_size, out=None, pdl=False) -> y``
+* ``gemm(x, w_q, w_lo, scales, zeros, bits, group_size, out=None, pdl=False) -> y``
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+_PKG = Path(__file__).resolve().parent
+LIB_PATH = _PKG / "libwq.so"
+
+STATUS = {
+    0: "WQ_OK",
+    1: "WQ_ERR_INVALID_ARG",
+    2: "WQ_ERR_UNSUPPORTED",
+    3: "WQ_ERR_ALIGNMENT",
+    4: "WQ_ERR_CODE_RANGE",
+    5: "WQ_ERR_TIMEOUT",
+    6: "WQ_ERR_CUDA",
+}
+WQ_FLAG_PDL = 1
+
+_lib = None
+
+
+class WQError(RuntimeError):
+    """A call into libwq.so returned a status other than WQ_OK."""
+
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        self.name = STATUS.get(status, f"status {status}")
+        super().__init__(f"{fn}: {self.name} ({describe(status)})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libwq.so`` (built in-tree by ``python -m gemm_wq_gemv_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not LIB_PATH.exists():
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m gemm_wq_gemv_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(str(LIB_PATH))
+        p, i, u = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint
+        L.wq_abi_version.restype = i
+        L.wq_status_string.argtypes = [i]
+        L.wq_status_string.restype = ctypes.c_char_p
+        L.wq_pack_kmajor.argtypes = [p, i, i, i, p, p, p, p]
+        L.wq_unpack_kmajor.argtypes = [p, p, i, i, i, p, p]
+        L.wq_gemv.argtypes = [p, p, p, p, p, p, i, i, i, i, i, u, p]
+        L.wq_gemm.argtypes = [p, p, p, p, p, p, i, i, i, i, i, u, p]
+        L.wq_device_status.argtypes = [i]
+        for f in ("wq_pack_kmajor", "wq_unpack_kmajor", "wq_gemv", "wq_gemm", "wq_device_status"):
+            getattr(L, f).restype = i
+        _lib = L
+    return _lib
+
+
+def describe(status: int) -> str:
+    return lib().wq_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise WQError(fn, status)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream():
+    torch = _torch()
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, dtype, name, ndim=2):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
+
+
+def words_shape(K: int, N: int, bits: int):
+    """Shapes of the packed planes for a (K, N) code matrix: (w_q, w_lo or None)."""
+    if bits == 3:
+        return (K // 16, N), (K // 32, N)
+    return (K // (32 // bits), N), None
+
+
+def pack_kmajor(codes_kn, bits: int, check_range: bool = True):
+    """(K, N) uint8 codes -> (w_q, w_lo) int32 words (w_lo is None unless bits == 3).
+
+    With ``check_range`` the call counts codes that do not fit ``bits`` bits on
+    the device, waits for the stream, and raises WQ_ERR_CODE_RANGE if any.
+    """
+    torch = _torch()
+    _need(codes_kn, torch.uint8, "codes_kn")
+    K, N = codes_kn.shape
+    hs, ls = words_shape(K, N, bits)
+    dev = codes_kn.device
+    w_q = torch.empty(hs, dtype=torch.int32, device=dev)
+    w_lo = torch.empty(ls, dtype=torch.int32, device=dev) if ls else None
+    bad = torch.zeros(1, dtype=torch.int32, device=dev) if check_range else None
+    _check("wq_pack_kmajor", lib().wq_pack_kmajor(_ptr(codes_kn), K, N, bits, _ptr(w_q),
+                                                  _ptr(w_lo), _ptr(bad), _stream()))
+    if check_range and int(bad.item()) != 0:
+        raise WQError("wq_pack_kmajor", 4)
+    return w_q, w_lo
+
+
+def unpack_kmajor(w_q, w_lo, K: int, bits: int):
+    torch = _torch()
+    _need(w_q, torch.int32, "w_q")
+    if w_lo is not None:
+        _need(w_lo, torch.int32, "w_lo")
+    N = w_q.shape[1]
+    out = torch.empty((K, N), dtype=torch.uint8, device=w_q.device)
+    _check("wq_unpack_kmajor", lib().wq_unpack_kmajor(_ptr(w_q), _ptr(w_lo), K, N, bits,
+                                                      _ptr(out), _stream()))
+    return out
+
+
+def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl):
+    torch = _torch()
+    _need(x, torch.float16, "x")
+    _need(w_q, torch.int32, "w_q")
+    if w_lo is not None:
+        _need(w_lo, torch.int32, "w_lo")
+    _need(scales, torch.float16, "scales")
+    _need(zeros, torch.float16, "zeros")
+    M, K = x.shape
+    N = w_q.shape[1]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    else:
+        _need(out, torch.float16, "out")
+    flags = WQ_FLAG_PDL if pdl else 0
+    st = getattr(lib(), fn)(_ptr(x), _ptr(w_q), _ptr(w_lo), _ptr(scales), _ptr(zeros), _ptr(out),
+                            M, K, N, bits, group_size, flags, _stream())
+    _check(fn, st)
+    return out
+
+
+def gemv(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl: bool = False):
+    """y (M, N) fp16 = x (M, K) @ dequant(w_q), 1 <= M <= 16 (``wq_gemv``)."""
+    return _product("wq_gemv", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl)
+
+
+def gemm(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl: bool = False):
+    """y (M, N) fp16 = x (M, K) @ dequant(w_q), any M >= 1 (``wq_gemm``)."""
+    return _product("wq_gemm", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl)
+
+
+def device_status(reset: bool = False) -> int:
+    """``wq_device_status``: 0, or 5 (WQ_ERR_TIMEOUT) if a kernel gave up a bounded wait."""
+    return int(lib().wq_device_status(1 if reset else 0))

@@ -1,0 +1,139 @@
+// wq_abi.cu -- the C entry points of libwq.so: argument checks and dispatch.
+//
+// Every rule checked here is stated next to the entry point in include/wq.h.
+// Nothing is launched unless every check passes.
+#include <cuda_runtime.h>
+
+#include "wq_internal.h"
+
+namespace {
+
+bool supported_bits(int b) { return b == 1 || b == 2 || b == 3 || b == 4 || b == 8; }
+
+// Rows of K that one word row covers for the shape rules (3-bit: the lo plane's 32).
+int k_quantum(int bits) { return bits == 3 ? 32 : 32 / bits; }
+
+// Codes per word of the main plane (3-bit: the 2-bit plane, 16).
+int main_eps(int bits) { return bits == 3 ? 16 : 32 / bits; }
+
+bool aligned(const void* p, unsigned a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// The library carries sm_100a code only: refuse any other device up front.
+wq_status check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    static int ok[64] = {0};  // 0 unknown, 1 sm_100, 2 other
+    if (dev >= 0 && dev < 64 && ok[dev]) return ok[dev] == 1 ? WQ_OK : WQ_ERR_UNSUPPORTED;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    const bool good = major == 10 && minor == 0;
+    if (dev >= 0 && dev < 64) ok[dev] = good ? 1 : 2;
+    return good ? WQ_OK : WQ_ERR_UNSUPPORTED;
+}
+
+wq_status check_plane_shape(int K, int N, int bits, const void* w_lo, bool need_lo_rule) {
+    if (!supported_bits(bits)) return WQ_ERR_UNSUPPORTED;
+    if (K < 1 || N < 1) return WQ_ERR_INVALID_ARG;
+    if (K % k_quantum(bits) != 0) return WQ_ERR_INVALID_ARG;
+    if ((long long)K * (long long)N > (1ll << 40)) return WQ_ERR_INVALID_ARG;
+    if (need_lo_rule && ((bits == 3) != (w_lo != nullptr))) return WQ_ERR_INVALID_ARG;
+    return WQ_OK;
+}
+
+// Shared checks of wq_gemv / wq_gemm; resolves G.
+wq_status check_product(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
+                        const uint16_t* s, const uint16_t* z, const uint16_t* y, int M, int K,
+                        int N, int bits, int group_size, int& G) {
+    wq_status st = check_plane_shape(K, N, bits, w_lo, true);
+    if (st != WQ_OK) return st;
+    if (M < 1) return WQ_ERR_INVALID_ARG;
+    if (!x || !w_q || !s || !z || !y) return WQ_ERR_INVALID_ARG;
+    if (group_size == -1) {
+        G = K;
+    } else {
+        if (group_size < 1 || K % group_size != 0 || group_size % k_quantum(bits) != 0)
+            return WQ_ERR_INVALID_ARG;
+        G = group_size;
+    }
+    if (N % 8 != 0) return WQ_ERR_ALIGNMENT;
+    if (!aligned(x, 16) || !aligned(w_q, 16) || !aligned(s, 16) || !aligned(z, 16) ||
+        !aligned(y, 16) || (w_lo && !aligned(w_lo, 16)))
+        return WQ_ERR_ALIGNMENT;
+    return WQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int wq_abi_version(void) { return WQ_ABI_VERSION; }
+
+const char* wq_status_string(wq_status s) {
+    switch (s) {
+        case WQ_OK: return "ok";
+        case WQ_ERR_INVALID_ARG: return "invalid argument";
+        case WQ_ERR_UNSUPPORTED: return "unsupported bit width, group size or device";
+        case WQ_ERR_ALIGNMENT: return "misaligned pointer or N not a multiple of 8";
+        case WQ_ERR_CODE_RANGE: return "code does not fit in the bit width";
+        case WQ_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+        case WQ_ERR_CUDA: return "CUDA runtime error";
+    }
+    return "unknown status";
+}
+
+wq_status wq_pack_kmajor(const uint8_t* codes_kn, int K, int N, int bits, uint32_t* w_q,
+                         uint32_t* w_lo, uint32_t* bad_count, void* stream) {
+    wq_status st = check_plane_shape(K, N, bits, w_lo, true);
+    if (st != WQ_OK) return st;
+    if (!codes_kn || !w_q) return WQ_ERR_INVALID_ARG;
+    if (!aligned(w_q, 4) || (w_lo && !aligned(w_lo, 4)) || (bad_count && !aligned(bad_count, 4)))
+        return WQ_ERR_ALIGNMENT;
+    if ((st = check_device()) != WQ_OK) return st;
+    return wq::launch_pack(codes_kn, K, N, bits, w_q, w_lo, bad_count, (cudaStream_t)stream);
+}
+
+wq_status wq_unpack_kmajor(const uint32_t* w_q, const uint32_t* w_lo, int K, int N, int bits,
+                           uint8_t* codes_kn, void* stream) {
+    wq_status st = check_plane_shape(K, N, bits, w_lo, true);
+    if (st != WQ_OK) return st;
+    if (!codes_kn || !w_q) return WQ_ERR_INVALID_ARG;
+    if (!aligned(w_q, 4) || (w_lo && !aligned(w_lo, 4))) return WQ_ERR_ALIGNMENT;
+    if ((st = check_device()) != WQ_OK) return st;
+    return wq::launch_unpack(w_q, w_lo, K, N, bits, codes_kn, (cudaStream_t)stream);
+}
+
+wq_status wq_gemv(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
+                  const uint16_t* scales, const uint16_t* zeros, uint16_t* y, int M, int K, int N,
+                  int bits, int group_size, unsigned flags, void* stream) {
+    int G = 0;
+    wq_status st = check_product(x, w_q, w_lo, scales, zeros, y, M, K, N, bits, group_size, G);
+    if (st != WQ_OK) return st;
+    if (M > 16) return WQ_ERR_INVALID_ARG;
+    if (G != K && G % (4 * main_eps(bits)) != 0) return WQ_ERR_UNSUPPORTED;
+    if ((st = check_device()) != WQ_OK) return st;
+    wq::Problem p{x, w_q, w_lo, scales, zeros, y, M, K, N, bits, G, flags};
+    return wq::launch_gemv(p, (cudaStream_t)stream);
+}
+
+wq_status wq_gemm(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
+                  const uint16_t* scales, const uint16_t* zeros, uint16_t* y, int M, int K, int N,
+                  int bits, int group_size, unsigned flags, void* stream) {
+    int G = 0;
+    wq_status st = check_product(x, w_q, w_lo, scales, zeros, y, M, K, N, bits, group_size, G);
+    if (st != WQ_OK) return st;
+    if (K % 64 != 0) return WQ_ERR_INVALID_ARG;
+    if ((st = check_device()) != WQ_OK) return st;
+    wq::Problem p{x, w_q, w_lo, scales, zeros, y, M, K, N, bits, G, flags};
+    return wq::launch_gemm(p, (cudaStream_t)stream);
+}
+
+wq_status wq_device_status(int reset) { return wq::gemm_device_status(reset); }
+
+}  // extern "C"

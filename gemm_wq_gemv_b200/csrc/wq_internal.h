@@ -1,0 +1,35 @@
+// wq_internal.h -- declarations shared by the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/wq.h"
+
+namespace wq {
+
+// Problem description handed from the ABI layer to a launcher (already validated).
+struct Problem {
+    const uint16_t* x;
+    const uint32_t* w_q;
+    const uint32_t* w_lo;
+    const uint16_t* scales;
+    const uint16_t* zeros;
+    uint16_t* y;
+    int M, K, N, bits, G;  // G resolved: group_size == -1 -> K
+    unsigned flags;
+};
+
+wq_status launch_pack(const uint8_t* codes, int K, int N, int bits, uint32_t* w_q, uint32_t* w_lo,
+                      uint32_t* bad_count, cudaStream_t s);
+wq_status launch_unpack(const uint32_t* w_q, const uint32_t* w_lo, int K, int N, int bits,
+                        uint8_t* codes, cudaStream_t s);
+wq_status launch_gemv(const Problem& p, cudaStream_t s);
+wq_status launch_gemm(const Problem& p, cudaStream_t s);
+
+// Device status words (one per kernel file), read and optionally cleared.
+wq_status gemm_device_status(int reset);
+
+inline wq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA; }
+
+}  // namespace wq

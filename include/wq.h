@@ -1,0 +1,143 @@
+/*
+ * wq.h -- C ABI of libwq.so: the weight-only quantized matrix product
+ *         y = x @ dequant(W_q) on an sm_100a GPU.
+ *
+ * Data format (dashq_kernel.py, module docstring, `_pack_kmajor`,
+ * `TritonQuantLinear.__init__`; "GPTQModel-Compatible Triton Kernel" README,
+ * sections "Quantization Format" and "Group Quantization"):
+ *
+ *   codes   (K, N)  uint8, row-major: the b-bit code q[k][n] of input row k,
+ *                   output column n, 0 <= q < 2^b.
+ *   w_q     (K/eps, N) uint32 words, row-major (N contiguous), eps = 32 / b:
+ *                   code q[k][n] sits in word w_q[k/eps][n] at bit b*(k%eps).
+ *                   b = 1, 2, 4, 8.
+ *   3-bit:  w_q (K/16, N) holds the 2-bit plane of q >> 1 (16 per word) and
+ *           w_lo (K/32, N) the 1-bit plane of q & 1 (32 per word):
+ *           q = (((w_q[k/16][n] >> 2*(k%16)) & 3) << 1) | ((w_lo[k/32][n] >> (k%32)) & 1).
+ *   scales, zeros  (K/G, N) IEEE binary16 bit patterns, row-major; G is the
+ *                   group size, group_size = -1 meaning G = K (one group per
+ *                   output column).  Row k uses group k / G.
+ *   dequant         w[k][n] = (q[k][n] - z[k/G][n]) * s[k/G][n]
+ *   x  (M, K) binary16 row-major;  y (M, N) binary16 row-major:
+ *                   y[m][n] = sum_k x[m][k] * w[k][n], accumulated in fp32
+ *                   and rounded to nearest even once at the end.
+ *
+ * Words are uint32 bit patterns: a code in the top bits makes the int32 view
+ * of a word negative, which changes nothing here.
+ *
+ * Conventions shared by every entry point:
+ *   - All array pointers are DEVICE pointers owned by the caller.  The library
+ *     never allocates or frees device or host memory.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     enqueue work on it and return once the launch is accepted; results are
+ *     ready when the stream reaches that point.
+ *   - Arguments are validated before anything is launched; a rejected call
+ *     launches nothing and returns the reason.
+ *   - wq_gemv / wq_gemm array pointers must be 16-byte aligned, and packed
+ *     word arrays 4-byte aligned everywhere (WQ_ERR_ALIGNMENT otherwise).
+ *   - N must be a multiple of 8 for wq_gemv and wq_gemm (128-bit word loads
+ *     and 16-byte aligned fp16 rows).
+ *   - The device must be compute capability 10.0 (B200, sm_100a); the
+ *     library holds sm_100a code only.
+ */
+#ifndef WQ_H_
+#define WQ_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define WQ_ABI_VERSION 1
+
+typedef enum {
+    WQ_OK = 0,
+    WQ_ERR_INVALID_ARG = 1,   /* a shape, size or pointer the operation cannot take */
+    WQ_ERR_UNSUPPORTED = 2,   /* bits outside {1,2,3,4,8}, or a device other than sm_100 */
+    WQ_ERR_ALIGNMENT = 3,     /* a pointer not 16-byte aligned, or N not a multiple of 8 */
+    WQ_ERR_CODE_RANGE = 4,    /* a code >= 2^bits was found (reported by the bindings) */
+    WQ_ERR_TIMEOUT = 5,       /* a kernel gave up a bounded wait (see wq_device_status) */
+    WQ_ERR_CUDA = 6           /* the CUDA runtime refused a launch or query */
+} wq_status;
+
+/*
+ * Launch flags for wq_gemv / wq_gemm.
+ * WQ_FLAG_PDL: launch as a programmatic dependent of the previous kernel on
+ *   the stream.  The kernel may start while that kernel still runs: it streams
+ *   w_q, w_lo, scales and zeros at once and reads x only after the previous
+ *   kernel has completed.  So with this flag the previous kernel on the stream
+ *   must not write w_q, w_lo, scales or zeros.  Decode loops over many layers
+ *   use it to overlap one product's weight reads with the previous product.
+ */
+#define WQ_FLAG_PDL 1u
+
+/* Version of this ABI (WQ_ABI_VERSION). */
+int wq_abi_version(void);
+
+/* A static, human-readable name for a status code.  Never NULL. */
+const char* wq_status_string(wq_status s);
+
+/*
+ * Pack codes into K-major words (dashq_kernel.py `_pack_kmajor`; 3-bit planes
+ * as in `TritonQuantLinear.__init__`).
+ *   codes_kn  (K, N) uint8 device array.
+ *   w_q       (K/eps, N) uint32 output (3-bit: (K/16, N) hi plane).
+ *   w_lo      3-bit: (K/32, N) uint32 output lo plane; must be NULL otherwise.
+ *   bad_count optional uint32 device counter, may be NULL.  When given, the
+ *             kernel adds the number of codes >= 2^bits to it (the caller sets
+ *             it to zero first).  Such codes are always masked to `bits` bits,
+ *             so they never spill into a neighbouring field.
+ * Requires K % eps == 0 (3-bit: K % 32 == 0), K >= 1, N >= 1.
+ */
+wq_status wq_pack_kmajor(const uint8_t* codes_kn, int K, int N, int bits,
+                         uint32_t* w_q, uint32_t* w_lo, uint32_t* bad_count, void* stream);
+
+/*
+ * Inverse of wq_pack_kmajor (dashq_kernel.py `_unpack_kmajor`; 3-bit
+ * recombination as in `dequantize_weight`): writes codes_kn (K, N) uint8.
+ * Same shape rules as packing; w_lo required iff bits == 3.
+ */
+wq_status wq_unpack_kmajor(const uint32_t* w_q, const uint32_t* w_lo, int K, int N, int bits,
+                           uint8_t* codes_kn, void* stream);
+
+/*
+ * Decode-time product for a few rows of x: 1 <= M <= 16
+ * (dashq_kernel.py `_dashq_gemv_kernel` and `forward` for one token; here any
+ * M up to 16 reads W_q once).  x (M, K), y (M, N), binary16.
+ * group_size: -1, or a positive divisor of K that is a multiple of 4 * eps
+ * (1-bit: 128, 2-bit: 64, 3-bit: 64, 4-bit: 32, 8-bit: 16); other group sizes
+ * give WQ_ERR_UNSUPPORTED here (wq_gemm takes them).  Requires K % eps == 0
+ * (3-bit: K % 32 == 0) and N % 8 == 0.
+ * One launch: the split-K partial sums are reduced on chip (thread-block
+ * cluster shared memory); no workspace and no zero-initialised output needed.
+ */
+wq_status wq_gemv(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
+                  const uint16_t* scales, const uint16_t* zeros, uint16_t* y,
+                  int M, int K, int N, int bits, int group_size, unsigned flags, void* stream);
+
+/*
+ * Batched product for any M >= 1 ("GPTQModel-Compatible Triton Kernel"
+ * README, `gptqmodel_quantized_matmul`; dashq_kernel.py `forward`, batched
+ * branch).  Same arguments as wq_gemv.  group_size: -1, or a positive divisor
+ * of K that is a multiple of eps (3-bit: of 32).  Requires K % 64 == 0 and
+ * N % 8 == 0.
+ * Packed tiles are dequantised to fp16 in shared memory and multiplied on the
+ * tensor cores (tcgen05, fp32 accumulators in tensor memory).
+ */
+wq_status wq_gemm(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
+                  const uint16_t* scales, const uint16_t* zeros, uint16_t* y,
+                  int M, int K, int N, int bits, int group_size, unsigned flags, void* stream);
+
+/*
+ * Device-side status of the current device: WQ_OK, or WQ_ERR_TIMEOUT when a
+ * kernel on this device gave up a bounded wait since the last reset (its
+ * output is then incomplete).  Synchronises the device.  reset != 0 clears it.
+ */
+wq_status wq_device_status(int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WQ_H_ */

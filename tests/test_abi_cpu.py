@@ -1,0 +1,89 @@
+"""libwq.so on a machine without a GPU: it loads, exports every declared entry
+point, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+def declared_functions():
+    text = (ROOT / "include" / "wq.h").read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(wq_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for n in ("wq_pack_kmajor", "wq_unpack_kmajor", "wq_gemv", "wq_gemm", "wq_status_string",
+              "wq_abi_version", "wq_device_status"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(libwq):
+    L = libwq.lib()
+    for n in declared_functions():
+        assert hasattr(L, n), f"{n} declared in include/wq.h but not exported"
+
+
+def test_version_and_strings(libwq):
+    L = libwq.lib()
+    assert L.wq_abi_version() == 1
+    for s in range(7):
+        assert L.wq_status_string(s)
+    assert L.wq_status_string(99) == b"unknown status"
+
+
+P = 0x10000  # a 16-byte aligned fake device address: never dereferenced on the host path
+
+
+def gemv(L, fn="wq_gemv", x=P, wq=P, wlo=None, s=P, z=P, y=P, M=1, K=512, N=256, bits=4, G=128,
+         flags=0):
+    return getattr(L, fn)(x, wq, wlo, s, z, y, M, K, N, bits, G, flags, None)
+
+
+@pytest.mark.parametrize("fn", ["wq_gemv", "wq_gemm"])
+def test_product_argument_checks(libwq, fn):
+    L = libwq.lib()
+    INV, UNS, ALI, CUDA = 1, 2, 3, 6
+    assert gemv(L, fn, bits=5) == UNS
+    assert gemv(L, fn, bits=0) == UNS
+    assert gemv(L, fn, M=0) == INV
+    assert gemv(L, fn, K=0) == INV
+    assert gemv(L, fn, N=0) == INV
+    assert gemv(L, fn, K=500, G=-1) == INV                # K not a multiple of 8 (4-bit)
+    assert gemv(L, fn, G=100) == INV                      # does not divide K
+    assert gemv(L, fn, G=0) == INV
+    assert gemv(L, fn, bits=3, K=512, G=128) == INV       # 3-bit needs w_lo
+    assert gemv(L, fn, bits=4, wlo=P) == INV              # w_lo only for 3-bit
+    assert gemv(L, fn, bits=3, K=528, wlo=P, G=-1) == INV  # 3-bit needs K % 32 == 0
+    assert gemv(L, fn, x=None) == INV
+    assert gemv(L, fn, y=None) == INV
+    assert gemv(L, fn, N=252) == ALI                      # N % 8
+    assert gemv(L, fn, x=P + 8) == ALI
+    assert gemv(L, fn, wq=P + 4) == ALI
+    # valid arguments: the host checks pass and the call reaches CUDA, which has no device here
+    import torch
+    if not torch.cuda.is_available():
+        assert gemv(L, fn) == CUDA
+        assert gemv(L, fn, bits=3, wlo=P, K=512, G=128) == CUDA
+
+
+def test_gemv_specific_limits(libwq):
+    L = libwq.lib()
+    assert gemv(L, "wq_gemv", M=17) == 1
+    assert gemv(L, "wq_gemv", bits=4, G=16, K=512) == 2   # group not a multiple of 4*eps
+    assert gemv(L, "wq_gemv", bits=1, G=64, K=512) == 2
+    assert gemv(L, "wq_gemm", K=544, G=-1) == 1           # gemm needs K % 64
+
+
+def test_pack_argument_checks(libwq):
+    L = libwq.lib()
+    assert L.wq_pack_kmajor(P, 12, 4, 4, P, None, None, None) == 1   # K % 8
+    assert L.wq_pack_kmajor(P, 32, 4, 6, P, None, None, None) == 2
+    assert L.wq_pack_kmajor(P, 32, 4, 3, P, None, None, None) == 1   # 3-bit needs w_lo
+    assert L.wq_pack_kmajor(None, 32, 4, 4, P, None, None, None) == 1
+    assert L.wq_pack_kmajor(P, 32, 4, 4, P + 2, None, None, None) == 3
+    assert L.wq_unpack_kmajor(P, P, 32, 4, 4, P, None) == 1          # w_lo with 4-bit

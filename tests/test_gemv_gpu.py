@@ -1,0 +1,136 @@
+"""wq_gemv (M <= 16) against the fp64 oracle, element by element."""
+import numpy as np
+import pytest
+
+import wq_inputs
+from gpu_cases import oracle_product, to_dev
+from parity import check_product
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gemv(libwq, d, bits, G, **kw):
+    w_q, w_lo = libwq.pack_kmajor(d["codes"], bits)
+    y = libwq.gemv(d["x"], w_q, w_lo, d["scales"], d["zeros"], bits, G, **kw)
+    return y.cpu().numpy()
+
+
+FULL = ["tiny_gemv", "decode_gemv_m1", "decode_gemv_m4", "decode_gemv_m16", "gemv_3bit",
+        "sweep_1bit", "sweep_2bit", "sweep_8bit", "sweep_8bit_perchannel"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_workloads_full(cuda, libwq, orc, name):
+    """Every output of each GEMV workload, at full size, in the bench's launch configuration."""
+    case = wq_inputs.draw(wq_inputs.WORKLOADS[name], seed=0)
+    d = to_dev(case, cuda)
+    y = run_gemv(libwq, d, case.wl.bits, case.wl.group_size)
+    y_ref, b = oracle_product(orc, case)
+    check_product(y, y_ref, b, name)
+
+
+SHAPES = [
+    # M, K, N, bits, G
+    (1, 32, 8, 4, 32),        # one quad, one ragged column block
+    (3, 40, 16, 4, -1),       # ragged last quad (5 word rows)
+    (1, 512, 264, 4, 64),
+    (2, 1024, 40, 8, 16),
+    (5, 2048, 72, 8, -1),
+    (8, 512, 128, 2, 64),
+    (9, 768, 96, 2, 256),
+    (16, 1024, 136, 1, 128),
+    (7, 4096, 64, 1, -1),
+    (1, 1024, 200, 3, 64),
+    (12, 2048, 56, 3, 128),
+    (16, 3072, 48, 3, -1),
+    (4, 8192, 16, 4, 128),    # long K per column block: many quads per warp
+    (16, 256, 4096, 4, 128),  # wide N, short K
+]
+
+
+@pytest.mark.parametrize("M,K,N,bits,G", SHAPES)
+def test_small_shapes(cuda, libwq, orc, M, K, N, bits, G):
+    case = wq_inputs.custom(M, K, N, bits, G, seed=M * 7 + K + N + bits)
+    d = to_dev(case, cuda)
+    y = run_gemv(libwq, d, bits, G)
+    y_ref, b = oracle_product(orc, case)
+    check_product(y, y_ref, b, f"{(M, K, N, bits, G)}")
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 8])
+def test_fractional_zero_points(cuda, libwq, orc, bits):
+    """Zero points that are not integers (any fp16 value is allowed)."""
+    import torch
+    K, N, M, G = 1024, 96, 3, (128 if bits in (1, 2, 3) else 64)
+    case = wq_inputs.custom(M, K, N, bits, G, seed=77 + bits)
+    rng = np.random.default_rng(bits)
+    case.zeros = rng.uniform(-0.5, (1 << bits) - 0.5, size=case.zeros.shape).astype(np.float16)
+    d = to_dev(case, cuda)
+    d["zeros"] = torch.from_numpy(case.zeros).to(cuda)
+    y = run_gemv(libwq, d, bits, G)
+    y_ref, b = oracle_product(orc, case)
+    check_product(y, y_ref, b, f"fractional z, {bits}-bit")
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("M", [1, 16])
+def test_q_equals_z_gives_zero(cuda, libwq, bits, M):
+    import torch
+    K, N = 512, 64
+    G = 128
+    case = wq_inputs.custom(M, K, N, bits, G, seed=5)
+    zq = np.random.default_rng(9).integers(0, 1 << bits, size=(K // G, N))
+    codes = np.repeat(zq, G, axis=0).astype(np.uint8)
+    d = to_dev(case, cuda)
+    d["codes"] = torch.from_numpy(codes).to(cuda)
+    d["zeros"] = torch.from_numpy(zq.astype(np.float16)).to(cuda)
+    y = run_gemv(libwq, d, bits, G)
+    assert np.all(y.astype(np.float64) == 0.0)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 8])
+def test_one_hot_rows_are_exact(cuda, libwq, orc, bits):
+    """x = e_k gives fp16(w[k]) exactly, for 16 rows k at once."""
+    import torch
+    K, N, G = 512, 64, 128
+    case = wq_inputs.custom(16, K, N, bits, G, seed=31)
+    ks = np.random.default_rng(3).choice(K, 16, replace=False)
+    x = np.zeros((16, K), np.float16)
+    x[np.arange(16), ks] = 1.0
+    d = to_dev(case, cuda)
+    d["x"] = torch.from_numpy(x).to(cuda)
+    y = run_gemv(libwq, d, bits, G)
+    q = case.codes.astype(np.float64)
+    g = ks // G
+    w = (q[ks] - case.zeros[g].astype(np.float64)) * case.scales[g].astype(np.float64)
+    assert np.array_equal(y, w.astype(np.float16))
+
+
+def test_pdl_flag_same_result(cuda, libwq):
+    case = wq_inputs.draw(wq_inputs.WORKLOADS["tiny_gemv"], seed=0)
+    d = to_dev(case, cuda)
+    a = run_gemv(libwq, d, 4, 128)
+    b = run_gemv(libwq, d, 4, 128, pdl=True)
+    assert np.array_equal(a, b)
+
+
+def test_deterministic(cuda, libwq):
+    case = wq_inputs.draw(wq_inputs.WORKLOADS["decode_gemv_m4"], seed=1)
+    d = to_dev(case, cuda)
+    a = run_gemv(libwq, d, 4, 128)
+    b = run_gemv(libwq, d, 4, 128)
+    assert np.array_equal(a, b)
+
+
+def test_rejected_calls(cuda, libwq):
+    import torch
+    case = wq_inputs.draw(wq_inputs.WORKLOADS["tiny_gemv"], seed=0)
+    d = to_dev(case, cuda)
+    w_q, _ = libwq.pack_kmajor(d["codes"], 4)
+    x17 = torch.zeros((17, 512), dtype=torch.float16, device=cuda)
+    with pytest.raises(libwq.WQError) as e:
+        libwq.gemv(x17, w_q, None, d["scales"], d["zeros"], 4, 128)
+    assert e.value.status == 1
+    with pytest.raises(libwq.WQError) as e:
+        libwq.gemv(d["x"], w_q, None, d["scales"], d["zeros"], 4, 16)
+    assert e.value.status == 2
