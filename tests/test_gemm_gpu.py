@@ -1,0 +1,124 @@
+"""wq_gemm (tcgen05 tensor cores) against the fp64 oracle, element by element."""
+import numpy as np
+import pytest
+
+import wq_inputs
+from gpu_cases import oracle_product, to_dev
+from parity import check_product
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gemm(libwq, d, bits, G, **kw):
+    w_q, w_lo = libwq.pack_kmajor(d["codes"], bits)
+    y = libwq.gemm(d["x"], w_q, w_lo, d["scales"], d["zeros"], bits, G, **kw)
+    return y.cpu().numpy()
+
+
+def test_prefill_workload_full(cuda, libwq, orc):
+    """Every output of the M=512 x K=4096 x N=2048 4-bit product, in the bench's launch configuration."""
+    case = wq_inputs.draw(wq_inputs.WORKLOADS["prefill_gemm"], seed=0)
+    d = to_dev(case, cuda)
+    y = run_gemm(libwq, d, 4, 128)
+    y_ref, b = oracle_product(orc, case)
+    check_product(y, y_ref, b, "prefill_gemm")
+
+
+@pytest.mark.parametrize("name", ["tiny_gemv", "decode_gemv_m16", "gemv_3bit", "sweep_1bit",
+                                  "sweep_8bit_perchannel"])
+def test_gemv_workloads_through_gemm(cuda, libwq, orc, name):
+    """The GEMV workloads also go through the batched path (any M)."""
+    case = wq_inputs.draw(wq_inputs.WORKLOADS[name], seed=0)
+    d = to_dev(case, cuda)
+    y = run_gemm(libwq, d, case.wl.bits, case.wl.group_size)
+    y_ref, b = oracle_product(orc, case)
+    check_product(y, y_ref, b, name)
+
+
+SHAPES = [
+    # M, K, N, bits, G
+    (1, 64, 8, 4, 64),          # one k block, one ragged column tile
+    (5, 128, 136, 4, 32),       # two groups per k block
+    (16, 4096, 128, 4, 128),    # one tile, split over an 8-CTA cluster
+    (33, 512, 264, 8, 16),      # 4 groups per k block, ragged tiles
+    (100, 1024, 256, 2, 64),
+    (128, 256, 512, 1, 128),
+    (200, 2048, 384, 3, 128),
+    (256, 192, 1024, 3, -1),
+    (300, 512, 128, 4, 64),     # two balanced token tiles of 160
+    (512, 128, 8192, 8, 128),   # many tiles, no split
+    (64, 8192, 136, 1, -1),
+    (7, 4096, 2048, 2, 32),
+]
+
+
+@pytest.mark.parametrize("M,K,N,bits,G", SHAPES)
+def test_shapes(cuda, libwq, orc, M, K, N, bits, G):
+    case = wq_inputs.custom(M, K, N, bits, G, seed=3 * M + K + N + bits)
+    d = to_dev(case, cuda)
+    y = run_gemm(libwq, d, bits, G)
+    y_ref, b = oracle_product(orc, case)
+    check_product(y, y_ref, b, f"{(M, K, N, bits, G)}")
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 8])
+def test_fractional_zero_points(cuda, libwq, orc, bits):
+    import torch
+    M, K, N, G = 48, 1024, 128, 64
+    case = wq_inputs.custom(M, K, N, bits, G, seed=40 + bits)
+    rng = np.random.default_rng(bits)
+    case.zeros = rng.uniform(-0.5, (1 << bits) - 0.5, size=case.zeros.shape).astype(np.float16)
+    d = to_dev(case, cuda)
+    d["zeros"] = torch.from_numpy(case.zeros).to(cuda)
+    y = run_gemm(libwq, d, bits, G)
+    y_ref, b = oracle_product(orc, case)
+    check_product(y, y_ref, b, f"fractional z, {bits}-bit")
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 8])
+def test_q_equals_z_gives_zero(cuda, libwq, bits):
+    import torch
+    M, K, N, G = 64, 512, 128, 128
+    case = wq_inputs.custom(M, K, N, bits, G, seed=8)
+    zq = np.random.default_rng(2).integers(0, 1 << bits, size=(K // G, N))
+    d = to_dev(case, cuda)
+    d["codes"] = torch.from_numpy(np.repeat(zq, G, axis=0).astype(np.uint8)).to(cuda)
+    d["zeros"] = torch.from_numpy(zq.astype(np.float16)).to(cuda)
+    y = run_gemm(libwq, d, bits, G)
+    assert np.all(y.astype(np.float64) == 0.0)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 8])
+def test_one_hot_rows_are_exact(cuda, libwq, bits):
+    """x = e_k for 64 rows k gives fp16(w[k]) exactly."""
+    import torch
+    K, N, G = 1024, 256, 128
+    case = wq_inputs.custom(64, K, N, bits, G, seed=13)
+    ks = np.random.default_rng(4).choice(K, 64, replace=False)
+    x = np.zeros((64, K), np.float16)
+    x[np.arange(64), ks] = 1.0
+    d = to_dev(case, cuda)
+    d["x"] = torch.from_numpy(x).to(cuda)
+    y = run_gemm(libwq, d, bits, G)
+    g = ks // G
+    w = (case.codes[ks].astype(np.float64) - case.zeros[g].astype(np.float64)) * case.scales[g].astype(np.float64)
+    assert np.array_equal(y, w.astype(np.float16))
+
+
+def test_deterministic_and_status(cuda, libwq):
+    case = wq_inputs.draw(wq_inputs.WORKLOADS["prefill_gemm"], seed=1)
+    d = to_dev(case, cuda)
+    a = run_gemm(libwq, d, 4, 128)
+    b = run_gemm(libwq, d, 4, 128, pdl=True)
+    assert np.array_equal(a, b)
+    assert libwq.device_status() == 0
+
+
+def test_rejected_calls(cuda, libwq):
+    import torch
+    case = wq_inputs.custom(4, 96, 64, 4, 32, seed=1)
+    d = to_dev(case, cuda)
+    w_q, _ = libwq.pack_kmajor(d["codes"], 4)
+    with pytest.raises(libwq.WQError) as e:   # K % 64 != 0
+        libwq.gemm(d["x"], w_q, None, d["scales"], d["zeros"], 4, 32)
+    assert e.value.status == 1
