@@ -1,0 +1,432 @@
+#!/usr/bin/env python
+"""Benchmark of the weight-only quantized product on B200.
+
+Headline workload: the decode GEMV y (1 x 4096) = x (1 x 4096) @ dequant(W_q),
+W_q 4-bit K-major words, group 128, fp16 scales and zero points.  One *step*
+is one decode pass over a stack of L distinct weight sets of that shape (each
+with its own x), launched back to back as programmatic dependents and replayed
+as one CUDA graph.  The stack's weights exceed twice the L2 size, so every
+launch reads its words from HBM.  ``value`` is the algorithmic HBM bytes of
+the products (packed words + s + z + x + y) per second, whole job.
+
+Also measured on the same box, in the same run:
+* ``gemm``: the batched product M=512, K=4096, N=2048 (4-bit, group 128) in TFLOP/s;
+* ``workloads``: every synthetic workload (bit-width sweep, 3-bit planes, M=4/16);
+* ``e2e``: the headline metric through the Python API with host buffers (x copied
+  in and y copied out every step);
+* ``cpu_baseline``: the CPU oracle (plain C, fp64) on a bounded sample.
+
+``--impl reference`` times the CPU oracle as the reference arm.
+``--gpus N`` (under torchrun) runs N independent replicas, one per GPU.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import wq_inputs  # noqa: E402
+
+HEADLINE = "decode_gemv_m1"
+GEMM_WL = "prefill_gemm"
+METRIC = "packed-int GEMV HBM GB/s and % of peak at M=1; wq_gemm TFLOPS at M=512"
+FALLBACK_HBM, FALLBACK_TF = 6650.0, 1590.0
+
+
+def algo_bytes(wl) -> int:
+    """Algorithmic bytes of one product: packed words, s, z, x and y."""
+    return wl.K * wl.N * wl.bits // 8 + 2 * 2 * wl.groups * wl.N + 2 * wl.M * wl.K + 2 * wl.M * wl.N
+
+
+def algo_flops(wl) -> int:
+    return 2 * wl.M * wl.N * wl.K
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0)), "measured"
+    return FALLBACK_HBM, FALLBACK_TF, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks (NVML)
+class ClockSampler:
+    """Samples SM clock and clock-event reasons of one GPU on a thread (NVML)."""
+
+    NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+             0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+             0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            self.reasons |= nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nv:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self.nv and self._t:
+            self._stop.set()
+            self._t.join()
+            self._sample()
+
+    def report(self):
+        if not self.nv or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for b, n in self.NAMES.items() if self.reasons & b and b != 0x1]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ helpers
+def src_digest() -> str:
+    h = hashlib.sha1()
+    for f in sorted((ROOT / "gemm_wq_gemv_b200" / "csrc").glob("*")):
+        h.update(f.read_bytes())
+    return h.hexdigest()[:12]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """dram read+write bytes per launch from profiles/ncu_traffic.txt, if taken on this source."""
+    p = ROOT / "profiles" / "ncu_traffic.txt"
+    if not p.exists():
+        return None
+    for line in p.read_text().splitlines():
+        if line.startswith("#") or not line.strip():
+            continue
+        kv = dict(t.split("=", 1) for t in line.split() if "=" in t)
+        if kv.get("kernel") == kernel and kv.get("workload") == workload and kv.get("src") == src_digest():
+            return float(kv["dram_bytes_per_launch"])
+    return None
+
+
+class Stack:
+    """L distinct weight sets of one workload on the device, plus x / y per set."""
+
+    def __init__(self, wq, torch, wl, L, dev, seed0=0):
+        import numpy as np
+        self.wl, self.L = wl, L
+        base = wq_inputs.draw(wl, seed=seed0)
+        codes = torch.from_numpy(base.codes).to(dev)
+        w_q, w_lo = wq.pack_kmajor(codes, wl.bits)
+        s = torch.from_numpy(base.scales).to(dev)
+        z = torch.from_numpy(base.zeros).to(dev)
+        del codes
+        self.sets = []
+        for i in range(L):
+            x = torch.from_numpy(wq_inputs.x_batch(wl.M, wl.K, seed=1000 + i)).to(dev)
+            y = torch.empty((wl.M, wl.N), dtype=torch.float16, device=dev)
+            self.sets.append((x, w_q.clone() if i else w_q, None if w_lo is None else (w_lo.clone() if i else w_lo),
+                              s.clone() if i else s, z.clone() if i else z, y))
+        self.np = np
+
+    def run(self, wq, fn, pdl):
+        wl = self.wl
+        for (x, a, b, s, z, y) in self.sets:
+            fn(x, a, b, s, z, wl.bits, wl.group_size, out=y, pdl=pdl)
+
+
+def time_graph(torch, graph, stream, steps, warmup, barrier=None, sampler=None):
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if sampler:
+        sampler.start()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.stop()
+    if barrier:
+        barrier()
+    return e0.elapsed_time(e1) / 1e3  # seconds
+
+
+def capture(torch, fn):
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        fn()  # first run outside the graph (lazy set-up)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            fn()
+    torch.cuda.synchronize()
+    return g, s
+
+
+def layers_for(wl, L2):
+    """Weight sets per step: enough distinct sets to exceed twice the L2 (at most 1024)."""
+    return min(1024, max(2, int(2 * L2 // algo_bytes(wl)) + 2))
+
+
+def cpu_baseline(seconds: float = 10.0):
+    """The CPU oracle (plain C fp64, OpenMP) on full decode GEMVs, for ~`seconds`."""
+    import oracle
+    wl = wq_inputs.WORKLOADS[HEADLINE]
+    case = wq_inputs.draw(wl, 0)
+    wq_, wlo = oracle.pack(case.codes, wl.bits)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.wq_matmul(case.x, wq_, wlo, case.scales, case.zeros, wl.bits, wl.group_size)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or reps >= 2000:
+            break
+    return {"value": round(algo_bytes(wl) * reps / el / 1e9, 3), "unit": "GB/s", "cores": oracle.threads(),
+            "kind": "oracle",
+            "sample": f"{reps} full decode GEMVs (M=1, K=N=4096, 4-bit, g128) in {el:.1f} s, fp64 C"}
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    """The CPU oracle timed as the reference arm, on the headline config and metric."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+    import oracle
+    wl = wq_inputs.WORKLOADS[HEADLINE]
+    case = wq_inputs.draw(wl, 0)
+    wq_, wlo = oracle.pack(case.codes, wl.bits)
+    # one step = the product for a slice of 256 output columns (1/16 of the GEMV)
+    cols = 256
+    rng = np.random.default_rng(0)
+    def step(i):
+        n0 = (i * cols) % wl.N
+        ms = np.zeros(cols, np.int32)
+        ns = np.arange(n0, n0 + cols, dtype=np.int32)
+        oracle.wq_matmul_sampled(case.x, wq_, wlo, case.scales, case.zeros, wl.bits, wl.group_size, ms, ns)
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    el = time.perf_counter() - t0
+    frac = cols / wl.N
+    bytes_step = algo_bytes(wl) * frac
+    v = bytes_step * args.steps / el / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "decode GEMV M=1 K=4096 N=4096 4-bit g128 (fp16 x, s, z)",
+                       "parallelism": "cpu oracle"},
+            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
+                             "sample": f"each step: {cols} of the {wl.N} output columns of the decode GEMV, "
+                                       "each output computed on its own from the packed words (fp64 C)"},
+            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["wq", "reference"], default="wq")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the per-workload table")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if dist:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if not dist:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    from gemm_wq_gemv_b200 import build as wq_build
+    wq_build.build()
+    import gemm_wq_gemv_b200 as wq
+
+    props = torch.cuda.get_device_properties(dev)
+    L2 = props.L2_cache_size
+    hbm_peak, tf_peak, tf_sust, peak_kind = peaks()
+
+    # ---- headline: decode GEMV stack
+    wl = wq_inputs.WORKLOADS[HEADLINE]
+    L = layers_for(wl, L2)
+    stack = Stack(wq, torch, wl, L, dev)
+    g, s = capture(torch, lambda: stack.run(wq, wq.gemv, True))
+    sampler = ClockSampler(local)
+    el = time_graph(torch, g, s, args.steps, args.warmup, barrier, sampler)
+    el = max_over_ranks(el)
+    bytes_step = algo_bytes(wl) * L
+    value = bytes_step * args.steps * world / el / 1e9
+    per_launch_s = el / (args.steps * L)
+    achieved = algo_bytes(wl) / per_launch_s / 1e9
+    traffic = ncu_traffic("gemv_kernel<4, 1>", HEADLINE)
+
+    # ---- e2e: the same stack through the API with host buffers
+    xs_host = torch.empty((L, wl.M, wl.K), dtype=torch.float16, pin_memory=True)
+    for i, st in enumerate(stack.sets):
+        xs_host[i].copy_(st[0].cpu())
+    ys_host = torch.empty((L, wl.M, wl.N), dtype=torch.float16, pin_memory=True)
+    xs_dev = torch.empty((L, wl.M, wl.K), dtype=torch.float16, device=dev)
+    ys_dev = torch.empty((L, wl.M, wl.N), dtype=torch.float16, device=dev)
+    e2e_steps = max(3, min(args.steps, 200))
+
+    def e2e_step():
+        xs_dev.copy_(xs_host, non_blocking=True)
+        for i, (x, a, b, sc, z, y) in enumerate(stack.sets):
+            wq.gemv(xs_dev[i], a, b, sc, z, wl.bits, wl.group_size, out=ys_dev[i])
+        ys_host.copy_(ys_dev, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    for _ in range(3):
+        e2e_step()
+    barrier()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e2e_el = max_over_ranks(time.perf_counter() - t0)
+    e2e_value = bytes_step * e2e_steps * world / e2e_el / 1e9
+    del stack, g
+
+    # ---- GEMM: M=512 prefill product
+    gwl = wq_inputs.WORKLOADS[GEMM_WL]
+    GL = layers_for(gwl, L2)
+    gstack = Stack(wq, torch, gwl, GL, dev)
+    gg, gs = capture(torch, lambda: gstack.run(wq, wq.gemm, False))
+    gsteps = max(3, min(args.steps, 200))
+    gel = max_over_ranks(time_graph(torch, gg, gs, gsteps, args.warmup, barrier))
+    g_launch_s = gel / (gsteps * GL)
+    g_tflops = algo_flops(gwl) / g_launch_s / 1e12
+    del gstack, gg
+
+    # ---- every workload once (rank-local, for the table)
+    table = []
+    if not args.no_secondary:
+        for name, w in wq_inputs.WORKLOADS.items():
+            fn = wq.gemm if w.M > 16 else wq.gemv
+            n_l = layers_for(w, L2)
+            stk = Stack(wq, torch, w, n_l, dev)
+            gr, st_ = capture(torch, lambda: stk.run(wq, fn, fn is wq.gemv))
+            reps = 20
+            t = time_graph(torch, gr, st_, reps, 3)
+            us = t / (reps * n_l) * 1e6
+            row = {"workload": name, "M": w.M, "K": w.K, "N": w.N, "bits": w.bits, "group": w.group_size,
+                   "kernel": "gemm" if fn is wq.gemm else "gemv", "us": round(us, 3)}
+            if fn is wq.gemm:
+                tfl = algo_flops(w) / (us * 1e-6) / 1e12
+                row.update({"TFLOPS": round(tfl, 1), "frac": round(tfl / tf_peak, 4)})
+            else:
+                gbs = algo_bytes(w) / (us * 1e-6) / 1e9
+                row.update({"GBps": round(gbs, 1), "frac": round(gbs / hbm_peak, 4)})
+            table.append(row)
+            del stk, gr
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(el / args.steps * 1e3, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16xf16->f32 (4-bit codes dequantised to f16)",
+        "data": "synthetic (seeded: x ~ N(0,1), codes U[0,15], s ~ U[0.005,0.02], integer z U[0,15])",
+        "config": {"workload": f"decode GEMV M=1 K=4096 N=4096 4-bit g128, stack of {L} weight sets per step",
+                   "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2: {bytes_step / 1e6:.0f} MB of distinct weights per step "
+                         f"> 2 x {L2 / 1e6:.0f} MB L2",
+                   "launch": "one CUDA graph per step, programmatic dependent launches"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
+                     "algorithmic_bytes_per_launch": algo_bytes(wl), "launch_us": round(per_launch_s * 1e6, 3)},
+        "gemm": {"workload": "M=512 K=4096 N=2048 4-bit g128", "TFLOPS": round(g_tflops, 1),
+                 "us": round(g_launch_s * 1e6, 3),
+                 "roofline": {"bound": "tensor", "achieved": round(g_tflops, 1), "peak": tf_peak, "unit": "TFLOP/s",
+                              "frac": round(g_tflops / tf_peak, 4),
+                              "peak_source": "measured bf16 burst (fp16 nominal ratio 1:1)"},
+                 "l2": f"{GL} rotating input sets ({algo_bytes(gwl) * GL / 1e6:.0f} MB) per graph"},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": L * wl.M * wl.K * 2, "d2h_bytes_per_step": L * wl.M * wl.N * 2,
+                "how": "python API per layer (wq.gemv), x copied in from pinned host memory and y copied "
+                       "back every step; weights resident"},
+        "clocks": sampler.report(),
+        "gpu_launches": args.steps * L * world,
+        "workloads": table,
+        "source": src_digest(),
+    }
+    if rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
