@@ -134,6 +134,11 @@ wq_status wq_gemm(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
     return wq::launch_gemm(p, (cudaStream_t)stream);
 }
 
-wq_status wq_device_status(int reset) { return wq::gemm_device_status(reset); }
+wq_status wq_device_status(int reset) {
+    const wq_status a = wq::gemm_device_status(reset);
+    const wq_status b = wq::gemv_device_status(reset);
+    if (a == WQ_ERR_CUDA || b == WQ_ERR_CUDA) return WQ_ERR_CUDA;
+    return (a != WQ_OK) ? a : b;
+}
 
 }  // extern "C"

@@ -25,8 +25,6 @@
 // Every wait on an mbarrier is bounded; on time-out the kernel records
 // WQ_ERR_TIMEOUT in a device status word, skips its remaining work, still
 // frees its tensor memory and returns.
-#include <cuda.h>
-#include <cudaTypedefs.h>
 
 #include <algorithm>
 
@@ -301,40 +299,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
 }
 
 // ------------------------------------------------------------------------ host
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-        else
-            cudaGetLastError();
-    }
-    return fn;
-}
-
-bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t outer,
-              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {row_bytes};
-    cuuint32_t box[2] = {box_inner, box_outer};
-    cuuint32_t es[2] = {1, 1};
-    CUresult r = fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-int sm_count_dev() {
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n > 0 ? n : 148;
-}
-
 template <int BITS>
 wq_status run(const Problem& pb, cudaStream_t stream) {
     constexpr int EPS = Fmt<BITS>::EPS;
@@ -358,7 +322,7 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     const int ntiles = (pb.N + BMW - 1) / BMW;
     const int tiles = ntiles * mt;
     const int KB = pb.K / BK;
-    const int sms = sm_count_dev();
+    const int sms = sm_count();
     int CS = 1;
     for (int c = 8; c >= 2; c >>= 1) {
         if (KB % c == 0 && KB / c >= 2 && tiles * c <= sms) { CS = c; break; }

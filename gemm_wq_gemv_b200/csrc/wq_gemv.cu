@@ -5,43 +5,46 @@
 // g = k / G, with fp32 accumulation and one fp16 rounding at the end.
 //
 // How (sm_100a):
-//  * Work split.  A CTA owns 32 output columns and a contiguous range of K; the
-//    CTAs of one thread-block cluster split K further and reduce their fp32
-//    partial sums through distributed shared memory (one launch, no workspace,
-//    no atomics).  Inside a CTA, 8 warps split K again; lanes never need a
-//    shuffle because the reduction over k happens inside the MMA.
-//  * Loads.  Lane (g, t) of a warp (g = lane / 4, t = lane % 4) reads one
-//    128-bit vector = 4 adjacent columns of one packed word row; the 8 lanes
-//    with the same t read 128 contiguous bytes.  Loads bypass L1 and are marked
-//    evict-first in L2; each warp keeps PD quads (4 word rows) in flight.
-//  * Dequant.  A code pair (code j, code j + eps/2), which sits in the two
-//    16-bit halves of a word at the same offset, is ORed into the mantissa of
-//    the fp16 constant 1024 (0x6400) with one LOP3, then one exact fp16x2 FMA
-//    scales it down and subtracts 1024 and the integer part of the zero point:
-//    the result q - round(z) is exact in fp16.
-//  * Dot product.  The exact (q - round(z)) values are the A operand of a warp
-//    MMA m16n8k16 (fp16 in, fp32 accumulate) with x as the B operand: rows of
-//    A are 16 output columns, the 16 k-slots are 4 word rows x 4 codes.  The
-//    k-slots are a permutation of k; x is staged in shared memory in the same
-//    permuted order, once per CTA.
-//  * Per group, the fp32 MMA sum is scaled: acc += s * (D - (z - round(z)) * X),
-//    X = sum of the x values of that group slice, so fractional zero points are
-//    exact too and q == z gives exactly 0.
+//  * Work split.  A CTA owns 32 output columns and a contiguous K range, split
+//    again over its WK warps; a warp owns a run of "quads" (4 packed word rows
+//    x 32 columns).  When there are few column blocks, the CTAs of a
+//    thread-block cluster split K further and reduce their fp32 partial sums
+//    through distributed shared memory.  One launch, no workspace, no atomics.
+//  * Loads.  Each warp streams its K range with 2-D TMA boxes of 32 word rows
+//    x 32 columns (8 quads, 128-byte swizzle) into two shared-memory stages,
+//    completing on an mbarrier: the bytes in flight cost neither registers nor
+//    L1 request slots.  Lane (g, t) (g = lane / 4, t = lane % 4) then reads one
+//    16-byte vector per quad (4 adjacent columns of one word row).
+//  * Dequant.  A code pair (code j, code j + eps/2) sits at the same offset in
+//    the two 16-bit halves of a word: one LOP3 ORs both into the mantissa of
+//    fp16 1024 and one exact fp16x2 FMA gives the integers q - round(z).
+//  * Dot product.  Those exact values are the A operand of a warp MMA m16n8k16
+//    (fp16 in, fp32 accumulate) with x as B: A rows are 16 output columns and
+//    the 16 k-slots are 4 word rows x 4 codes, a permutation of k; x is staged
+//    once per CTA in shared memory in the same permuted order.
+//  * Per group, acc += s * (D - (z - round(z)) * X) in fp32, X = the sum of the
+//    x values of that group slice, so fractional zero points are exact and
+//    q == z gives exactly 0.
 #include <algorithm>
+#include <type_traits>
 
 #include "wq_dequant.cuh"
 #include "wq_internal.h"
 #include "wq_ptx.cuh"
 
 namespace wq {
+
+// Device status of the GEMV: 0, or 1 once a bounded wait ran out.
+__device__ unsigned int g_gemv_status = 0;
+
 namespace {
 
-constexpr int COLS = 32;    // output columns per CTA
-constexpr int MAXW = 8;     // warps per CTA (split along K)
-// quads (4 word rows) each warp keeps in flight
-template <int BITS, int NT> constexpr int pd_for() { return (BITS == 3 || (BITS == 1 && NT == 2)) ? 4 : 8; }
+constexpr int COLS = 32;     // output columns per CTA
+constexpr int MAXW = 16;     // warps per CTA (split along K)
+constexpr int SQ = 8;        // quads per TMA stage (32 word rows x 32 columns = 4 KB)
+constexpr int MAXST = 2;     // stages per warp (at most)
+constexpr uint64_t WAIT_NS = 2000000000ull;
 
-// ------------------------------------------------------------------ kernel
 struct Params {
     const uint16_t* x;
     const uint32_t* w_q;
@@ -52,71 +55,68 @@ struct Params {
     int M, K, N, G;
     int Kw;        // word rows of the main plane
     int Q;         // quads = ceil(Kw / 4)
-    int QW;        // quads per warp
+    int QW;        // quads per warp (a power of two)
     int WK;        // warps per CTA
     int CS;        // CTAs per cluster (along K)
-    int rows_cta;  // word rows staged per CTA = WK * QW * 4
-    int groups_cta;
     int qpg;       // quads per group (a large number when one group spans K)
     int cpt_shift; // log2(x chunks per token staged by a CTA)
     int qc_shift;  // log2(quads per CTA)
+    int groups_cta;
+    int nst;       // TMA stages per warp: 1 or 2
     int xs_tok_stride;  // bytes between tokens in the x stage (padded)
-    uint32_t off_xq, off_tab, off_red, off_part;  // smem byte offsets
+    uint32_t off_x, off_xq, off_tab, off_red, off_part, off_bar;  // smem byte offsets (stages at 0)
 };
 
+// bytes of one stage: 32 x 32 words of the main plane (+ 16 x 32 lo-plane words)
+template <int BITS>
+constexpr int stage_bytes() { return BITS == 3 ? 6144 : 4096; }
+
+// Sum of red[w * stride + i] over the wk (<= MAXW) warps: all loads issued
+// first, then a pairwise tree, so the latency is paid once.
+__device__ __forceinline__ float sum_warps(const float* red, int wk, int stride, int i) {
+    float v[MAXW];
+#pragma unroll
+    for (int w = 0; w < MAXW; ++w) v[w] = (w < wk) ? red[w * stride + i] : 0.0f;
+#pragma unroll
+    for (int h = MAXW / 2; h >= 1; h >>= 1)
+#pragma unroll
+        for (int w = 0; w < h; ++w) v[w] += v[w + h];
+    return v[0];
+}
+
 template <int BITS, int NT>
-__global__ void __launch_bounds__(MAXW * 32, 2)
-gemv_kernel(const Params p) {
+__global__ void __launch_bounds__(MAXW * 32, (NT == 1 && BITS != 1) ? 2 : 1)
+gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_lo, const Params p) {
     using F = Fmt<BITS>;
     constexpr int EPS = F::EPS;
     constexpr int NC = F::NC;
     constexpr int QK = 4 * EPS;  // k values per quad
     constexpr int MMAS = EPS / 4;
-    constexpr int PD = pd_for<BITS, NT>();
-    extern __shared__ __align__(16) uint8_t smem[];
+    constexpr int SB = stage_bytes<BITS>();
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte aligned base: the 128-byte swizzle of the TMA stages repeats every 1024 bytes
+    uint8_t* smem = smem_raw + (((smem_u32(smem_raw) + 1023u) & ~1023u) - smem_u32(smem_raw));
 
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
-    const int rank = (int)blockIdx.y;  // cluster spans the whole grid y extent
+    const int rank = (int)blockIdx.y;  // the cluster spans the grid's y extent
     const int col0 = blockIdx.x * COLS;
     const int mycol = col0 + 4 * g;
     const bool col_ok = mycol < p.N;
 
-    // quad range of the CTA and of this warp
     const int cta_q0 = rank * p.WK * p.QW;
     const int q_begin = cta_q0 + warp * p.QW;
     const int q_end = min(p.Q, q_begin + p.QW);
     const int nq = max(0, q_end - q_begin);
 
-    const uint64_t pol = policy_evict_first();
-
-    // ---- (1) W: issue the first PD quads before anything else (weights need no dependency wait)
-    uint4 buf[PD];
-    uint4 bufl[PD];
-    auto load_quad = [&](int q, uint4& hv, uint4& lv) {
-        const int r = 4 * q + t;
-        if (col_ok && r < p.Kw) {
-            hv = ld_stream_v4(p.w_q + (size_t)r * p.N + mycol, pol);
-            if constexpr (BITS == 3)
-                lv = ld_stream_v4(p.w_lo + (size_t)(r >> 1) * p.N + mycol, pol);
-        } else {
-            hv = make_uint4(0, 0, 0, 0);
-            lv = make_uint4(0, 0, 0, 0);
-        }
-    };
-#pragma unroll
-    for (int j = 0; j < PD; ++j) {
-        if (j < nq) load_quad(q_begin + j, buf[j], bufl[j]);
-    }
-
-    // ---- (2) s, z of the CTA's (group, column) records: first round of loads now
+    // ---- s, z of the CTA's (group, column) records
     const int k_cta0 = cta_q0 * QK;
     const int g_cta0 = min(k_cta0, p.K - 1) / p.G;
     const int n_groups = (p.K + p.G - 1) / p.G;
     const int nrec = p.groups_cta * COLS;
     Rec<BITS>* tab = reinterpret_cast<Rec<BITS>*>(smem + p.off_tab);
-    constexpr int TB = 4;
+    constexpr int TB = 2;
     bool any_frac = false;
     auto tab_load = [&](int base, uint32_t (&v)[TB]) {
 #pragma unroll
@@ -149,8 +149,41 @@ gemv_kernel(const Params p) {
             }
         }
     };
+    // ---- (1) s, z first: these small loads then do not queue behind the weight stream
     uint32_t tv[TB];
     tab_load(0, tv);
+
+    // ---- (2) weights: each warp streams its K range with 2-D TMA boxes of 32
+    // word rows x 32 columns (8 quads, 128-byte swizzle) into nst stages
+    const int nst = p.nst;
+    const uint32_t st0 = smem_u32(smem) + (uint32_t)(warp * nst * SB);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + p.off_bar) + warp * MAXST;
+    const int nst_w = (nq + SQ - 1) / SQ;  // stages this warp consumes
+    auto issue = [&](int k) {              // stage number k of this warp -> slot k % nst
+        const int slot = k & (nst - 1);
+        const uint32_t dst = st0 + slot * SB;
+        mbar_arrive_expect_tx(&bar[slot], (uint32_t)SB);
+        tma_load_2d_u32(dst, &tm_w, &bar[slot], col0, 4 * (q_begin + k * SQ));
+        if constexpr (BITS == 3) tma_load_2d_u32(dst + 4096, &tm_lo, &bar[slot], col0, 2 * (q_begin + k * SQ));
+    };
+    if (lane == 0) {
+#pragma unroll
+        for (int k = 0; k < MAXST; ++k) mbar_init(&bar[k], 1);
+        fence_mbarrier_init();
+        prefetch_tmap(&tm_w);
+        for (int k = 0; k < nst && k < nst_w; ++k) issue(k);
+    }
+    __syncwarp();
+    // the next kernel on the stream may start now (it waits for this grid before reading its x)
+    grid_launch_dependents();
+
+    tab_store(0, tv);
+    for (int base = TB * (int)blockDim.x; base < nrec; base += TB * (int)blockDim.x) {
+        tab_load(base, tv);
+        tab_store(base, tv);
+    }
+    // fractional zero points anywhere in this CTA's records?  (CTA-uniform)
+    const bool frac = __syncthreads_or(any_frac) != 0;
 
     // ---- (3) x may come from the previous kernel on the stream: wait, then load it
     grid_dependency_wait();
@@ -160,10 +193,11 @@ gemv_kernel(const Params p) {
     // (two for 8-bit), read as 16-byte vectors.
     constexpr int CH = EPS >= 8 ? EPS : 8;        // halves per chunk
     constexpr int UPC = CH / 8;                   // 16-byte vectors per chunk
-    constexpr int XB = UPC >= 4 ? 1 : (UPC == 2 ? 2 : 4);  // chunks per thread per round
+    constexpr int XB = UPC >= 2 ? 1 : 2;          // chunks per thread per round
     const int row_cta0 = cta_q0 * 4;
-    const int cpt = 1 << p.cpt_shift;             // chunks per token (rows_cta * EPS / CH)
+    const int cpt = 1 << p.cpt_shift;             // chunks per token
     const int nchunk = p.M * cpt;
+    uint8_t* xs = smem + p.off_x;
     auto x_load = [&](int base, uint4 (&v)[XB][UPC]) {
 #pragma unroll
         for (int u = 0; u < XB; ++u) {
@@ -213,37 +247,27 @@ gemv_kernel(const Params p) {
                         P[rr * (EPS / 2) + j] = prmt(Wr[j / 2], Wr[j / 2 + EPS / 4], (j & 1) ? 0x7632u : 0x5410u);
                     }
                 }
-                uint8_t* dst = smem + m * p.xs_tok_stride + (size_t)ci * CH * 2;
+                uint8_t* dst = xs + m * p.xs_tok_stride + (size_t)ci * CH * 2;
 #pragma unroll
                 for (int w = 0; w < UPC; ++w)
                     *reinterpret_cast<uint4*>(dst + 16 * w) = make_uint4(P[4 * w], P[4 * w + 1], P[4 * w + 2], P[4 * w + 3]);
             }
         }
     };
-    {
+    for (int base = 0; base < nchunk; base += XB * (int)blockDim.x) {
         uint4 xv[XB][UPC];
-        x_load(0, xv);
-        tab_store(0, tv);
-        for (int base = TB * (int)blockDim.x; base < nrec; base += TB * (int)blockDim.x) {
-            tab_load(base, tv);
-            tab_store(base, tv);
-        }
-        x_store(0, xv);
-        for (int base = XB * (int)blockDim.x; base < nchunk; base += XB * (int)blockDim.x) {
-            x_load(base, xv);
-            x_store(base, xv);
-        }
+        x_load(base, xv);
+        x_store(base, xv);
     }
-    // fractional zero points anywhere in this CTA's records?  (CTA-uniform)
-    const bool frac = __syncthreads_or(any_frac) != 0;
+    __syncthreads();
 
-    // ---- (4) per-quad x sums (fp32) from the staged x, for the fractional zero-point term
+    // ---- (4) per-quad x sums (fp32), only needed for fractional zero points
     const int quads_cta = 1 << p.qc_shift;
+    float* xq = reinterpret_cast<float*>(smem + p.off_xq);
     if (frac) {
-        float* xqw = reinterpret_cast<float*>(smem + p.off_xq);
         for (int i = threadIdx.x; i < p.M * quads_cta; i += blockDim.x) {
             const int m = i >> p.qc_shift, ql = i & (quads_cta - 1);
-            const uint4* src = reinterpret_cast<const uint4*>(smem + m * p.xs_tok_stride + (size_t)ql * QK * 2);
+            const uint4* src = reinterpret_cast<const uint4*>(xs + m * p.xs_tok_stride + (size_t)ql * QK * 2);
             float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
             for (int w = 0; w < QK / 8; ++w) {
@@ -256,173 +280,206 @@ gemv_kernel(const Params p) {
                     a1 += f.y;
                 }
             }
-            xqw[i] = a0 + a1;
+            xq[i] = a0 + a1;
         }
         __syncthreads();
     }
-    grid_launch_dependents();
-
-    const float* xq = reinterpret_cast<const float*>(smem + p.off_xq);
-
     float acc[4][NT][2];
-    float dsum[2][NT][4];
-    float xs_sum[NT][2];
 #pragma unroll
     for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int n = 0; n < NT; ++n) acc[c][n][0] = acc[c][n][1] = 0.0f;
-#pragma unroll
-    for (int T = 0; T < 2; ++T)
-#pragma unroll
-        for (int n = 0; n < NT; ++n)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dsum[T][n][i] = 0.0f;
-#pragma unroll
-    for (int n = 0; n < NT; ++n) xs_sum[n][0] = xs_sum[n][1] = 0.0f;
-
-    // token rows feeding the B operand of this lane (duplicates beyond M are harmless)
-    const uint8_t* xb[NT];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) xb[n] = smem + min(g + 8 * n, p.M - 1) * p.xs_tok_stride;
     int tok[NT][2];
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
         tok[n][0] = 2 * t + 8 * n;
         tok[n][1] = 2 * t + 1 + 8 * n;
     }
-    // group bookkeeping without divisions in the loop
-    int gl = (q_begin * QK) / p.G - g_cta0;
-    int left = p.qpg - ((q_begin * QK) % p.G) / QK;  // quads left in the current group
-    // bias constants of the lane's 4 columns, held in registers for narrow records
-    constexpr bool CREG = NC <= 2;
-    uint32_t creg[4][CREG ? NC : 1];
-    auto load_creg = [&](int gidx) {
-        if constexpr (CREG) {
-            const Rec<BITS>* r = tab + gidx * COLS + 4 * g;
+
+    // The main loop, specialised on whether fractional zero-point terms are needed.
+    auto main_loop = [&](auto frac_tag) {
+        constexpr bool FRAC = decltype(frac_tag)::value;
+        constexpr uint32_t RS = sizeof(Rec<BITS>);
+        float dsum[2][NT][4];
+        float xs_sum[NT][2];
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+        for (int T = 0; T < 2; ++T)
 #pragma unroll
-                for (int ci = 0; ci < NC; ++ci) creg[c][ci] = r[c].c[ci];
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dsum[T][n][e] = 0.0f;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) xs_sum[n][0] = xs_sum[n][1] = 0.0f;
+
+        // B-fragment addresses (token rows; duplicates beyond M are harmless)
+        uint32_t xaddr[NT];
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+            xaddr[n] = smem_u32(xs) + (uint32_t)(min(g + 8 * n, p.M - 1) * p.xs_tok_stride +
+                                                 (4 * (q_begin - cta_q0) + t) * EPS * 2);
+        uint32_t xqaddr[NT][2];
+        if constexpr (FRAC) {
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+                    xqaddr[n][e] = smem_u32(xq) + 4u * (uint32_t)((min(tok[n][e], p.M - 1) << p.qc_shift) +
+                                                                  (q_begin - cta_q0));
         }
-    };
-    if (nq > 0) load_creg(gl);
-    const uint32_t lo_sel = (t & 1) ? 0x7372u : 0x7170u;  // 3-bit: which half of the lo word
-
-    for (int base = 0; base < nq; base += PD) {
+        // group bookkeeping without divisions in the loop
+        int left = p.qpg - ((q_begin * QK) % p.G) / QK;  // quads left in the current group
+        uint32_t rc = smem_u32(tab) + RS * (uint32_t)(((q_begin * QK) / p.G - g_cta0) * COLS + 4 * g);
+        // bias constants of the lane's 4 columns, in registers for narrow records
+        constexpr bool CREG = NC <= 2;
+        uint32_t creg[4][CREG ? NC : 1];
+        auto load_creg = [&]() {
+            if constexpr (CREG) {
 #pragma unroll
-        for (int jj = 0; jj < PD; ++jj) {
-            const int i = base + jj;
-            if (i < nq) {
-                const int q = q_begin + i;
-                const uint4 hv = buf[jj];
-                const uint4 lv = bufl[jj];
-                if (i + PD < nq) load_quad(q + PD, buf[jj], bufl[jj]);
-
-                const int ql = q - cta_q0;
-                const Rec<BITS>* rc = tab + gl * COLS + 4 * g;
-
-                // B fragments: this lane's word row of the quad, all MMAS pairs
-                const int rl = 4 * ql + t;
-                uint32_t bx[NT][EPS / 2];
+                for (int c = 0; c < 4; ++c)
 #pragma unroll
-                for (int n = 0; n < NT; ++n) {
+                    for (int ci = 0; ci < NC; ++ci) creg[c][ci] = lds32_u32(rc + c * RS + 8 + 4 * ci);
+            }
+        };
+        if (nq > 0) load_creg();
+        const uint32_t lo_sel = (t & 1) ? 0x7372u : 0x7170u;  // 3-bit: which half of the lo word
+        // Per-lane offsets of this lane's 16-byte vector inside a stage: quad iq,
+        // word row R = 4 iq + t, 16-byte chunk g swizzled with (R & 7), whose
+        // value only depends on the parity of iq.
+        const uint32_t off_even = (uint32_t)t * 128 + (((uint32_t)g ^ (uint32_t)t) << 4);
+        const uint32_t off_odd = (uint32_t)t * 128 + (((uint32_t)g ^ (uint32_t)(t + 4)) << 4);
+        // 3-bit lo plane: row R >> 1 = 2 iq + (t >> 1), swizzled with ((R >> 1) & 7)
+        const uint32_t tl = (uint32_t)(t >> 1);
+        const uint32_t lo_off[4] = {tl * 128 + (((uint32_t)g ^ tl) << 4), tl * 128 + (((uint32_t)g ^ (tl + 2)) << 4),
+                                    tl * 128 + (((uint32_t)g ^ (tl + 4)) << 4), tl * 128 + (((uint32_t)g ^ (tl + 6)) << 4)};
+
+        auto quad = [&](uint32_t stage, int iq, int i) {
+            const uint4 hv = lds128_u32(stage + 512 * iq + ((iq & 1) ? off_odd : off_even));
+            uint4 lv = make_uint4(0, 0, 0, 0);
+            if constexpr (BITS == 3) lv = lds128_u32(stage + 4096 + 256 * iq + lo_off[iq & 3]);
+            // B fragments: this lane's word row of the quad, all MMAS pairs
+            uint32_t bx[NT][EPS / 2];
 #pragma unroll
-                    for (int v = 0; v < EPS / 8; ++v) {
-                        const uint4 u = *reinterpret_cast<const uint4*>(xb[n] + (size_t)rl * EPS * 2 + 16 * v);
-                        bx[n][4 * v + 0] = u.x;
-                        bx[n][4 * v + 1] = u.y;
-                        bx[n][4 * v + 2] = u.z;
-                        bx[n][4 * v + 3] = u.w;
-                    }
-                    if constexpr (EPS / 8 == 0) {
-                        const uint2 u = *reinterpret_cast<const uint2*>(xb[n] + (size_t)rl * EPS * 2);
-                        bx[n][0] = u.x;
-                        bx[n][1] = u.y;
-                    }
+            for (int n = 0; n < NT; ++n) {
+#pragma unroll
+                for (int v = 0; v < EPS / 8; ++v) {
+                    const uint4 u = lds128_u32(xaddr[n] + QK * 2 * iq + 16 * v);
+                    bx[n][4 * v + 0] = u.x;
+                    bx[n][4 * v + 1] = u.y;
+                    bx[n][4 * v + 2] = u.z;
+                    bx[n][4 * v + 3] = u.w;
                 }
-                // x sums of this quad for the tokens this lane accumulates
-                if (frac) {
-#pragma unroll
-                    for (int n = 0; n < NT; ++n) {
-                        xs_sum[n][0] += (tok[n][0] < p.M) ? xq[tok[n][0] * quads_cta + ql] : 0.0f;
-                        xs_sum[n][1] += (tok[n][1] < p.M) ? xq[tok[n][1] * quads_cta + ql] : 0.0f;
-                    }
-                }
-
-                const uint32_t wv[4] = {hv.x, hv.y, hv.z, hv.w};
-                const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
-#pragma unroll
-                for (int T = 0; T < 2; ++T) {
-                    const int ca = 2 * T, cb = 2 * T + 1;
-                    uint32_t cA[NC], cB[NC];
-#pragma unroll
-                    for (int ci = 0; ci < NC; ++ci) {
-                        if constexpr (CREG) {
-                            cA[ci] = creg[ca][ci];
-                            cB[ci] = creg[cb][ci];
-                        } else {
-                            cA[ci] = rc[ca].c[ci];
-                            cB[ci] = rc[cb].c[ci];
-                        }
-                    }
-                    uint32_t wA = wv[ca], wB = wv[cb], wAh, wBh, lA = 0, lB = 0;
-                    if constexpr (BITS == 4) { wAh = wA >> 8; wBh = wB >> 8; }
-                    else if constexpr (BITS == 2 || BITS == 1) { wAh = wA >> 10; wBh = wB >> 10; }
-                    else if constexpr (BITS == 3) {
-                        wAh = wA >> 7; wBh = wB >> 7;
-                        wA <<= 1; wB <<= 1;
-                        lA = prmt(lw[ca], 0u, lo_sel) << 1;
-                        lB = prmt(lw[cb], 0u, lo_sel) << 1;
-                    } else { wAh = wA; wBh = wB; }
-#pragma unroll
-                    for (int h = 0; h < MMAS; ++h) {
-                        uint32_t a[4];
-                        a[0] = pair_q<BITS>(wA, wAh, lA, cA, 2 * h);
-                        a[1] = pair_q<BITS>(wB, wBh, lB, cB, 2 * h);
-                        a[2] = pair_q<BITS>(wA, wAh, lA, cA, 2 * h + 1);
-                        a[3] = pair_q<BITS>(wB, wBh, lB, cB, 2 * h + 1);
-#pragma unroll
-                        for (int n = 0; n < NT; ++n) mma_16816(dsum[T][n], a, bx[n][2 * h], bx[n][2 * h + 1]);
-                    }
-                }
-
-                // end of a group (or of this warp's range): scale and fold into acc
-                --left;
-                const bool last = (i == nq - 1) || left == 0;
-                if (last) {
-#pragma unroll
-                    for (int T = 0; T < 2; ++T) {
-#pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-                            const int c = 2 * T + half;
-                            const float s = rc[c].s;
-                            const float zr = frac ? rc[c].zr : 0.0f;
-#pragma unroll
-                            for (int n = 0; n < NT; ++n) {
-#pragma unroll
-                                for (int e = 0; e < 2; ++e) {
-                                    const float d = frac ? dsum[T][n][2 * half + e] - zr * xs_sum[n][e]
-                                                         : dsum[T][n][2 * half + e];
-                                    acc[c][n][e] = fmaf(s, d, acc[c][n][e]);
-                                }
-                            }
-                        }
-#pragma unroll
-                        for (int n = 0; n < NT; ++n)
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) dsum[T][n][e] = 0.0f;
-                    }
-#pragma unroll
-                    for (int n = 0; n < NT; ++n) xs_sum[n][0] = xs_sum[n][1] = 0.0f;
-                    if (left == 0) {
-                        ++gl;
-                        left = p.qpg;
-                        if (i + 1 < nq) load_creg(gl);
-                    }
+                if constexpr (EPS / 8 == 0) {
+                    const uint2 u = lds64_u32(xaddr[n] + QK * 2 * iq);
+                    bx[n][0] = u.x;
+                    bx[n][1] = u.y;
                 }
             }
+            if constexpr (FRAC) {
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) xs_sum[n][e] += __uint_as_float(lds32_u32(xqaddr[n][e] + 4 * iq));
+            }
+
+            const uint32_t wv[4] = {hv.x, hv.y, hv.z, hv.w};
+            const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
+#pragma unroll
+            for (int T = 0; T < 2; ++T) {
+                const int ca = 2 * T, cb = 2 * T + 1;
+                uint32_t cA[NC], cB[NC];
+#pragma unroll
+                for (int ci = 0; ci < NC; ++ci) {
+                    if constexpr (CREG) {
+                        cA[ci] = creg[ca][ci];
+                        cB[ci] = creg[cb][ci];
+                    } else {
+                        cA[ci] = lds32_u32(rc + ca * RS + 8 + 4 * ci);
+                        cB[ci] = lds32_u32(rc + cb * RS + 8 + 4 * ci);
+                    }
+                }
+                uint32_t wA = wv[ca], wB = wv[cb], wAh = 0, wBh = 0, lA = 0, lB = 0;
+                prep_word<BITS>(wA, wAh, lA, lw[ca], lo_sel);
+                prep_word<BITS>(wB, wBh, lB, lw[cb], lo_sel);
+#pragma unroll
+                for (int h = 0; h < MMAS; ++h) {
+                    uint32_t a[4];
+                    a[0] = pair_q<BITS>(wA, wAh, lA, cA, 2 * h);
+                    a[1] = pair_q<BITS>(wB, wBh, lB, cB, 2 * h);
+                    a[2] = pair_q<BITS>(wA, wAh, lA, cA, 2 * h + 1);
+                    a[3] = pair_q<BITS>(wB, wBh, lB, cB, 2 * h + 1);
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) mma_16816(dsum[T][n], a, bx[n][2 * h], bx[n][2 * h + 1]);
+                }
+            }
+
+            // end of a group (or of this warp's range): scale and fold into acc
+            if (--left == 0 || i == nq - 1) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float sc = __uint_as_float(lds32_u32(rc + c * RS));
+                    const float zr = FRAC ? __uint_as_float(lds32_u32(rc + c * RS + 4)) : 0.0f;
+                    const int T = c >> 1, half = c & 1;
+#pragma unroll
+                    for (int n = 0; n < NT; ++n)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const float d = FRAC ? dsum[T][n][2 * half + e] - zr * xs_sum[n][e]
+                                                 : dsum[T][n][2 * half + e];
+                            acc[c][n][e] = fmaf(sc, d, acc[c][n][e]);
+                        }
+                }
+#pragma unroll
+                for (int T = 0; T < 2; ++T)
+#pragma unroll
+                    for (int n = 0; n < NT; ++n)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) dsum[T][n][e] = 0.0f;
+                if constexpr (FRAC) {
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) xs_sum[n][0] = xs_sum[n][1] = 0.0f;
+                }
+                if (left == 0) {
+                    left = p.qpg;
+                    rc += COLS * RS;
+                    if (i + 1 < nq) load_creg();
+                }
+            }
+        };
+
+        for (int kst = 0; kst < nst_w; ++kst) {
+            const bool good = mbar_wait_bounded(&bar[kst & (nst - 1)], (kst / nst) & 1, WAIT_NS);
+            if (!good) atomicExch(&g_gemv_status, 1u);
+            if (!__all_sync(0xffffffffu, good)) break;  // give up this warp's range
+            const uint32_t stage = st0 + (kst & (nst - 1)) * SB;
+            const int i0 = kst * SQ;
+            if (i0 + SQ <= nq) {
+#pragma unroll
+                for (int iq = 0; iq < SQ; ++iq) quad(stage, iq, i0 + iq);
+            } else {
+#pragma unroll
+                for (int iq = 0; iq < SQ; ++iq)
+                    if (i0 + iq < nq) quad(stage, iq, i0 + iq);
+            }
+#pragma unroll
+            for (int n = 0; n < NT; ++n) xaddr[n] += QK * 2 * SQ;
+            if constexpr (FRAC) {
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) xqaddr[n][e] += 4 * SQ;
+            }
+            // every lane has used this stage's words: refill its slot with stage kst + nst
+            __syncwarp();
+            if (lane == 0 && kst + nst < nst_w) {
+                fence_proxy_async_smem();
+                issue(kst + nst);
+            }
         }
-    }
+    };
+    if (frac)
+        main_loop(std::true_type{});
+    else
+        main_loop(std::false_type{});
 
     // ---- reduce over the warps of the CTA
     float* red = reinterpret_cast<float*>(smem + p.off_red);  // [WK][M][COLS]
@@ -437,14 +494,11 @@ gemv_kernel(const Params p) {
             }
     __syncthreads();
     float* part = reinterpret_cast<float*>(smem + p.off_part);  // [M][COLS]
-    for (int i = threadIdx.x; i < p.M * COLS; i += blockDim.x) {
-        float sacc = 0.0f;
-        for (int w = 0; w < p.WK; ++w) sacc += red[w * p.M * COLS + i];
-        part[i] = sacc;
-    }
-
-    // ---- reduce over the CTAs of the cluster through distributed shared memory
     if (p.CS > 1) {
+        for (int i = threadIdx.x; i < p.M * COLS; i += blockDim.x) {
+            part[i] = sum_warps(red, p.WK, p.M * COLS, i);
+        }
+        // reduce over the CTAs of the cluster through distributed shared memory
         cluster_sync();
         const uint32_t part_addr = smem_u32(part);
         for (int i = rank + p.CS * (int)threadIdx.x; i < p.M * COLS; i += p.CS * blockDim.x) {
@@ -455,29 +509,15 @@ gemv_kernel(const Params p) {
         }
         cluster_sync();  // peers keep their shared memory until every read is done
     } else {
-        __syncthreads();
         for (int i = threadIdx.x; i < p.M * COLS; i += blockDim.x) {
+            const float sacc = sum_warps(red, p.WK, p.M * COLS, i);
             const int m = i / COLS, col = col0 + i % COLS;
-            if (col < p.N) p.y[(size_t)m * p.N + col] = __half_as_ushort(__float2half_rn(part[i]));
+            if (col < p.N) p.y[(size_t)m * p.N + col] = __half_as_ushort(__float2half_rn(sacc));
         }
     }
 }
 
 // ------------------------------------------------------------------- host
-int sm_count() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
-
-template <int BITS>
-size_t rec_bytes() { return sizeof(Rec<BITS>); }
-
 int ilog2(int v) {
     int r = 0;
     while ((1 << (r + 1)) <= v) ++r;
@@ -494,8 +534,7 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return WQ_ERR_CUDA;
     if (dev < 64 && !(attr_done & (1ull << dev))) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
             return WQ_ERR_CUDA;
         attr_done |= 1ull << dev;
     }
@@ -506,70 +545,89 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     prm.Q = (prm.Kw + 3) / 4;
     prm.qpg = (pb.G == pb.K) ? (1 << 29) : pb.G / QK;
     const int colblocks = (pb.N + COLS - 1) / COLS;
-    const int WK = std::min(MAXW, std::max(1, prm.Q >= 8 ? 8 : (prm.Q >= 4 ? 4 : (prm.Q >= 2 ? 2 : 1))));
     const int sms = sm_count();
 
-    auto smem_for = [&](int CS, int QW, Params& q) -> size_t {
+    auto layout = [&](int WK, int CS, int QW, Params& q) -> size_t {
         q.WK = WK; q.CS = CS; q.QW = QW;
-        q.rows_cta = WK * QW * 4;
+        const int rows_cta = WK * QW * 4;
         const int quads_cta = WK * QW;
         const int ch = EPS >= 8 ? EPS : 8;
-        q.cpt_shift = ilog2(q.rows_cta * EPS / ch);
+        q.cpt_shift = ilog2(rows_cta * EPS / ch);
         q.qc_shift = ilog2(quads_cta);
-        const int k0 = 0, k1 = quads_cta * QK;  // span of one CTA
-        q.groups_cta = std::min((k1 - k0 + pb.G - 1) / pb.G + 1, (pb.K + pb.G - 1) / pb.G);
-        q.xs_tok_stride = q.rows_cta * EPS * 2 + 16;
-        size_t off = (size_t)pb.M * q.xs_tok_stride;
+        q.groups_cta = std::min((quads_cta * QK + pb.G - 1) / pb.G + 1, (pb.K + pb.G - 1) / pb.G);
+        q.xs_tok_stride = rows_cta * EPS * 2 + 16;
+        q.nst = QW > SQ ? 2 : 1;
+        size_t off = (size_t)WK * q.nst * stage_bytes<BITS>();
+        q.off_bar = (uint32_t)off;
+        off += (size_t)WK * MAXST * 8;
+        q.off_x = (uint32_t)off;
+        off += (size_t)pb.M * q.xs_tok_stride;
         off = (off + 15) & ~(size_t)15;
         q.off_xq = (uint32_t)off;
         off += (size_t)pb.M * quads_cta * 4;
         off = (off + 15) & ~(size_t)15;
         q.off_tab = (uint32_t)off;
-        off += (size_t)q.groups_cta * COLS * rec_bytes<BITS>();
+        off += (size_t)q.groups_cta * COLS * sizeof(Rec<BITS>);
         q.off_red = (uint32_t)off;
         off += (size_t)WK * pb.M * COLS * 4;
         q.off_part = (uint32_t)off;
         off += (size_t)pb.M * COLS * 4;
-        return off;
+        return off + 1024;  // slack for aligning the base to 1024 bytes
     };
 
-    // Pick the widest cluster split whose grid is resident in one wave.
-    int best_cs = 1;
-    Params chosen{};
-    size_t chosen_smem = 0;
+    // Among (warps per CTA, cluster size), pick the plan with the fewest waves x
+    // quads per warp; ties go to no cluster and larger CTAs.
     bool found = false;
-    for (int CS = 8; CS >= 1; CS >>= 1) {
-        if (WK * CS > prm.Q && CS > 1) continue;
-        int QW = 1;
-        while (QW * WK * CS < prm.Q) QW <<= 1;
-        Params q = prm;
-        const size_t sm = smem_for(CS, QW, q);
-        if (sm > 227 * 1024) continue;
-        int occ = 0;
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, WK * 32, sm);
-        cudaGetLastError();
-        if (occ <= 0) continue;
-        if ((long)colblocks * CS <= (long)occ * sms || CS == 1) {
-            best_cs = CS;
-            chosen = q;
-            chosen_smem = sm;
-            found = true;
-            break;
+    Params best{};
+    size_t best_smem = 0;
+    long best_score = 0;
+    for (int WK : {16, 8, 4}) {
+        for (int CS : {1, 2, 4, 8}) {
+            if (CS > 1 && WK * CS > prm.Q) continue;
+            int QW = 1;
+            while (QW * WK * CS < prm.Q) QW <<= 1;
+            Params q = prm;
+            const size_t sm = layout(WK, CS, QW, q);
+            if (sm > 227 * 1024) continue;
+            int occ = 0;
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, WK * 32, sm);
+            cudaGetLastError();
+            if (occ <= 0) continue;
+            const long ctas = (long)colblocks * CS;
+            const long waves = (ctas + (long)occ * sms - 1) / ((long)occ * sms);
+            // per-warp serial work (quads, at least a full ring of them) x waves,
+            // plus a penalty for the cluster reduction
+            const long score = waves * std::max(QW, SQ) * 64 + (CS > 1 ? 96 : 0) + (16 / WK);
+            if (!found || score < best_score) {
+                found = true;
+                best = q;
+                best_smem = sm;
+                best_score = score;
+            }
         }
     }
     if (!found) return WQ_ERR_INVALID_ARG;  // shape too large for the shared-memory plan
-    (void)best_cs;
+
+    CUtensorMap mw, ml;
+    bool ok = make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, pb.w_q, pb.N, prm.Kw, (uint64_t)pb.N * 4, COLS, 4 * SQ,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    if (BITS == 3)
+        ok = ok && make_map(&ml, CU_TENSOR_MAP_DATA_TYPE_UINT32, pb.w_lo, pb.N, pb.K / 32, (uint64_t)pb.N * 4, COLS,
+                            2 * SQ, CU_TENSOR_MAP_SWIZZLE_128B);
+    else
+        ml = mw;
+    if (!ok) return WQ_ERR_CUDA;
 
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(colblocks, chosen.CS, 1);
-    cfg.blockDim = dim3(WK * 32, 1, 1);
-    cfg.dynamicSmemBytes = chosen_smem;
+    cfg.gridDim = dim3(colblocks, best.CS, 1);
+    cfg.blockDim = dim3(best.WK * 32, 1, 1);
+    cfg.dynamicSmemBytes = best_smem;
     cfg.stream = stream;
     cudaLaunchAttribute attrs[2];
     int na = 0;
     attrs[na].id = cudaLaunchAttributeClusterDimension;
     attrs[na].val.clusterDim.x = 1;
-    attrs[na].val.clusterDim.y = chosen.CS;
+    attrs[na].val.clusterDim.y = best.CS;
     attrs[na].val.clusterDim.z = 1;
     ++na;
     if (pb.flags & WQ_FLAG_PDL) {
@@ -579,10 +637,21 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     }
     cfg.attrs = attrs;
     cfg.numAttrs = na;
-    return from_cuda(cudaLaunchKernelEx(&cfg, kern, chosen));
+    return from_cuda(cudaLaunchKernelEx(&cfg, kern, mw, ml, best));
 }
 
 }  // namespace
+
+wq_status gemv_device_status(int reset) {
+    unsigned int v = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return WQ_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&v, g_gemv_status, sizeof(v)) != cudaSuccess) return WQ_ERR_CUDA;
+    if (reset) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_gemv_status, &zero, sizeof(zero)) != cudaSuccess) return WQ_ERR_CUDA;
+    }
+    return v ? WQ_ERR_TIMEOUT : WQ_OK;
+}
 
 wq_status launch_gemv(const Problem& p, cudaStream_t s) {
     const bool two = p.M > 8;

@@ -1,6 +1,7 @@
 // wq_internal.h -- declarations shared by the C-ABI layer and the kernel files.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -27,8 +28,15 @@ wq_status launch_unpack(const uint32_t* w_q, const uint32_t* w_lo, int K, int N,
 wq_status launch_gemv(const Problem& p, cudaStream_t s);
 wq_status launch_gemm(const Problem& p, cudaStream_t s);
 
-// Device status words (one per kernel file), read and optionally cleared.
+// Device status words (one per kernel file): nonzero once a bounded wait ran out.
+// Reading synchronises the device; reset clears the word.
 wq_status gemm_device_status(int reset);
+wq_status gemv_device_status(int reset);
+
+// 2-D tiled TMA descriptor for a row-major (outer, inner) array.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
+int sm_count();
 
 inline wq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA; }
 
