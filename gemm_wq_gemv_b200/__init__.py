@@ -10,7 +10,9 @@ Entry points (same names as the C ABI, without the ``wq_`` prefix):
 * ``pack_kmajor(codes_kn, bits) -> (w_q, w_lo)``
 * ``unpack_kmajor(w_q, w_lo, K, bits) -> codes_kn``
 * ``gemv(x, w_q, w_lo, scales, zeros, bits, group_size, out=None, pdl=False) -> y``
-* ``gemm(x, w_q, w_lo, scales, zeros, bits, group_size, out=None, pdl=False) -> y``
+* ``gemm(x, w_q, w_lo, scales, zeros, bits, group_size, out=None, pdl=False,
+  workspace=None) -> y``
+* ``gemm_workspace_size(M, K, N, bits, group_size) -> bytes``
 """
 from __future__ import annotations
 
@@ -58,7 +60,9 @@ def lib() -> ctypes.CDLL:
         L.wq_pack_kmajor.argtypes = [p, i, i, i, p, p, p, p]
         L.wq_unpack_kmajor.argtypes = [p, p, i, i, i, p, p]
         L.wq_gemv.argtypes = [p, p, p, p, p, p, i, i, i, i, i, u, p]
-        L.wq_gemm.argtypes = [p, p, p, p, p, p, i, i, i, i, i, u, p]
+        L.wq_gemm.argtypes = [p, p, p, p, p, p, i, i, i, i, i, u, p, ctypes.c_size_t, p]
+        L.wq_gemm_workspace_size.argtypes = [i, i, i, i, i]
+        L.wq_gemm_workspace_size.restype = ctypes.c_size_t
         L.wq_device_status.argtypes = [i]
         for f in ("wq_pack_kmajor", "wq_unpack_kmajor", "wq_gemv", "wq_gemm", "wq_device_status"):
             getattr(L, f).restype = i
@@ -141,7 +145,7 @@ def unpack_kmajor(w_q, w_lo, K: int, bits: int):
     return out
 
 
-def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl):
+def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, workspace=False):
     torch = _torch()
     _need(x, torch.float16, "x")
     _need(w_q, torch.int32, "w_q")
@@ -156,8 +160,13 @@ def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl):
     else:
         _need(out, torch.float16, "out")
     flags = WQ_FLAG_PDL if pdl else 0
-    st = getattr(lib(), fn)(_ptr(x), _ptr(w_q), _ptr(w_lo), _ptr(scales), _ptr(zeros), _ptr(out),
-                            M, K, N, bits, group_size, flags, _stream())
+    args = [_ptr(x), _ptr(w_q), _ptr(w_lo), _ptr(scales), _ptr(zeros), _ptr(out),
+            M, K, N, bits, group_size, flags]
+    if workspace is not False:  # wq_gemm: (workspace, bytes)
+        if workspace is None:
+            workspace = _cached_workspace(x.device, gemm_workspace_size(M, K, N, bits, group_size))
+        args += [_ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size()]
+    st = getattr(lib(), fn)(*args, _stream())
     _check(fn, st)
     return out
 
@@ -167,9 +176,47 @@ def gemv(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl:
     return _product("wq_gemv", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl)
 
 
-def gemm(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl: bool = False):
-    """y (M, N) fp16 = x (M, K) @ dequant(w_q), any M >= 1 (``wq_gemm``)."""
-    return _product("wq_gemm", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl)
+def gemm_workspace_size(M: int, K: int, N: int, bits: int, group_size: int) -> int:
+    """Bytes of split-K workspace ``wq_gemm`` uses for this shape on the current device."""
+    return int(lib().wq_gemm_workspace_size(M, K, N, bits, group_size))
+
+
+_workspaces = {}
+
+
+def _cached_workspace(device, nbytes: int):
+    """A workspace of at least ``nbytes`` for calls on the current stream of ``device``.
+
+    One buffer per (device, stream): calls on one stream run one after another,
+    so they may share it; calls on different streams get their own.  It only
+    grows.  Allocated inside a CUDA graph capture it comes from the graph's
+    pool and stays valid while cached, like any tensor the capture returns.  A
+    captured graph keeps the buffer's address: graphs replayed at the same time
+    on different streams must be captured with workspaces of their own
+    (``workspace=``).
+    """
+    if nbytes == 0:
+        return None
+    torch = _torch()
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
+def gemm(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl: bool = False,
+         workspace=None):
+    """y (M, N) fp16 = x (M, K) @ dequant(w_q), any M >= 1 (``wq_gemm``).
+
+    ``workspace``: a CUDA uint8 tensor of at least ``gemm_workspace_size(...)``
+    bytes for splitting K over a cluster; by default one cached per stream.
+    """
+    if workspace is not None:
+        torch = _torch()
+        _need(workspace, torch.uint8, "workspace", ndim=1)
+    return _product("wq_gemm", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, workspace)
 
 
 def device_status(reset: bool = False) -> int:

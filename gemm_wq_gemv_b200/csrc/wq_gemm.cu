@@ -13,15 +13,18 @@
 //    shared-memory stages: the x tile (TN x 64 fp16, 128-byte swizzle, which is
 //    the MMA's K-major layout), the packed word tile (64 / eps rows x 128 columns),
 //    the 3-bit lo-plane tile and the s, z rows of the block's group(s).
-//  * Warps 2-5 (one thread per weight column) turn that column's words into 64
-//    fp16 values (q - z) * s -- code pairs become exact q - round(z) with one
-//    LOP3 + one FMA, are put in k order with PRMT and scaled with one more FMA --
-//    and store them into the A tile in the same swizzled K-major layout.
+//  * Warps 2-9 (two threads per weight column, each taking half of the stage's
+//    word rows) turn that column's words into 32 fp16 values (q - z) * s each --
+//    code pairs become exact q - round(z) with one LOP3 + one FMA, are put in k
+//    order with PRMT and scaled with one more FMA -- and store them with
+//    tcgen05.st into tensor memory, where the MMA reads its A operand.
 //  * Warp 1 (one lane) issues four tcgen05.mma (K = 16 each) per stage and
 //    frees the stage with tcgen05.commit when they have read it.
-//  * K is split over the CTAs of a thread-block cluster; after the main loop the
-//    fp32 tiles are summed through distributed shared memory (one launch, no
-//    workspace), converted to fp16 and stored by warps 2-5.
+//  * K may be split over the CTAs of a thread-block cluster; after the main loop
+//    each CTA writes the 32-token slices of its fp32 tile that another rank owns
+//    into a caller-provided global workspace (it stays in L2), one cluster
+//    barrier (release / acquire) orders those writes, and each owner adds its
+//    peers' slices to its own before converting to fp16 and storing y.
 // Every wait on an mbarrier is bounded; on time-out the kernel records
 // WQ_ERR_TIMEOUT in a device status word, skips its remaining work, still
 // frees its tensor memory and returns.
@@ -41,7 +44,9 @@ namespace {
 
 constexpr int BMW = 128;    // weight columns per tile (MMA M)
 constexpr int BK = 64;      // k per stage
-constexpr int NWARPS = 6;   // 0 TMA, 1 MMA + TMEM, 2-5 dequant + epilogue
+constexpr int NWARPS = 10;  // 0 TMA, 1 MMA + TMEM, 2-9 dequant + epilogue (two per TMEM lane quadrant)
+constexpr int NDQ = NWARPS - 2;
+constexpr size_t CHUNK_BYTES = 128 * 32 * 4;  // one 32-token fp32 slice of the tile
 constexpr uint64_t WAIT_NS = 2000000000ull;
 
 struct GemmParams {
@@ -52,11 +57,12 @@ struct GemmParams {
     int kb_cta;          // k blocks per CTA
     int GPB;             // s/z rows per stage
     int stages;
-    uint32_t stage_bytes, off_a, off_w, off_lo, off_s, off_z;
+    uint32_t stage_bytes, off_w, off_lo, off_s, off_z;
+    uint32_t a_col;      // first tensor-memory column of the A stages (32 columns per stage)
     uint32_t tx_bytes;
     uint32_t tmem_cols;
     uint32_t bar_off;    // offset of the barrier block from the aligned base
-    int njl;             // token chunks (32) owned per CTA in the split-K reduction
+    uint4* ws;           // split-K slices: [tile][rank][32-token chunk][16-byte piece][128 columns]
 };
 
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
@@ -94,7 +100,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&full_tma[s], 1);
-            mbar_init(&full_a[s], 4);
+            mbar_init(&full_a[s], NDQ);
             mbar_init(&empty[s], 1);
         }
         mbar_init(accum, 1);
@@ -152,77 +158,77 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
                 tc_fence_after();
                 const uint32_t st = smem_u32(base + (size_t)s * p.stage_bytes);
                 const uint64_t bdesc = sw128_desc(st);
-                const uint64_t adesc = sw128_desc(st + p.off_a);
+                const uint32_t a_tm = tmem_d + p.a_col + 32u * s;  // lane 0, this stage's A columns
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk)
-                    tc_mma_f16(tmem_d, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                    tc_mma_f16_ts(tmem_d, a_tm + 8 * kk, bdesc + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(&empty[s]);
             }
             tc_commit(accum);
         }
     } else {
-        // ------------------------------------------- dequantisation (one column each)
+        // ----------------------- dequantisation: a column per thread, half of its words per warp
         const int qd = warp & 3;                 // TMEM lane quadrant this warp may read
+        const int hf = (warp - 2) >> 2;          // which half of the stage's word rows
         const int nl = 32 * qd + lane;           // weight column within the tile
+        constexpr int RH = RW / 2;               // word rows per half (RW >= 2 for every width)
         const uint32_t lo_sel0 = 0x7170u, lo_sel1 = 0x7372u;
+
+        // (q - z) * s for word row rw of this column, in k order, into out[0 .. EPS/2)
+        auto word = [&](const uint8_t* st, int rw, const uint32_t (&c)[NC], uint32_t s2, uint32_t zs2,
+                        uint32_t* out) {
+            const uint32_t* wt = reinterpret_cast<const uint32_t*>(st + p.off_w);
+            uint32_t w = wt[rw * BMW + nl], wh = 0, ls = 0, lw = 0;
+            if constexpr (BITS == 3) lw = reinterpret_cast<const uint32_t*>(st + p.off_lo)[(rw >> 1) * BMW + nl];
+            prep_word<BITS>(w, wh, ls, lw, (rw & 1) ? lo_sel1 : lo_sel0);
+            uint32_t P[EPS / 2];
+#pragma unroll
+            for (int j = 0; j < EPS / 2; ++j) P[j] = pair_q<BITS>(w, wh, ls, c, j);
+#pragma unroll
+            for (int i = 0; i < EPS / 4; ++i) {
+                out[i] = hfma2_u32(prmt(P[2 * i], P[2 * i + 1], 0x5410u), s2, zs2);
+                out[i + EPS / 4] = hfma2_u32(prmt(P[2 * i], P[2 * i + 1], 0x7632u), s2, zs2);
+            }
+        };
+        // per-(group, column) constants from the stage's s, z rows
+        auto consts = [&](const uint8_t* st, int gi, uint32_t (&c)[NC], uint32_t& s2, uint32_t& zs2) {
+            const float sv = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(st + p.off_s)[gi * BMW + nl]));
+            const float zv = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(st + p.off_z)[gi * BMW + nl]));
+            const float zi = fminf(fmaxf(rintf(zv), -256.0f), 256.0f);
+#pragma unroll
+            for (int ci = 0; ci < NC; ++ci) c[ci] = dup_half(-(bias_magnitude<BITS>(ci) + zi));
+            s2 = dup_half(sv);
+            zs2 = dup_half(-(zv - zi) * sv);
+        };
+
         for (int kb = 0; kb < p.kb_cta; ++kb) {
             const int s = kb % p.stages, r = kb / p.stages;
             if (!mbar_wait_bounded(&full_tma[s], r & 1, WAIT_NS)) { fail(); break; }
             if (*abort_flag) break;
-            uint8_t* st = base + (size_t)s * p.stage_bytes;
-            const uint32_t* wt = reinterpret_cast<const uint32_t*>(st + p.off_w);
-            const uint32_t* lt = reinterpret_cast<const uint32_t*>(st + p.off_lo);
-            const uint16_t* sr = reinterpret_cast<const uint16_t*>(st + p.off_s);
-            const uint16_t* zr_ = reinterpret_cast<const uint16_t*>(st + p.off_z);
-            uint8_t* arow = st + p.off_a + nl * 128;
-            const int sw = nl & 7;
-
-            int cur_g = -1;
-            uint32_t c[NC];
-            uint32_t s2 = 0, zs2 = 0;
+            const uint8_t* st = base + (size_t)s * p.stage_bytes;
+            uint32_t c[NC], s2, zs2;
+            uint32_t a16[16];  // this thread's 32 k values (16 fp16 pairs) of the stage's A row
+            if (p.GPB == 1) {  // one group covers the whole k block
+                consts(st, 0, c, s2, zs2);
 #pragma unroll
-            for (int rw = 0; rw < RW; ++rw) {
-                // group row of this word within the stage's s/z rows
-                const int gi = (p.GPB == 1) ? 0 : (rw * EPS) / p.G;
-                if (gi != cur_g) {
-                    cur_g = gi;
-                    const float sv = __half2float(__ushort_as_half(sr[gi * BMW + nl]));
-                    const float zv = __half2float(__ushort_as_half(zr_[gi * BMW + nl]));
-                    const float zi = fminf(fmaxf(rintf(zv), -256.0f), 256.0f);
+                for (int u = 0; u < RH; ++u) word(st, hf * RH + u, c, s2, zs2, a16 + u * (EPS / 2));
+            } else {
+                int cur = -1;
 #pragma unroll
-                    for (int ci = 0; ci < NC; ++ci) c[ci] = dup_half(-(bias_magnitude<BITS>(ci) + zi));
-                    s2 = dup_half(sv);
-                    zs2 = dup_half(-(zv - zi) * sv);
-                }
-                uint32_t w = wt[rw * BMW + nl], wh = 0, ls = 0;
-                uint32_t lw = 0;
-                if constexpr (BITS == 3) lw = lt[(rw >> 1) * BMW + nl];
-                prep_word<BITS>(w, wh, ls, lw, (rw & 1) ? lo_sel1 : lo_sel0);
-                uint32_t P[EPS / 2];
-#pragma unroll
-                for (int j = 0; j < EPS / 2; ++j) P[j] = pair_q<BITS>(w, wh, ls, c, j);
-                uint32_t Nh[EPS / 2];
-#pragma unroll
-                for (int i = 0; i < EPS / 4; ++i) {
-                    Nh[i] = prmt(P[2 * i], P[2 * i + 1], 0x5410u);
-                    Nh[i + EPS / 4] = prmt(P[2 * i], P[2 * i + 1], 0x7632u);
-                }
-#pragma unroll
-                for (int i = 0; i < EPS / 2; ++i) Nh[i] = hfma2_u32(Nh[i], s2, zs2);
-                // k = rw * EPS .. + EPS - 1 -> 16-byte chunks of 8 halves, swizzled
-                if constexpr (EPS >= 8) {
-#pragma unroll
-                    for (int v = 0; v < EPS / 8; ++v) {
-                        const int chunk = rw * (EPS / 8) + v;
-                        *reinterpret_cast<uint4*>(arow + ((chunk ^ sw) << 4)) =
-                            make_uint4(Nh[4 * v], Nh[4 * v + 1], Nh[4 * v + 2], Nh[4 * v + 3]);
+                for (int u = 0; u < RH; ++u) {
+                    const int rw = hf * RH + u;
+                    const int gi = (rw * EPS) / p.G;
+                    if (gi != cur) {
+                        cur = gi;
+                        consts(st, gi, c, s2, zs2);
                     }
-                } else {
-                    const int chunk = rw >> 1;
-                    *reinterpret_cast<uint2*>(arow + ((chunk ^ sw) << 4) + 8 * (rw & 1)) = make_uint2(Nh[0], Nh[1]);
+                    word(st, rw, c, s2, zs2, a16 + u * (EPS / 2));
                 }
             }
-            fence_proxy_async_smem();
+            // A row of weight column nl = tensor-memory lane nl; k pairs along the columns
+            tmem_st_32x32b_x16(tmem_d + ((uint32_t)(32 * qd) << 16) + p.a_col + 32u * s + 16u * hf, a16);
+            tmem_st_wait();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&full_a[s]);
         }
@@ -234,51 +240,60 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     grid_launch_dependents();
     const bool split = p.CS > 1;
     const int nchunks = p.TN / 32;
-    uint8_t* recv = base;  // reuses the stage ring once every CTA of the cluster is done
     if (warp >= 2) {
         if (!*abort_flag) {
             if (!mbar_wait_bounded(accum, 0, WAIT_NS)) fail();
         }
         tc_fence_after();
     }
-    if (split) cluster_sync();  // every CTA of the cluster has finished its main loop
 
     const int qd = warp & 3;
+    const int hf = (warp - 2) >> 2;   // epilogue warps of a quadrant take alternate 32-token chunks
     const int nl = 32 * qd + lane;
     const int ncol = n0 + nl;
-    if (warp >= 2 && !*abort_flag) {
-        if (split) {
-            for (int j = 0; j < nchunks; ++j) {
-                const int owner = j % p.CS;
-                if (owner == rank) continue;
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(32 * qd) << 16) + 32 * j, v);
-                tmem_ld_wait();
-                const int jl = j / p.CS;
-                const uint32_t dst = smem_u32(recv) + (uint32_t)((((rank * p.njl + jl) * 32) * BMW + nl) * 4);
-                const uint32_t rdst = map_shared_rank(dst, owner);
+    const uint32_t tm_row = tmem_d + ((uint32_t)(32 * qd) << 16);
+    // Split-K exchange.  Chunk j (32 tokens) of the tile is owned by rank j % CS.
+    // A slice in the workspace is 8 pieces x 128 columns x 16 bytes, so the 32
+    // threads of a warp write (and later read) 512 contiguous bytes per piece.
+    constexpr size_t CHUNK_U4 = CHUNK_BYTES / 16;
+    const size_t tile_slot = (size_t)(blockIdx.y * gridDim.x + blockIdx.x) * (size_t)p.CS;
+    if (split && warp >= 2 && !*abort_flag) {
+        uint4* mine = p.ws + (tile_slot + rank) * nchunks * CHUNK_U4;
+        for (int j = hf; j < nchunks; j += 2) {
+            if (j % p.CS == rank) continue;
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tm_row + 32 * j, v);
+            tmem_ld_wait();
+            uint4* dst = mine + (size_t)j * CHUNK_U4 + nl;
 #pragma unroll
-                for (int cc = 0; cc < 32; ++cc) st_shared_cluster_f32(rdst + cc * BMW * 4, __uint_as_float(v[cc]));
-            }
+            for (int pc = 0; pc < 8; ++pc)
+                __stcg(dst + pc * 128, make_uint4(v[4 * pc], v[4 * pc + 1], v[4 * pc + 2], v[4 * pc + 3]));
         }
     }
-    if (split) cluster_sync();  // all partial tiles have landed in their owners
+    if (split) cluster_sync();  // release / acquire: the slices above are visible to the owners
     if (warp >= 2 && !*abort_flag) {
-        for (int j = 0; j < nchunks; ++j) {
+        for (int j = hf; j < nchunks; j += 2) {
             if (split && (j % p.CS) != rank) continue;
             uint32_t v[32];
-            tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(32 * qd) << 16) + 32 * j, v);
+            tmem_ld_32x32b_x32(tm_row + 32 * j, v);
             tmem_ld_wait();
             float acc[32];
 #pragma unroll
             for (int cc = 0; cc < 32; ++cc) acc[cc] = __uint_as_float(v[cc]);
             if (split) {
-                const int jl = j / p.CS;
                 for (int src = 0; src < p.CS; ++src) {
                     if (src == rank) continue;
-                    const float* rb = reinterpret_cast<const float*>(recv) + ((src * p.njl + jl) * 32) * BMW + nl;
+                    const uint4* sp = p.ws + ((tile_slot + src) * nchunks + j) * CHUNK_U4 + nl;
+                    uint4 u[8];
 #pragma unroll
-                    for (int cc = 0; cc < 32; ++cc) acc[cc] += rb[cc * BMW];
+                    for (int pc = 0; pc < 8; ++pc) u[pc] = __ldcg(sp + pc * 128);
+#pragma unroll
+                    for (int pc = 0; pc < 8; ++pc) {
+                        acc[4 * pc] += __uint_as_float(u[pc].x);
+                        acc[4 * pc + 1] += __uint_as_float(u[pc].y);
+                        acc[4 * pc + 2] += __uint_as_float(u[pc].z);
+                        acc[4 * pc + 3] += __uint_as_float(u[pc].w);
+                    }
                 }
             }
             if (ncol < p.N) {
@@ -299,6 +314,39 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
 }
 
 // ------------------------------------------------------------------------ host
+// Tile plan shared by the launcher and the workspace query.
+struct Tiling {
+    int TN;      // tokens per tile, a multiple of 32, at most 256
+    int mt;      // token tiles
+    int ntiles;  // weight-column tiles
+    int CS;      // CTAs per cluster along K (1: no split)
+};
+
+size_t split_bytes(const Tiling& t, int CS) {
+    return (size_t)t.ntiles * t.mt * CS * (t.TN / 32) * CHUNK_BYTES;
+}
+
+// Splits K over up to 8 CTAs while the grid still fits the SMs once and each CTA
+// keeps at least two k blocks, as far as ws_bytes of workspace allows.
+Tiling plan(int M, int K, int N, size_t ws_bytes) {
+    Tiling t{};
+    t.mt = (M + 255) / 256;
+    const int tn = (M + t.mt - 1) / t.mt;
+    t.TN = std::max(32, (tn + 31) / 32 * 32);  // the epilogue reads tensor memory 32 columns at a time
+    t.ntiles = (N + BMW - 1) / BMW;
+    const int tiles = t.ntiles * t.mt;
+    const int KB = K / BK;
+    const int sms = sm_count();
+    t.CS = 1;
+    for (int c = 8; c >= 2; c >>= 1) {
+        if (KB % c == 0 && KB / c >= 2 && tiles * c <= sms && split_bytes(t, c) <= ws_bytes) {
+            t.CS = c;
+            break;
+        }
+    }
+    return t;
+}
+
 template <int BITS>
 wq_status run(const Problem& pb, cudaStream_t stream) {
     constexpr int EPS = Fmt<BITS>::EPS;
@@ -314,28 +362,17 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     else if (BK % pb.G == 0) p.GPB = BK / pb.G;
     else return WQ_ERR_UNSUPPORTED;
 
-    // token tile: balanced tiles of at most 256 tokens, multiple of 16
-    const int mt = (pb.M + 255) / 256;
-    int TN = (pb.M + mt - 1) / mt;
-    TN = std::max(32, (TN + 31) / 32 * 32);  // the epilogue reads tensor memory 32 columns at a time
+    // token tiles of at most 256 (balanced), K split over a cluster where it pays
+    const Tiling t = plan(pb.M, pb.K, pb.N, pb.ws ? pb.ws_bytes : 0);
+    const int TN = t.TN, mt = t.mt, ntiles = t.ntiles, CS = t.CS;
     p.TN = TN;
-    const int ntiles = (pb.N + BMW - 1) / BMW;
-    const int tiles = ntiles * mt;
-    const int KB = pb.K / BK;
-    const int sms = sm_count();
-    int CS = 1;
-    for (int c = 8; c >= 2; c >>= 1) {
-        if (KB % c == 0 && KB / c >= 2 && tiles * c <= sms) { CS = c; break; }
-    }
     p.CS = CS;
-    p.kb_cta = KB / CS;
-    p.tmem_cols = 32;
-    while ((int)p.tmem_cols < TN) p.tmem_cols <<= 1;
+    p.kb_cta = pb.K / BK / CS;
+    p.ws = static_cast<uint4*>(pb.ws);
 
     // stage layout: x tile | A tile | words | lo words | s rows | z rows (1024-aligned stage)
     const uint32_t xb = (uint32_t)TN * 128u;
-    p.off_a = (xb + 1023u) & ~1023u;
-    p.off_w = p.off_a + BMW * 128u;
+    p.off_w = (xb + 1023u) & ~1023u;
     p.off_lo = p.off_w + RW * BMW * 4u;
     p.off_s = p.off_lo + RL * BMW * 4u;
     p.off_z = p.off_s + p.GPB * BMW * 2u;
@@ -347,17 +384,21 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     int stages = (int)((limit - 1024 - bar_bytes) / p.stage_bytes);
     stages = std::min(stages, 6);
     stages = std::min(stages, std::max(2, p.kb_cta));
+    // tensor memory: the fp32 accumulator (TN columns), then 32 columns of fp16 A pairs per stage
+    p.a_col = (uint32_t)((TN + 31) / 32 * 32);
+    if (p.a_col + 32u * (uint32_t)stages > 512u) stages = (int)((512u - p.a_col) / 32u);
+    p.tmem_cols = 32;
+    while (p.tmem_cols < p.a_col + 32u * (uint32_t)stages) p.tmem_cols <<= 1;
     if (stages < 2) return WQ_ERR_UNSUPPORTED;
     p.stages = stages;
-    p.njl = (TN / 32 + CS - 1) / CS;
-    const size_t recv_bytes = (size_t)CS * p.njl * 32 * BMW * 4;
-    size_t ring = (size_t)stages * p.stage_bytes;
-    if (CS > 1 && recv_bytes > ring) ring = (recv_bytes + 1023) & ~(size_t)1023;
+    const size_t ring = (size_t)stages * p.stage_bytes;
     p.bar_off = (uint32_t)ring;
-    // At least 80 KB so that no more than two CTAs share an SM: two tensor-memory
-    // allocations of at most 256 columns always fit in the SM's 512 columns, so
-    // tcgen05.alloc never waits on a CTA of another cluster.
-    const size_t smem = std::max<size_t>(1024 + ring + bar_bytes, 80 * 1024);
+    // Enough shared memory that the CTAs resident on one SM never ask for more
+    // than the SM's 512 tensor-memory columns together, so tcgen05.alloc never
+    // waits on a CTA of another cluster: over 116 KB (one CTA per SM) when a CTA
+    // takes more than 256 columns, else at least 80 KB (at most two per SM).
+    const size_t smem_floor = p.tmem_cols > 256 ? 116 * 1024 : 80 * 1024;
+    const size_t smem = std::max<size_t>(1024 + ring + bar_bytes, smem_floor);
     if (smem > limit) return WQ_ERR_UNSUPPORTED;
 
     CUtensorMap mx, mw, ml, ms, mz;
@@ -419,6 +460,13 @@ wq_status launch_gemm(const Problem& p, cudaStream_t s) {
         case 8: return run<8>(p, s);
         default: return WQ_ERR_UNSUPPORTED;
     }
+}
+
+size_t gemm_workspace_bytes(int M, int K, int N, int bits, int G) {
+    (void)bits;
+    if (G % BK != 0 && BK % G != 0) return 0;
+    const Tiling t = plan(M, K, N, ~(size_t)0);
+    return t.CS > 1 ? split_bytes(t, t.CS) : 0;
 }
 
 wq_status gemm_device_status(int reset) {

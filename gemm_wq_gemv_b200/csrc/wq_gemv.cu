@@ -102,8 +102,6 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     const int g = lane >> 2, t = lane & 3;
     const int rank = (int)blockIdx.y;  // the cluster spans the grid's y extent
     const int col0 = blockIdx.x * COLS;
-    const int mycol = col0 + 4 * g;
-    const bool col_ok = mycol < p.N;
 
     const int cta_q0 = rank * p.WK * p.QW;
     const int q_begin = cta_q0 + warp * p.QW;

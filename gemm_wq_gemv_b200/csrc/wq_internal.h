@@ -19,6 +19,8 @@ struct Problem {
     uint16_t* y;
     int M, K, N, bits, G;  // G resolved: group_size == -1 -> K
     unsigned flags;
+    void* ws;              // wq_gemm split-K workspace (may be null)
+    size_t ws_bytes;
 };
 
 wq_status launch_pack(const uint8_t* codes, int K, int N, int bits, uint32_t* w_q, uint32_t* w_lo,
@@ -27,6 +29,7 @@ wq_status launch_unpack(const uint32_t* w_q, const uint32_t* w_lo, int K, int N,
                         uint8_t* codes, cudaStream_t s);
 wq_status launch_gemv(const Problem& p, cudaStream_t s);
 wq_status launch_gemm(const Problem& p, cudaStream_t s);
+size_t gemm_workspace_bytes(int M, int K, int N, int bits, int G);
 
 // Device status words (one per kernel file): nonzero once a bounded wait ran out.
 // Reading synchronises the device; reset clears the word.

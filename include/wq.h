@@ -43,6 +43,7 @@
 #ifndef WQ_H_
 #define WQ_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -119,15 +120,28 @@ wq_status wq_gemv(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
 /*
  * Batched product for any M >= 1 ("GPTQModel-Compatible Triton Kernel"
  * README, `gptqmodel_quantized_matmul`; dashq_kernel.py `forward`, batched
- * branch).  Same arguments as wq_gemv.  group_size: -1, or a positive divisor
- * of K that is a multiple of eps (3-bit: of 32).  Requires K % 64 == 0 and
- * N % 8 == 0.
- * Packed tiles are dequantised to fp16 in shared memory and multiplied on the
+ * branch).  Same arguments as wq_gemv, plus a workspace.  group_size: -1, or a
+ * positive divisor of K that is a multiple of eps (3-bit: of 32) and either a
+ * multiple or a divisor of 64.  Requires K % 64 == 0 and N % 8 == 0.
+ * Packed tiles are dequantised to fp16 into tensor memory and multiplied on the
  * tensor cores (tcgen05, fp32 accumulators in tensor memory).
+ *   workspace        device scratch for splitting K over the CTAs of a cluster
+ *                    (fp32 partial tiles, reduced through L2), owned by the
+ *                    caller; it needs no initialisation and keeps no state
+ *                    between calls.  Calls that may run at the same time on
+ *                    the device must not share one.
+ *   workspace_bytes  its size; with less than wq_gemm_workspace_size() (or
+ *                    NULL) the product is computed without splitting K, which
+ *                    is correct but uses fewer SMs for small M x N.
  */
 wq_status wq_gemm(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
                   const uint16_t* scales, const uint16_t* zeros, uint16_t* y,
-                  int M, int K, int N, int bits, int group_size, unsigned flags, void* stream);
+                  int M, int K, int N, int bits, int group_size, unsigned flags,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes wq_gemm uses for this shape (0 when it does not split K, or
+ * when the arguments are invalid).  Host-only; needs no device. */
+size_t wq_gemm_workspace_size(int M, int K, int N, int bits, int group_size);
 
 /*
  * Device-side status of the current device: WQ_OK, or WQ_ERR_TIMEOUT when a

@@ -40,7 +40,10 @@ P = 0x10000  # a 16-byte aligned fake device address: never dereferenced on the 
 
 
 def gemv(L, fn="wq_gemv", x=P, wq=P, wlo=None, s=P, z=P, y=P, M=1, K=512, N=256, bits=4, G=128,
-         flags=0):
+         flags=0, ws=None, ws_bytes=0):
+    if fn == "wq_gemm":
+        return L.wq_gemm(x, wq, wlo, s, z, y, M, K, N, bits, G, flags, ws, ctypes.c_size_t(ws_bytes),
+                         None)
     return getattr(L, fn)(x, wq, wlo, s, z, y, M, K, N, bits, G, flags, None)
 
 
@@ -77,6 +80,29 @@ def test_gemv_specific_limits(libwq):
     assert gemv(L, "wq_gemv", bits=4, G=16, K=512) == 2   # group not a multiple of 4*eps
     assert gemv(L, "wq_gemv", bits=1, G=64, K=512) == 2
     assert gemv(L, "wq_gemm", K=544, G=-1) == 1           # gemm needs K % 64
+    assert gemv(L, "wq_gemm", K=576, G=96) == 2           # group neither a multiple nor a divisor of 64
+    assert gemv(L, "wq_gemm", ws=P + 8, ws_bytes=1 << 20) == 3  # workspace alignment
+
+
+def test_gemm_workspace_size(libwq):
+    """The size query follows the tile plan: 128-column x (<= 256)-token tiles,
+    K split over 8, 4 or 2 CTAs while the grid fits the SMs once (148 SMs are
+    assumed without a device) and each CTA keeps two 64-deep k blocks; one
+    128 x 32 fp32 slice per CTA and 32-token chunk."""
+    import torch
+    L = libwq.lib()
+    size = lambda *a: int(L.wq_gemm_workspace_size(*a))
+    slice_bytes = 128 * 32 * 4
+    if not torch.cuda.is_available():
+        assert size(1, 4096, 4096, 4, 128) == 32 * 4 * 1 * slice_bytes       # 32 tiles x CS 4
+        assert size(512, 4096, 4096, 4, 128) == 64 * 2 * 8 * slice_bytes     # 64 tiles x CS 2
+        assert size(16, 1024, 1024, 4, 128) == 8 * 8 * 1 * slice_bytes       # KB 16: CS 8
+    assert size(512, 4096, 16384, 4, 128) == 0   # 256 tiles: no split
+    assert size(1, 128, 4096, 4, 128) == 0       # two k blocks: no split
+    assert size(0, 4096, 4096, 4, 128) == 0      # invalid arguments
+    assert size(1, 4096, 4096, 5, 128) == 0
+    assert size(1, 4000, 4096, 4, 128) == 0
+    assert size(1, 4096, 4096, 4, 96) == 0
 
 
 def test_pack_argument_checks(libwq):
