@@ -13,6 +13,7 @@ Entry points (same names as the C ABI, without the ``wq_`` prefix):
 * ``gemm(x, w_q, w_lo, scales, zeros, bits, group_size, out=None, pdl=False,
   workspace=None) -> y``
 * ``gemm_workspace_size(M, K, N, bits, group_size) -> bytes``
+* ``gemm_noalloc(x, w_q, w_lo, scales, zeros, bits, group_size, out) -> out``
 """
 from __future__ import annotations
 
@@ -30,6 +31,7 @@ STATUS = {
     4: "WQ_ERR_CODE_RANGE",
     5: "WQ_ERR_TIMEOUT",
     6: "WQ_ERR_CUDA",
+    7: "WQ_ERR_SCRATCH_LIMIT",
 }
 WQ_FLAG_PDL = 1
 
@@ -63,6 +65,8 @@ def lib() -> ctypes.CDLL:
         L.wq_gemm.argtypes = [p, p, p, p, p, p, i, i, i, i, i, u, p, ctypes.c_size_t, p]
         L.wq_gemm_workspace_size.argtypes = [i, i, i, i, i]
         L.wq_gemm_workspace_size.restype = ctypes.c_size_t
+        L.wq_gemm_noalloc.argtypes = [p, p, p, p, p, p, i, i, i, i, i, u, p]
+        L.wq_gemm_noalloc.restype = i
         L.wq_device_status.argtypes = [i]
         for f in ("wq_pack_kmajor", "wq_unpack_kmajor", "wq_gemv", "wq_gemm", "wq_device_status"):
             getattr(L, f).restype = i
@@ -222,3 +226,12 @@ def gemm(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl:
 def device_status(reset: bool = False) -> int:
     """``wq_device_status``: 0, or 5 (WQ_ERR_TIMEOUT) if a kernel gave up a bounded wait."""
     return int(lib().wq_device_status(1 if reset else 0))
+
+
+def gemm_noalloc(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out, pdl: bool = False):
+    """``wq_gemm_noalloc``: the product into the caller's ``out`` with the
+    library's fixed split-K scratch; neither the call nor this wrapper
+    allocates device memory."""
+    torch = _torch()
+    _need(out, torch.float16, "out")
+    return _product("wq_gemm_noalloc", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl)

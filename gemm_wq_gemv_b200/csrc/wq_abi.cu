@@ -84,6 +84,7 @@ const char* wq_status_string(wq_status s) {
         case WQ_ERR_CODE_RANGE: return "code does not fit in the bit width";
         case WQ_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
         case WQ_ERR_CUDA: return "CUDA runtime error";
+        case WQ_ERR_SCRATCH_LIMIT: return "shape needs more split-K scratch than the static array holds";
     }
     return "unknown status";
 }

@@ -59,7 +59,8 @@ typedef enum {
     WQ_ERR_ALIGNMENT = 3,     /* a pointer not 16-byte aligned, or N not a multiple of 8 */
     WQ_ERR_CODE_RANGE = 4,    /* a code >= 2^bits was found (reported by the bindings) */
     WQ_ERR_TIMEOUT = 5,       /* a kernel gave up a bounded wait (see wq_device_status) */
-    WQ_ERR_CUDA = 6           /* the CUDA runtime refused a launch or query */
+    WQ_ERR_CUDA = 6,          /* the CUDA runtime refused a launch or query */
+    WQ_ERR_SCRATCH_LIMIT = 7  /* the shape needs more split-K scratch than wq_gemm_noalloc holds */
 } wq_status;
 
 /*
@@ -142,6 +143,33 @@ wq_status wq_gemm(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
 /* Workspace bytes wq_gemm uses for this shape (0 when it does not split K, or
  * when the arguments are invalid).  Host-only; needs no device. */
 size_t wq_gemm_workspace_size(int M, int K, int N, int bits, int group_size);
+
+/*
+ * wq_gemm without a caller workspace, for callers that cannot allocate device
+ * memory when they call: a runtime that has handed all device memory to its
+ * own pool, or a plug-in whose host forbids allocation after initialisation
+ * (cudaMalloc also synchronises the device, which a per-token decode loop
+ * cannot afford).  The pages have no counterpart: their kernels take no
+ * workspace.
+ *
+ * Same arguments, rules and result as wq_gemm given a workspace of
+ * wq_gemm_workspace_size() bytes.  The split-K scratch is a fixed array of
+ * WQ_GEMM_NOALLOC_SCRATCH_BYTES in the library's device image, one per
+ * device, so the call allocates nothing.  Nothing in it needs to start at zero
+ * and no state is kept in it between calls.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Calls that may run at the same time on one device (other streams, other
+ *     host threads) share the array and race; calls in one stream do not.
+ *   - A shape whose wq_gemm_workspace_size() exceeds the array is rejected
+ *     with WQ_ERR_SCRATCH_LIMIT before anything is launched.
+ */
+#define WQ_GEMM_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+wq_status wq_gemm_noalloc(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
+                          const uint16_t* scales, const uint16_t* zeros, uint16_t* y,
+                          int M, int K, int N, int bits, int group_size, unsigned flags,
+                          void* stream);
 
 /*
  * Device-side status of the current device: WQ_OK, or WQ_ERR_TIMEOUT when a
