@@ -34,6 +34,7 @@ STATUS = {
     7: "WQ_ERR_SCRATCH_LIMIT",
 }
 WQ_FLAG_PDL = 1
+WQ_FLAG_PDL_INPUTS_READY = 2
 
 _lib = None
 
@@ -149,7 +150,8 @@ def unpack_kmajor(w_q, w_lo, K: int, bits: int):
     return out
 
 
-def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, workspace=False):
+def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, workspace=False,
+             inputs_ready=False):
     torch = _torch()
     _need(x, torch.float16, "x")
     _need(w_q, torch.int32, "w_q")
@@ -163,7 +165,7 @@ def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, worksp
         out = torch.empty((M, N), dtype=torch.float16, device=x.device)
     else:
         _need(out, torch.float16, "out")
-    flags = WQ_FLAG_PDL if pdl else 0
+    flags = (WQ_FLAG_PDL if pdl else 0) | (WQ_FLAG_PDL_INPUTS_READY if inputs_ready else 0)
     args = [_ptr(x), _ptr(w_q), _ptr(w_lo), _ptr(scales), _ptr(zeros), _ptr(out),
             M, K, N, bits, group_size, flags]
     if workspace is not False:  # wq_gemm: (workspace, bytes)
@@ -175,9 +177,14 @@ def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, worksp
     return out
 
 
-def gemv(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl: bool = False):
-    """y (M, N) fp16 = x (M, K) @ dequant(w_q), 1 <= M <= 16 (``wq_gemv``)."""
-    return _product("wq_gemv", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl)
+def gemv(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl: bool = False,
+         inputs_ready: bool = False):
+    """y (M, N) fp16 = x (M, K) @ dequant(w_q), 1 <= M <= 16 (``wq_gemv``).
+
+    ``pdl``: WQ_FLAG_PDL; ``inputs_ready``: WQ_FLAG_PDL_INPUTS_READY (the previous
+    kernel on the stream writes none of this call's inputs)."""
+    return _product("wq_gemv", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl,
+                    inputs_ready=inputs_ready)
 
 
 def gemm_workspace_size(M: int, K: int, N: int, bits: int, group_size: int) -> int:
@@ -211,7 +218,7 @@ def _cached_workspace(device, nbytes: int):
 
 
 def gemm(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl: bool = False,
-         workspace=None):
+         workspace=None, inputs_ready: bool = False):
     """y (M, N) fp16 = x (M, K) @ dequant(w_q), any M >= 1 (``wq_gemm``).
 
     ``workspace``: a CUDA uint8 tensor of at least ``gemm_workspace_size(...)``
@@ -220,7 +227,8 @@ def gemm(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl:
     if workspace is not None:
         torch = _torch()
         _need(workspace, torch.uint8, "workspace", ndim=1)
-    return _product("wq_gemm", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, workspace)
+    return _product("wq_gemm", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, workspace,
+                    inputs_ready=inputs_ready)
 
 
 def device_status(reset: bool = False) -> int:

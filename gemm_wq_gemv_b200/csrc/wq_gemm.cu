@@ -63,6 +63,7 @@ struct GemmParams {
     uint32_t tmem_cols;
     uint32_t bar_off;    // offset of the barrier block from the aligned base
     uint4* ws;           // split-K slices: [tile][rank][32-token chunk][16-byte piece][128 columns]
+    int late_wait;       // wait for the previous kernel only before writing the workspace / y
 };
 
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
@@ -130,7 +131,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
             prefetch_tmap(&tm_z);
             if constexpr (BITS == 3) prefetch_tmap(&tm_lo);
             const uint64_t pol_w = policy_evict_first();
-            grid_dependency_wait();
+            if (!p.late_wait) grid_dependency_wait();
             for (int kb = 0; kb < p.kb_cta; ++kb) {
                 const int s = kb % p.stages, r = kb / p.stages;
                 if (r > 0 && !mbar_wait_bounded(&empty[s], (r - 1) & 1, WAIT_NS)) { fail(); break; }
@@ -252,6 +253,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     const int nl = 32 * qd + lane;
     const int ncol = n0 + nl;
     const uint32_t tm_row = tmem_d + ((uint32_t)(32 * qd) << 16);
+    if (p.late_wait) grid_dependency_wait();  // the workspace and y may still be in use before this
     // Split-K exchange.  Chunk j (32 tokens) of the tile is owned by rank j % CS.
     // A slice in the workspace is 8 pieces x 128 columns x 16 bytes, so the 32
     // threads of a warp write (and later read) 512 contiguous bytes per piece.
@@ -369,6 +371,7 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     p.CS = CS;
     p.kb_cta = pb.K / BK / CS;
     p.ws = static_cast<uint4*>(pb.ws);
+    p.late_wait = (pb.flags & WQ_FLAG_PDL_INPUTS_READY) ? 1 : 0;
 
     // stage layout: x tile | A tile | words | lo words | s rows | z rows (1024-aligned stage)
     const uint32_t xb = (uint32_t)TN * 128u;
@@ -439,7 +442,7 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     attrs[na].val.clusterDim.y = 1;
     attrs[na].val.clusterDim.z = CS;
     ++na;
-    if (pb.flags & WQ_FLAG_PDL) {
+    if (pb.flags & (WQ_FLAG_PDL | WQ_FLAG_PDL_INPUTS_READY)) {
         attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attrs[na].val.programmaticStreamSerializationAllowed = 1;
         ++na;

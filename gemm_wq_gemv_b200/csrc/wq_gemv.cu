@@ -14,7 +14,9 @@
 //    x 32 columns (8 quads, 128-byte swizzle) into two shared-memory stages,
 //    completing on an mbarrier: the bytes in flight cost neither registers nor
 //    L1 request slots.  Lane (g, t) (g = lane / 4, t = lane % 4) then reads one
-//    16-byte vector per quad (4 adjacent columns of one word row).
+//    16-byte vector per quad (4 adjacent columns of one word row); the column
+//    chunk each lane reads is chosen so that these reads are free of bank
+//    conflicts.
 //  * Dequant.  A code pair (code j, code j + eps/2) sits at the same offset in
 //    the two 16-bit halves of a word: one LOP3 ORs both into the mantissa of
 //    fp16 1024 and one exact fp16x2 FMA gives the integers q - round(z).
@@ -63,6 +65,7 @@ struct Params {
     int qc_shift;  // log2(quads per CTA)
     int groups_cta;
     int nst;       // TMA stages per warp: 1 or 2
+    int late_wait; // wait for the previous kernel only before writing y
     int xs_tok_stride;  // bytes between tokens in the x stage (padded)
     uint32_t off_x, off_xq, off_tab, off_red, off_part, off_bar;  // smem byte offsets (stages at 0)
 };
@@ -100,6 +103,10 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
+    // 16-byte column chunk this lane reads (columns 4 cg .. 4 cg + 3): lanes g and
+    // g + 1 of a quarter-warp then differ in bit 2, which the row swizzle never
+    // touches, so each quarter-warp's eight 16-byte reads hit distinct banks.
+    const int cg = ((g & 1) << 2) | (g >> 1);
     const int rank = (int)blockIdx.y;  // the cluster spans the grid's y extent
     const int col0 = blockIdx.x * COLS;
 
@@ -116,11 +123,14 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     Rec<BITS>* tab = reinterpret_cast<Rec<BITS>*>(smem + p.off_tab);
     constexpr int TB = 2;
     bool any_frac = false;
+    // Record slot sl of a group holds column 4 (sl % 8) + sl / 8: the eight lanes
+    // reading one column offset c of their chunks then read consecutive records.
     auto tab_load = [&](int base, uint32_t (&v)[TB]) {
 #pragma unroll
         for (int u = 0; u < TB; ++u) {
             const int i = base + u * (int)blockDim.x + (int)threadIdx.x;
-            const int gg = g_cta0 + i / COLS, col = col0 + i % COLS;
+            const int sl = i % COLS;
+            const int gg = g_cta0 + i / COLS, col = col0 + 4 * (sl & 7) + (sl >> 3);
             v[u] = 0u;
             if (i < nrec && col < p.N && gg < n_groups) {
                 const size_t o = (size_t)gg * p.N + col;
@@ -147,10 +157,6 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
             }
         }
     };
-    // ---- (1) s, z first: these small loads then do not queue behind the weight stream
-    uint32_t tv[TB];
-    tab_load(0, tv);
-
     // ---- (2) weights: each warp streams its K range with 2-D TMA boxes of 32
     // word rows x 32 columns (8 quads, 128-byte swizzle) into nst stages
     const int nst = p.nst;
@@ -175,6 +181,11 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     // the next kernel on the stream may start now (it waits for this grid before reading its x)
     grid_launch_dependents();
 
+    // ---- (1) s, z (after the weight copies are issued: lane 0's mbarrier fence
+    // above would otherwise wait for these loads)
+    uint32_t tv[TB];
+    tab_load(0, tv);
+
     tab_store(0, tv);
     for (int base = TB * (int)blockDim.x; base < nrec; base += TB * (int)blockDim.x) {
         tab_load(base, tv);
@@ -184,7 +195,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     const bool frac = __syncthreads_or(any_frac) != 0;
 
     // ---- (3) x may come from the previous kernel on the stream: wait, then load it
-    grid_dependency_wait();
+    if (!p.late_wait) grid_dependency_wait();
 
     // x is staged per token in k-slot order: word row r holds the pairs
     // (x[r*EPS + j], x[r*EPS + j + EPS/2]), j < EPS/2.  A chunk is one word row
@@ -326,7 +337,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
         }
         // group bookkeeping without divisions in the loop
         int left = p.qpg - ((q_begin * QK) % p.G) / QK;  // quads left in the current group
-        uint32_t rc = smem_u32(tab) + RS * (uint32_t)(((q_begin * QK) / p.G - g_cta0) * COLS + 4 * g);
+        uint32_t rc = smem_u32(tab) + RS * (uint32_t)(((q_begin * QK) / p.G - g_cta0) * COLS + cg);
+        constexpr uint32_t CS8 = 8 * RS;  // record stride between the lane's columns
         // bias constants of the lane's 4 columns, in registers for narrow records
         constexpr bool CREG = NC <= 2;
         uint32_t creg[4][CREG ? NC : 1];
@@ -335,20 +347,20 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
 #pragma unroll
-                    for (int ci = 0; ci < NC; ++ci) creg[c][ci] = lds32_u32(rc + c * RS + 8 + 4 * ci);
+                    for (int ci = 0; ci < NC; ++ci) creg[c][ci] = lds32_u32(rc + c * CS8 + 8 + 4 * ci);
             }
         };
         if (nq > 0) load_creg();
         const uint32_t lo_sel = (t & 1) ? 0x7372u : 0x7170u;  // 3-bit: which half of the lo word
         // Per-lane offsets of this lane's 16-byte vector inside a stage: quad iq,
-        // word row R = 4 iq + t, 16-byte chunk g swizzled with (R & 7), whose
+        // word row R = 4 iq + t, 16-byte chunk cg swizzled with (R & 7), whose
         // value only depends on the parity of iq.
-        const uint32_t off_even = (uint32_t)t * 128 + (((uint32_t)g ^ (uint32_t)t) << 4);
-        const uint32_t off_odd = (uint32_t)t * 128 + (((uint32_t)g ^ (uint32_t)(t + 4)) << 4);
+        const uint32_t off_even = (uint32_t)t * 128 + (((uint32_t)cg ^ (uint32_t)t) << 4);
+        const uint32_t off_odd = (uint32_t)t * 128 + (((uint32_t)cg ^ (uint32_t)(t + 4)) << 4);
         // 3-bit lo plane: row R >> 1 = 2 iq + (t >> 1), swizzled with ((R >> 1) & 7)
         const uint32_t tl = (uint32_t)(t >> 1);
-        const uint32_t lo_off[4] = {tl * 128 + (((uint32_t)g ^ tl) << 4), tl * 128 + (((uint32_t)g ^ (tl + 2)) << 4),
-                                    tl * 128 + (((uint32_t)g ^ (tl + 4)) << 4), tl * 128 + (((uint32_t)g ^ (tl + 6)) << 4)};
+        const uint32_t lo_off[4] = {tl * 128 + (((uint32_t)cg ^ tl) << 4), tl * 128 + (((uint32_t)cg ^ (tl + 2)) << 4),
+                                    tl * 128 + (((uint32_t)cg ^ (tl + 4)) << 4), tl * 128 + (((uint32_t)cg ^ (tl + 6)) << 4)};
 
         auto quad = [&](uint32_t stage, int iq, int i) {
             const uint4 hv = lds128_u32(stage + 512 * iq + ((iq & 1) ? off_odd : off_even));
@@ -391,8 +403,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
                         cA[ci] = creg[ca][ci];
                         cB[ci] = creg[cb][ci];
                     } else {
-                        cA[ci] = lds32_u32(rc + ca * RS + 8 + 4 * ci);
-                        cB[ci] = lds32_u32(rc + cb * RS + 8 + 4 * ci);
+                        cA[ci] = lds32_u32(rc + ca * CS8 + 8 + 4 * ci);
+                        cB[ci] = lds32_u32(rc + cb * CS8 + 8 + 4 * ci);
                     }
                 }
                 uint32_t wA = wv[ca], wB = wv[cb], wAh = 0, wBh = 0, lA = 0, lB = 0;
@@ -414,8 +426,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
             if (--left == 0 || i == nq - 1) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const float sc = __uint_as_float(lds32_u32(rc + c * RS));
-                    const float zr = FRAC ? __uint_as_float(lds32_u32(rc + c * RS + 4)) : 0.0f;
+                    const float sc = __uint_as_float(lds32_u32(rc + c * CS8));
+                    const float zr = FRAC ? __uint_as_float(lds32_u32(rc + c * CS8 + 4)) : 0.0f;
                     const int T = c >> 1, half = c & 1;
 #pragma unroll
                     for (int n = 0; n < NT; ++n)
@@ -479,7 +491,9 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     else
         main_loop(std::false_type{});
 
-    // ---- reduce over the warps of the CTA
+    // ---- reduce over the warps of the CTA (and write y: with late_wait, only
+    // once the previous kernel on the stream has completed)
+    if (p.late_wait) grid_dependency_wait();
     float* red = reinterpret_cast<float*>(smem + p.off_red);  // [WK][M][COLS]
 #pragma unroll
     for (int c = 0; c < 4; ++c)
@@ -488,7 +502,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int m = tok[n][e];
-                if (m < p.M) red[(warp * p.M + m) * COLS + 4 * g + c] = acc[c][n][e];
+                if (m < p.M) red[(warp * p.M + m) * COLS + 4 * cg + c] = acc[c][n][e];
             }
     __syncthreads();
     float* part = reinterpret_cast<float*>(smem + p.off_part);  // [M][COLS]
@@ -539,6 +553,7 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     Params prm{};
     prm.x = pb.x; prm.w_q = pb.w_q; prm.w_lo = pb.w_lo; prm.s = pb.scales; prm.z = pb.zeros;
     prm.y = pb.y; prm.M = pb.M; prm.K = pb.K; prm.N = pb.N; prm.G = pb.G;
+    prm.late_wait = (pb.flags & WQ_FLAG_PDL_INPUTS_READY) ? 1 : 0;
     prm.Kw = pb.K / EPS;
     prm.Q = (prm.Kw + 3) / 4;
     prm.qpg = (pb.G == pb.K) ? (1 << 29) : pb.G / QK;
@@ -628,7 +643,7 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     attrs[na].val.clusterDim.y = best.CS;
     attrs[na].val.clusterDim.z = 1;
     ++na;
-    if (pb.flags & WQ_FLAG_PDL) {
+    if (pb.flags & (WQ_FLAG_PDL | WQ_FLAG_PDL_INPUTS_READY)) {
         attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attrs[na].val.programmaticStreamSerializationAllowed = 1;
         ++na;

@@ -58,21 +58,24 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// Shared-memory loads by address.  Not volatile, so the compiler may schedule
+// them freely against arithmetic; the "memory" clobber keeps them in order with
+// barriers, mbarrier waits and fences.
 __device__ __forceinline__ uint4 lds128_u32(uint32_t a) {
     uint4 r;
-    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(a));
+    asm("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(a) : "memory");
     return r;
 }
 
 __device__ __forceinline__ uint2 lds64_u32(uint32_t a) {
     uint2 r;
-    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(a));
+    asm("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(a) : "memory");
     return r;
 }
 
 __device__ __forceinline__ uint32_t lds32_u32(uint32_t a) {
     uint32_t r;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(a));
+    asm("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(a) : "memory");
     return r;
 }
 
@@ -136,7 +139,7 @@ __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
 // D(16x8, f32) = A(16x16, f16, row) * B(16x8, f16, col) + C.
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                           uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])

@@ -73,6 +73,15 @@ typedef enum {
  *   use it to overlap one product's weight reads with the previous product.
  */
 #define WQ_FLAG_PDL 1u
+/*
+ * WQ_FLAG_PDL_INPUTS_READY: like WQ_FLAG_PDL, but the kernel waits for the
+ *   previous kernel on the stream only before it writes y (and, for wq_gemm,
+ *   its workspace): it reads x as well as the weights at once.  So the previous
+ *   kernel must write none of x, w_q, w_lo, scales and zeros.  Independent
+ *   products that follow one another on a stream (projections of one
+ *   activation, expert weights of one token) use it to overlap completely.
+ */
+#define WQ_FLAG_PDL_INPUTS_READY 2u
 
 /* Version of this ABI (WQ_ABI_VERSION). */
 int wq_abi_version(void);

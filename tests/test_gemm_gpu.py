@@ -122,3 +122,40 @@ def test_rejected_calls(cuda, libwq):
     with pytest.raises(libwq.WQError) as e:   # K % 64 != 0
         libwq.gemm(d["x"], w_q, None, d["scales"], d["zeros"], 4, 32)
     assert e.value.status == 1
+
+
+def test_pdl_flags(cuda, libwq):
+    """WQ_FLAG_PDL on a chain where each x is the previous y, and
+    WQ_FLAG_PDL_INPUTS_READY on calls that overwrite the previous call's input
+    and output, give the same bits as plain calls."""
+    import torch
+    M, K = 96, 1024
+    case = wq_inputs.custom(M, K, K, 4, 128, seed=5)
+    d = to_dev(case, cuda)
+    w_q, w_lo = libwq.pack_kmajor(d["codes"], 4)
+    s = d["scales"] * 0.1
+
+    def chain(pdl):
+        ys, x = [], d["x"]
+        for _ in range(4):
+            x = libwq.gemm(x, w_q, w_lo, s, d["zeros"], 4, 128, pdl=pdl)
+            ys.append(x)
+        torch.cuda.synchronize()
+        return [y.cpu().numpy() for y in ys]
+
+    for a, b in zip(chain(False), chain(True)):
+        assert np.isfinite(a).all()
+        assert np.array_equal(a, b)
+
+    other = to_dev(wq_inputs.custom(M, K, K, 4, 128, seed=6), cuda)
+    w2, _ = libwq.pack_kmajor(other["codes"], 4)
+    ref0 = libwq.gemm(d["x"], w_q, None, s, d["zeros"], 4, 128).cpu().numpy()
+    ref1 = libwq.gemm(other["x"], w2, None, other["scales"], other["zeros"], 4, 128).cpu().numpy()
+    buf = d["x"].clone()
+    y0 = torch.empty((M, K), dtype=torch.float16, device=cuda)
+    libwq.gemm(buf, w_q, None, s, d["zeros"], 4, 128, out=y0)
+    libwq.gemm(other["x"], w2, None, other["scales"], other["zeros"], 4, 128, out=buf, inputs_ready=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(y0.cpu().numpy(), ref0)
+    assert np.array_equal(buf.cpu().numpy(), ref1)
+    assert libwq.device_status() == 0

@@ -114,6 +114,59 @@ def test_pdl_flag_same_result(cuda, libwq):
     assert np.array_equal(a, b)
 
 
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_pdl_chain_where_each_input_is_the_previous_output(cuda, libwq, M):
+    """WQ_FLAG_PDL: x of each call is y of the one before; the chain must give
+    the same bits as the same calls without the flag."""
+    import torch
+    K = N = 1024
+    case = wq_inputs.custom(M, K, N, 4, 128, seed=11)
+    d = to_dev(case, cuda)
+    w_q, w_lo = libwq.pack_kmajor(d["codes"], 4)
+    s = d["scales"] * 0.1  # keeps the chained values in range
+
+    def chain(pdl):
+        ys, x = [], d["x"]
+        for _ in range(4):
+            x = libwq.gemv(x, w_q, w_lo, s, d["zeros"], 4, 128, pdl=pdl)
+            ys.append(x)
+        torch.cuda.synchronize()
+        return [y.cpu().numpy() for y in ys]
+
+    for a, b in zip(chain(False), chain(True)):
+        assert np.isfinite(a).all()
+        assert np.array_equal(a, b)
+
+
+def test_inputs_ready_orders_the_writes_of_y(cuda, libwq):
+    """WQ_FLAG_PDL_INPUTS_READY: inputs are read at once, y is written only after
+    the previous kernel completes -- so a call may overwrite the previous call's
+    input (write after read) and its output (write after write)."""
+    import torch
+    cases = [wq_inputs.custom(4, 4096, 4096, 4, 128, seed=20 + i) for i in range(3)]
+    ds = [to_dev(c, cuda) for c in cases]
+    packed = [libwq.pack_kmajor(d["codes"], 4) for d in ds]
+    ref = [run_gemv(libwq, d, 4, 128) for d in ds]
+    buf = ds[0]["x"].clone()                       # call 0 reads buf ...
+    y0 = torch.empty((4, 4096), dtype=torch.float16, device=cuda)
+    out = torch.empty((4, 4096), dtype=torch.float16, device=cuda)
+    for _ in range(3):
+        buf.copy_(ds[0]["x"])
+        libwq.gemv(buf, packed[0][0], None, ds[0]["scales"], ds[0]["zeros"], 4, 128, out=y0)
+        # ... call 1 writes buf (its output, 4 x 4096 like x of call 0)
+        libwq.gemv(ds[1]["x"], packed[1][0], None, ds[1]["scales"], ds[1]["zeros"], 4, 128,
+                   out=buf, inputs_ready=True)
+        # calls 2 and 3 write the same output; the last one must win
+        libwq.gemv(ds[2]["x"], packed[2][0], None, ds[2]["scales"], ds[2]["zeros"], 4, 128,
+                   out=out, inputs_ready=True)
+        libwq.gemv(ds[1]["x"], packed[1][0], None, ds[1]["scales"], ds[1]["zeros"], 4, 128,
+                   out=out, inputs_ready=True)
+        torch.cuda.synchronize()
+        assert np.array_equal(y0.cpu().numpy(), ref[0])
+        assert np.array_equal(buf.cpu().numpy(), ref[1])
+        assert np.array_equal(out.cpu().numpy(), ref[1])
+
+
 def test_deterministic(cuda, libwq):
     case = wq_inputs.draw(wq_inputs.WORKLOADS["decode_gemv_m4"], seed=1)
     d = to_dev(case, cuda)
