@@ -56,6 +56,7 @@ struct GemmParams {
     int CS;              // CTAs per cluster along K
     int kb_cta;          // k blocks per CTA
     int GPB;             // s/z rows per stage
+    int g_shift;         // log2(G) when G < 64
     int stages;
     uint32_t stage_bytes, off_w, off_lo, off_s, off_z;
     uint32_t a_col;      // first tensor-memory column of the A stages (32 columns per stage)
@@ -132,38 +133,50 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
             if constexpr (BITS == 3) prefetch_tmap(&tm_lo);
             const uint64_t pol_w = policy_evict_first();
             if (!p.late_wait) grid_dependency_wait();
+            // stage slot, its use parity and the s/z row, advanced without divisions
+            int s = 0;
+            uint32_t ph = 0;
+            int kg = kb0 * BK;
+            int grow = kg / p.G, gnext = (grow + 1) * p.G;
             for (int kb = 0; kb < p.kb_cta; ++kb) {
-                const int s = kb % p.stages, r = kb / p.stages;
-                if (r > 0 && !mbar_wait_bounded(&empty[s], (r - 1) & 1, WAIT_NS)) { fail(); break; }
+                if (kb >= p.stages && !mbar_wait_bounded(&empty[s], ph ^ 1u, WAIT_NS)) { fail(); break; }
                 if (*abort_flag) break;
                 uint8_t* st = base + (size_t)s * p.stage_bytes;
-                const int kg = (kb0 + kb) * BK;
                 mbar_arrive_expect_tx(&full_tma[s], p.tx_bytes);
                 tma_load_2d(st, &tm_x, &full_tma[s], kg, m0);
                 tma_load_2d_hint(st + p.off_w, &tm_w, &full_tma[s], n0, kg / EPS, pol_w);
                 if constexpr (BITS == 3) tma_load_2d_hint(st + p.off_lo, &tm_lo, &full_tma[s], n0, kg / 32, pol_w);
-                const int grow = kg / p.G;
                 tma_load_2d(st + p.off_s, &tm_s, &full_tma[s], n0, grow);
                 tma_load_2d(st + p.off_z, &tm_z, &full_tma[s], n0, grow);
+                kg += BK;
+                if (p.GPB == 1) {  // a group spans whole k blocks: next row once kg reaches it
+                    if (kg >= gnext) { ++grow; gnext += p.G; }
+                } else {           // 64 / G rows per k block
+                    grow += p.GPB;
+                }
+                if (++s == p.stages) { s = 0; ph ^= 1u; }
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t idesc = (1u << 4) | ((uint32_t)(p.TN >> 3) << 17) | (8u << 24);
+            int s = 0;
+            uint32_t ph = 0;
+            const uint64_t bdesc0 = sw128_desc(smem_u32(base));
+            const uint64_t bstep = (uint64_t)(p.stage_bytes >> 4);  // descriptor address units
             for (int kb = 0; kb < p.kb_cta; ++kb) {
-                const int s = kb % p.stages, r = kb / p.stages;
-                if (!mbar_wait_bounded(&full_tma[s], r & 1, WAIT_NS)) { fail(); break; }
-                if (!mbar_wait_bounded(&full_a[s], r & 1, WAIT_NS)) { fail(); break; }
-                if (*abort_flag) break;
+                // the dequantising warps arrive on full_a only after they saw full_tma complete
+                if (!mbar_wait_bounded(&full_a[s], ph, WAIT_NS)) { fail(); break; }
+                if (!mbar_wait_bounded(&full_tma[s], ph, WAIT_NS)) { fail(); break; }
                 tc_fence_after();
-                const uint32_t st = smem_u32(base + (size_t)s * p.stage_bytes);
-                const uint64_t bdesc = sw128_desc(st);
+                const uint64_t bdesc = bdesc0 + bstep * (uint64_t)s;
                 const uint32_t a_tm = tmem_d + p.a_col + 32u * s;  // lane 0, this stage's A columns
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk)
                     tc_mma_f16_ts(tmem_d, a_tm + 8 * kk, bdesc + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(&empty[s]);
+                if (++s == p.stages) { s = 0; ph ^= 1u; }
             }
             tc_commit(accum);
         }
@@ -202,9 +215,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
             zs2 = dup_half(-(zv - zi) * sv);
         };
 
+        int s = 0;
+        uint32_t ph = 0;
         for (int kb = 0; kb < p.kb_cta; ++kb) {
-            const int s = kb % p.stages, r = kb / p.stages;
-            if (!mbar_wait_bounded(&full_tma[s], r & 1, WAIT_NS)) { fail(); break; }
+            if (!mbar_wait_bounded(&full_tma[s], ph, WAIT_NS)) { fail(); break; }
             if (*abort_flag) break;
             const uint8_t* st = base + (size_t)s * p.stage_bytes;
             uint32_t c[NC], s2, zs2;
@@ -218,7 +232,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
 #pragma unroll
                 for (int u = 0; u < RH; ++u) {
                     const int rw = hf * RH + u;
-                    const int gi = (rw * EPS) / p.G;
+                    const int gi = (rw * EPS) >> p.g_shift;  // G divides 64: a power of two
                     if (gi != cur) {
                         cur = gi;
                         consts(st, gi, c, s2, zs2);
@@ -232,6 +246,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&full_a[s]);
+            if (++s == p.stages) { s = 0; ph ^= 1u; }
         }
     }
 
@@ -261,8 +276,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     const size_t tile_slot = (size_t)(blockIdx.y * gridDim.x + blockIdx.x) * (size_t)p.CS;
     if (split && warp >= 2 && !*abort_flag) {
         uint4* mine = p.ws + (tile_slot + rank) * nchunks * CHUNK_U4;
-        for (int j = hf; j < nchunks; j += 2) {
+        // this CTA's non-owned chunks, alternately to the two warps of the quadrant
+        for (int j = 0, sidx = 0; j < nchunks; ++j) {
             if (j % p.CS == rank) continue;
+            if ((sidx++ & 1) != hf) continue;
             uint32_t v[32];
             tmem_ld_32x32b_x32(tm_row + 32 * j, v);
             tmem_ld_wait();
@@ -274,8 +291,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     }
     if (split) cluster_sync();  // release / acquire: the slices above are visible to the owners
     if (warp >= 2 && !*abort_flag) {
-        for (int j = hf; j < nchunks; j += 2) {
-            if (split && (j % p.CS) != rank) continue;
+        // owned chunks j = rank + CS i (every chunk without a split), alternately per warp half
+        for (int j = (split ? rank : 0) + hf * p.CS; j < nchunks; j += 2 * p.CS) {
             uint32_t v[32];
             tmem_ld_32x32b_x32(tm_row + 32 * j, v);
             tmem_ld_wait();
@@ -363,6 +380,8 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     if (pb.G % BK == 0) p.GPB = 1;
     else if (BK % pb.G == 0) p.GPB = BK / pb.G;
     else return WQ_ERR_UNSUPPORTED;
+    p.g_shift = 0;
+    while ((1 << (p.g_shift + 1)) <= pb.G && p.g_shift < 6) ++p.g_shift;
 
     // token tiles of at most 256 (balanced), K split over a cluster where it pays
     const Tiling t = plan(pb.M, pb.K, pb.N, pb.ws ? pb.ws_bytes : 0);
