@@ -4,8 +4,10 @@
 Headline workload: the decode GEMV y (1 x 4096) = x (1 x 4096) @ dequant(W_q),
 W_q 4-bit K-major words, group 128, fp16 scales and zero points.  One *step*
 is one decode pass over a stack of L distinct weight sets of that shape (each
-with its own x), launched back to back as programmatic dependents and replayed
-as one CUDA graph.  The stack's weights exceed twice the L2 size, so every
+with its own x and y: independent products, as the projections of one token),
+launched back to back with WQ_FLAG_PDL_INPUTS_READY and replayed as one CUDA
+graph.  ``chained`` reports the same stack run as a dependency chain (each x
+is the previous y, WQ_FLAG_PDL).  The stack's weights exceed twice the L2 size, so every
 launch reads its words from HBM.  ``value`` is the algorithmic HBM bytes of
 the products (packed words + s + z + x + y) per second, whole job.
 
@@ -156,10 +158,19 @@ class Stack:
                               s.clone() if i else s, z.clone() if i else z, y))
         self.np = np
 
-    def run(self, wq, fn, pdl):
+    def run(self, wq, fn, pdl=False, inputs_ready=False):
         wl = self.wl
         for (x, a, b, s, z, y) in self.sets:
-            fn(x, a, b, s, z, wl.bits, wl.group_size, out=y, pdl=pdl)
+            fn(x, a, b, s, z, wl.bits, wl.group_size, out=y, pdl=pdl, inputs_ready=inputs_ready)
+
+    def run_chain(self, wq):
+        """Each product's x is the previous product's y (square K = N): a true
+        dependency chain, launched with WQ_FLAG_PDL."""
+        wl = self.wl
+        x = self.sets[0][0]
+        for (_, a, b, s, z, y) in self.sets:
+            wq.gemv(x, a, b, s, z, wl.bits, wl.group_size, out=y, pdl=True)
+            x = y
 
 
 def time_graph(torch, graph, stream, steps, warmup, barrier=None, sampler=None):
@@ -262,6 +273,26 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------------ profiler case
+def run_case(name: str, reps: int) -> int:
+    """Launch one workload's product `reps` times on one weight set, untimed: the
+    command the profiler summaries under profiles/ capture."""
+    import torch
+    from gemm_wq_gemv_b200 import build as wq_build
+    wq_build.build()
+    import gemm_wq_gemv_b200 as wq
+    dev = torch.device("cuda", 0)
+    wl = wq_inputs.WORKLOADS[name]
+    stack = Stack(wq, torch, wl, 1, dev)
+    fn = wq.gemv if wl.M <= 16 else wq.gemm
+    for _ in range(reps):
+        stack.run(wq, fn)
+    torch.cuda.synchronize()
+    assert wq.device_status() == 0
+    print(json.dumps({"case": name, "reps": reps, "kernel": "gemv" if fn is wq.gemv else "gemm"}))
+    return 0
+
+
 # ------------------------------------------------------------------ GPU arm
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
@@ -271,11 +302,16 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["wq", "reference"], default="wq")
     ap.add_argument("--no-secondary", action="store_true", help="skip the per-workload table")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ncu-case", metavar="WORKLOAD", default=None,
+                    help="only launch WORKLOAD's kernel --reps times, untimed (for profiler captures)")
+    ap.add_argument("--reps", type=int, default=6)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.ncu_case:
+        return run_case(args.ncu_case, args.reps)
 
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -312,7 +348,7 @@ def main(argv=None):
     wl = wq_inputs.WORKLOADS[HEADLINE]
     L = layers_for(wl, L2)
     stack = Stack(wq, torch, wl, L, dev)
-    g, s = capture(torch, lambda: stack.run(wq, wq.gemv, True))
+    g, s = capture(torch, lambda: stack.run(wq, wq.gemv, inputs_ready=True))
     sampler = ClockSampler(local)
     el = time_graph(torch, g, s, args.steps, args.warmup, barrier, sampler)
     el = max_over_ranks(el)
@@ -320,7 +356,18 @@ def main(argv=None):
     value = bytes_step * args.steps * world / el / 1e9
     per_launch_s = el / (args.steps * L)
     achieved = algo_bytes(wl) / per_launch_s / 1e9
-    traffic = ncu_traffic("gemv_kernel<4, 1>", HEADLINE)
+    traffic = ncu_traffic("gemv_kernel<4,_1>", HEADLINE)
+
+    # ---- the same stack as a dependency chain (x of each product = y of the previous)
+    cg, cs = capture(torch, lambda: stack.run_chain(wq))
+    c_steps = max(3, min(args.steps, 500))
+    c_el = max_over_ranks(time_graph(torch, cg, cs, c_steps, args.warmup, barrier))
+    c_launch_s = c_el / (c_steps * L)
+    chained = {"us_per_launch": round(c_launch_s * 1e6, 3),
+               "GBps": round(algo_bytes(wl) / c_launch_s / 1e9, 1),
+               "frac": round(algo_bytes(wl) / c_launch_s / 1e9 / hbm_peak, 4),
+               "how": "same stack, x of each product = y of the previous, WQ_FLAG_PDL (wait before reading x)"}
+    del cg
 
     # ---- e2e: the same stack through the API with host buffers
     xs_host = torch.empty((L, wl.M, wl.K), dtype=torch.float16, pin_memory=True)
@@ -334,7 +381,7 @@ def main(argv=None):
     def e2e_step():
         xs_dev.copy_(xs_host, non_blocking=True)
         for i, (x, a, b, sc, z, y) in enumerate(stack.sets):
-            wq.gemv(xs_dev[i], a, b, sc, z, wl.bits, wl.group_size, out=ys_dev[i])
+            wq.gemv(xs_dev[i], a, b, sc, z, wl.bits, wl.group_size, out=ys_dev[i], inputs_ready=True)
         ys_host.copy_(ys_dev, non_blocking=True)
         torch.cuda.current_stream().synchronize()
 
@@ -352,11 +399,12 @@ def main(argv=None):
     gwl = wq_inputs.WORKLOADS[GEMM_WL]
     GL = layers_for(gwl, L2)
     gstack = Stack(wq, torch, gwl, GL, dev)
-    gg, gs = capture(torch, lambda: gstack.run(wq, wq.gemm, False))
+    gg, gs = capture(torch, lambda: gstack.run(wq, wq.gemm, inputs_ready=True))
     gsteps = max(3, min(args.steps, 200))
     gel = max_over_ranks(time_graph(torch, gg, gs, gsteps, args.warmup, barrier))
     g_launch_s = gel / (gsteps * GL)
     g_tflops = algo_flops(gwl) / g_launch_s / 1e12
+    g_traffic = ncu_traffic("gemm_kernel<4>", GEMM_WL)
     del gstack, gg
 
     # ---- every workload once (rank-local, for the table)
@@ -366,7 +414,7 @@ def main(argv=None):
             fn = wq.gemm if w.M > 16 else wq.gemv
             n_l = layers_for(w, L2)
             stk = Stack(wq, torch, w, n_l, dev)
-            gr, st_ = capture(torch, lambda: stk.run(wq, fn, fn is wq.gemv))
+            gr, st_ = capture(torch, lambda: stk.run(wq, fn, inputs_ready=True))
             reps = 20
             t = time_graph(torch, gr, st_, reps, 3)
             us = t / (reps * n_l) * 1e6
@@ -398,7 +446,8 @@ def main(argv=None):
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: {bytes_step / 1e6:.0f} MB of distinct weights per step "
                          f"> 2 x {L2 / 1e6:.0f} MB L2",
-                   "launch": "one CUDA graph per step, programmatic dependent launches"},
+                   "launch": "one CUDA graph per step; independent products launched with "
+                             "WQ_FLAG_PDL_INPUTS_READY (each waits for the previous only before writing y)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
@@ -406,13 +455,14 @@ def main(argv=None):
         "gemm": {"workload": "M=512 K=4096 N=2048 4-bit g128", "TFLOPS": round(g_tflops, 1),
                  "us": round(g_launch_s * 1e6, 3),
                  "roofline": {"bound": "tensor", "achieved": round(g_tflops, 1), "peak": tf_peak, "unit": "TFLOP/s",
-                              "frac": round(g_tflops / tf_peak, 4),
+                              "frac": round(g_tflops / tf_peak, 4), "traffic": g_traffic,
                               "peak_source": "measured bf16 burst (fp16 nominal ratio 1:1)"},
                  "l2": f"{GL} rotating input sets ({algo_bytes(gwl) * GL / 1e6:.0f} MB) per graph"},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": L * wl.M * wl.K * 2, "d2h_bytes_per_step": L * wl.M * wl.N * 2,
                 "how": "python API per layer (wq.gemv), x copied in from pinned host memory and y copied "
                        "back every step; weights resident"},
+        "chained": chained,
         "clocks": sampler.report(),
         "gpu_launches": args.steps * L * world,
         "workloads": table,
