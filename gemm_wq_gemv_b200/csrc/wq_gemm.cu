@@ -102,7 +102,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&full_tma[s], 1);
-            mbar_init(&full_a[s], NDQ);
+            mbar_init(&full_a[s], NDQ / 2);  // the four warps of the half that dequantises stage s
             mbar_init(&empty[s], 1);
         }
         mbar_init(accum, 1);
@@ -181,11 +181,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
             tc_commit(accum);
         }
     } else {
-        // ----------------------- dequantisation: a column per thread, half of its words per warp
+        // ----------------------- dequantisation: a column per thread; the two warps of a
+        // TMEM lane quadrant take alternate stages, all of a stage's word rows each
         const int qd = warp & 3;                 // TMEM lane quadrant this warp may read
-        const int hf = (warp - 2) >> 2;          // which half of the stage's word rows
+        const int hf = (warp - 2) >> 2;          // this warp takes the k blocks with kb % 2 == hf
         const int nl = 32 * qd + lane;           // weight column within the tile
-        constexpr int RH = RW / 2;               // word rows per half (RW >= 2 for every width)
         const uint32_t lo_sel0 = 0x7170u, lo_sel1 = 0x7372u;
 
         // (q - z) * s for word row rw of this column, in k order, into out[0 .. EPS/2)
@@ -218,34 +218,35 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
         int s = 0;
         uint32_t ph = 0;
         for (int kb = 0; kb < p.kb_cta; ++kb) {
-            if (!mbar_wait_bounded(&full_tma[s], ph, WAIT_NS)) { fail(); break; }
-            if (*abort_flag) break;
-            const uint8_t* st = base + (size_t)s * p.stage_bytes;
-            uint32_t c[NC], s2, zs2;
-            uint32_t a16[16];  // this thread's 32 k values (16 fp16 pairs) of the stage's A row
-            if (p.GPB == 1) {  // one group covers the whole k block
-                consts(st, 0, c, s2, zs2);
+            if ((kb & 1) == hf) {
+                if (!mbar_wait_bounded(&full_tma[s], ph, WAIT_NS)) { fail(); break; }
+                if (*abort_flag) break;
+                const uint8_t* st = base + (size_t)s * p.stage_bytes;
+                uint32_t c[NC], s2, zs2;
+                uint32_t a32[32];  // this thread's 64 k values (32 fp16 pairs) of the stage's A row
+                if (p.GPB == 1) {  // one group covers the whole k block
+                    consts(st, 0, c, s2, zs2);
 #pragma unroll
-                for (int u = 0; u < RH; ++u) word(st, hf * RH + u, c, s2, zs2, a16 + u * (EPS / 2));
-            } else {
-                int cur = -1;
+                    for (int rw = 0; rw < RW; ++rw) word(st, rw, c, s2, zs2, a32 + rw * (EPS / 2));
+                } else {
+                    int cur = -1;
 #pragma unroll
-                for (int u = 0; u < RH; ++u) {
-                    const int rw = hf * RH + u;
-                    const int gi = (rw * EPS) >> p.g_shift;  // G divides 64: a power of two
-                    if (gi != cur) {
-                        cur = gi;
-                        consts(st, gi, c, s2, zs2);
+                    for (int rw = 0; rw < RW; ++rw) {
+                        const int gi = (rw * EPS) >> p.g_shift;  // G divides 64: a power of two
+                        if (gi != cur) {
+                            cur = gi;
+                            consts(st, gi, c, s2, zs2);
+                        }
+                        word(st, rw, c, s2, zs2, a32 + rw * (EPS / 2));
                     }
-                    word(st, rw, c, s2, zs2, a16 + u * (EPS / 2));
                 }
+                // A row of weight column nl = tensor-memory lane nl; k pairs along the columns
+                tmem_st_32x32b_x32(tmem_d + ((uint32_t)(32 * qd) << 16) + p.a_col + 32u * s, a32);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full_a[s]);
             }
-            // A row of weight column nl = tensor-memory lane nl; k pairs along the columns
-            tmem_st_32x32b_x16(tmem_d + ((uint32_t)(32 * qd) << 16) + p.a_col + 32u * s + 16u * hf, a16);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&full_a[s]);
             if (++s == p.stages) { s = 0; ph ^= 1u; }
         }
     }
