@@ -61,6 +61,8 @@ struct Params {
     int WK;        // warps per CTA
     int CS;        // CTAs per cluster (along K)
     int qpg;       // quads per group (a large number when one group spans K)
+    int qpg_shift; // log2(qpg) when qpg is a power of two, else -1
+    int n_groups;  // ceil(K / G)
     int cpt_shift; // log2(x chunks per token staged by a CTA)
     int qc_shift;  // log2(quads per CTA)
     int groups_cta;
@@ -68,6 +70,10 @@ struct Params {
     int late_wait; // wait for the previous kernel only before writing y
     int xs_tok_stride;  // bytes between tokens in the x stage (padded)
     uint32_t off_x, off_xq, off_tab, off_red, off_part, off_bar;  // smem byte offsets (stages at 0)
+    uint32_t off_sz;  // raw s rows then z rows of the CTA's groups (sz_rows x COLS fp16 each)
+    int sz_rows;      // rows loaded per tile: sz_box x sz_nbox >= groups_cta
+    int sz_box;       // rows per TMA box (<= 256)
+    uint32_t sz_stride;  // bytes from the s tile to the z tile (128-byte multiple)
 };
 
 // bytes of one stage: 32 x 32 words of the main plane (+ 16 x 32 lo-plane words)
@@ -89,7 +95,8 @@ __device__ __forceinline__ float sum_warps(const float* red, int wk, int stride,
 
 template <int BITS, int NT>
 __global__ void __launch_bounds__(MAXW * 32, (NT == 1 && BITS != 1) ? 2 : 1)
-gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_lo, const Params p) {
+gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_lo,
+            const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_z, const Params p) {
     using F = Fmt<BITS>;
     constexpr int EPS = F::EPS;
     constexpr int NC = F::NC;
@@ -116,45 +123,33 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     const int nq = max(0, q_end - q_begin);
 
     // ---- s, z of the CTA's (group, column) records
-    const int k_cta0 = cta_q0 * QK;
-    const int g_cta0 = min(k_cta0, p.K - 1) / p.G;
-    const int n_groups = (p.K + p.G - 1) / p.G;
+    // group of quad q (G = qpg * QK): a shift for the usual power-of-two group sizes
+    auto gdiv = [&](int q) { return p.qpg_shift >= 0 ? (q >> p.qpg_shift) : q / p.qpg; };
+    const int g_cta0 = gdiv(min(cta_q0, p.Q - 1));
+    const int n_groups = p.n_groups;
     const int nrec = p.groups_cta * COLS;
     Rec<BITS>* tab = reinterpret_cast<Rec<BITS>*>(smem + p.off_tab);
-    constexpr int TB = 2;
     bool any_frac = false;
     // Record slot sl of a group holds column 4 (sl % 8) + sl / 8: the eight lanes
     // reading one column offset c of their chunks then read consecutive records.
-    auto tab_load = [&](int base, uint32_t (&v)[TB]) {
+    // Built from the raw s and z tiles that one TMA copy brought in (columns or
+    // groups outside the matrix read as 0: s = 0 and z = 0).
+    const uint16_t* s_raw = reinterpret_cast<const uint16_t*>(smem + p.off_sz);
+    const uint16_t* z_raw = reinterpret_cast<const uint16_t*>(smem + p.off_sz + p.sz_stride);
+    auto tab_build = [&]() {
+        for (int i = threadIdx.x; i < nrec; i += blockDim.x) {
+            const int sl = i & (COLS - 1);
+            const int o = (i & ~(COLS - 1)) + 4 * (sl & 7) + (sl >> 3);
+            const float sv = __half2float(__ushort_as_half(s_raw[o]));
+            const float zv = __half2float(__ushort_as_half(z_raw[o]));
+            const float zi = fminf(fmaxf(rintf(zv), -256.0f), 256.0f);
+            Rec<BITS> rec;
+            rec.s = sv;
+            rec.zr = zv - zi;
+            any_frac |= (rec.zr != 0.0f);
 #pragma unroll
-        for (int u = 0; u < TB; ++u) {
-            const int i = base + u * (int)blockDim.x + (int)threadIdx.x;
-            const int sl = i % COLS;
-            const int gg = g_cta0 + i / COLS, col = col0 + 4 * (sl & 7) + (sl >> 3);
-            v[u] = 0u;
-            if (i < nrec && col < p.N && gg < n_groups) {
-                const size_t o = (size_t)gg * p.N + col;
-                v[u] = (uint32_t)p.s[o] | ((uint32_t)p.z[o] << 16);
-            }
-        }
-    };
-    auto tab_store = [&](int base, const uint32_t (&v)[TB]) {
-#pragma unroll
-        for (int u = 0; u < TB; ++u) {
-            const int i = base + u * (int)blockDim.x + (int)threadIdx.x;
-            if (i < nrec) {
-                // a column or group outside the matrix gets s = 0 and z = 0
-                const float s = __half2float(__ushort_as_half((uint16_t)(v[u] & 0xffffu)));
-                const float z = __half2float(__ushort_as_half((uint16_t)(v[u] >> 16)));
-                const float zi = fminf(fmaxf(rintf(z), -256.0f), 256.0f);
-                Rec<BITS> rec;
-                rec.s = s;
-                rec.zr = z - zi;
-                any_frac |= (rec.zr != 0.0f);
-#pragma unroll
-                for (int ci = 0; ci < NC; ++ci) rec.c[ci] = dup_half(-(bias_magnitude<BITS>(ci) + zi));
-                tab[i] = rec;
-            }
+            for (int ci = 0; ci < NC; ++ci) rec.c[ci] = dup_half(-(bias_magnitude<BITS>(ci) + zi));
+            tab[i] = rec;
         }
     };
     // ---- (2) weights: each warp streams its K range with 2-D TMA boxes of 32
@@ -170,32 +165,27 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
         tma_load_2d_u32(dst, &tm_w, &bar[slot], col0, 4 * (q_begin + k * SQ));
         if constexpr (BITS == 3) tma_load_2d_u32(dst + 4096, &tm_lo, &bar[slot], col0, 2 * (q_begin + k * SQ));
     };
+    uint64_t* bar_sz = reinterpret_cast<uint64_t*>(smem + p.off_bar) + p.WK * MAXST;
     if (lane == 0) {
 #pragma unroll
         for (int k = 0; k < MAXST; ++k) mbar_init(&bar[k], 1);
+        if (warp == 0) mbar_init(bar_sz, 1);
         fence_mbarrier_init();
         prefetch_tmap(&tm_w);
+        if (warp == 0) {  // ---- (1) the raw s and z rows of the CTA's groups, first in line
+            const int nbox = p.sz_rows / p.sz_box;
+            mbar_arrive_expect_tx(bar_sz, (uint32_t)(2 * p.sz_rows * COLS * 2));
+            for (int b = 0; b < nbox; ++b) {
+                const uint32_t d = smem_u32(smem + p.off_sz) + (uint32_t)(b * p.sz_box * COLS * 2);
+                tma_load_2d_u32(d, &tm_s, bar_sz, col0, g_cta0 + b * p.sz_box);
+                tma_load_2d_u32(d + p.sz_stride, &tm_z, bar_sz, col0, g_cta0 + b * p.sz_box);
+            }
+        }
         for (int k = 0; k < nst && k < nst_w; ++k) issue(k);
     }
-    __syncwarp();
+    __syncthreads();  // every mbarrier above is initialised before anyone waits on it
     // the next kernel on the stream may start now (it waits for this grid before reading its x)
     grid_launch_dependents();
-
-    // ---- (1) s, z (after the weight copies are issued: lane 0's mbarrier fence
-    // above would otherwise wait for these loads)
-    uint32_t tv[TB];
-    tab_load(0, tv);
-
-    tab_store(0, tv);
-    for (int base = TB * (int)blockDim.x; base < nrec; base += TB * (int)blockDim.x) {
-        tab_load(base, tv);
-        tab_store(base, tv);
-    }
-    // fractional zero points anywhere in this CTA's records?  (CTA-uniform)
-    const bool frac = __syncthreads_or(any_frac) != 0;
-
-    // ---- (3) x may come from the previous kernel on the stream: wait, then load it
-    if (!p.late_wait) grid_dependency_wait();
 
     // x is staged per token in k-slot order: word row r holds the pairs
     // (x[r*EPS + j], x[r*EPS + j + EPS/2]), j < EPS/2.  A chunk is one word row
@@ -263,12 +253,32 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
             }
         }
     };
+    auto stage_x = [&]() {
     for (int base = 0; base < nchunk; base += XB * (int)blockDim.x) {
         uint4 xv[XB][UPC];
         x_load(base, xv);
         x_store(base, xv);
     }
-    __syncthreads();
+    };
+    auto table = [&]() {
+        const bool good = mbar_wait_bounded(bar_sz, 0, WAIT_NS);
+        if (!good) atomicExch(&g_gemv_status, 1u);
+        if (good) tab_build();
+    };
+    // ---- (3) the records, and x.  x may come from the previous kernel on the
+    // stream (WQ_FLAG_PDL): build the records while that kernel runs, then wait.
+    // Without that dependency stage x first, while the s/z copy lands.
+    if (!p.late_wait) {
+        table();
+        grid_dependency_wait();
+        stage_x();
+    } else {
+        stage_x();
+        table();
+    }
+    // fractional zero points anywhere in this CTA's records?  (CTA-uniform; the
+    // barrier also publishes the staged x and the records)
+    const bool frac = __syncthreads_or(any_frac) != 0;
 
     // ---- (4) per-quad x sums (fp32), only needed for fractional zero points
     const int quads_cta = 1 << p.qc_shift;
@@ -336,8 +346,9 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
                                                                   (q_begin - cta_q0));
         }
         // group bookkeeping without divisions in the loop
-        int left = p.qpg - ((q_begin * QK) % p.G) / QK;  // quads left in the current group
-        uint32_t rc = smem_u32(tab) + RS * (uint32_t)(((q_begin * QK) / p.G - g_cta0) * COLS + cg);
+        const int g_first = gdiv(q_begin);
+        int left = p.qpg - (q_begin - g_first * p.qpg);  // quads left in the current group
+        uint32_t rc = smem_u32(tab) + RS * (uint32_t)((g_first - g_cta0) * COLS + cg);
         constexpr uint32_t CS8 = 8 * RS;  // record stride between the lane's columns
         // bias constants of the lane's 4 columns, in registers for narrow records
         constexpr bool CREG = NC <= 2;
@@ -557,10 +568,12 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     prm.Kw = pb.K / EPS;
     prm.Q = (prm.Kw + 3) / 4;
     prm.qpg = (pb.G == pb.K) ? (1 << 29) : pb.G / QK;
+    prm.qpg_shift = (prm.qpg & (prm.qpg - 1)) == 0 ? ilog2(prm.qpg) : -1;
+    prm.n_groups = (pb.K + pb.G - 1) / pb.G;
     const int colblocks = (pb.N + COLS - 1) / COLS;
     const int sms = sm_count();
 
-    auto layout = [&](int WK, int CS, int QW, Params& q) -> size_t {
+    auto layout = [&](int WK, int CS, int QW, Params& q, bool one_slot = false) -> size_t {
         q.WK = WK; q.CS = CS; q.QW = QW;
         const int rows_cta = WK * QW * 4;
         const int quads_cta = WK * QW;
@@ -569,10 +582,16 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
         q.qc_shift = ilog2(quads_cta);
         q.groups_cta = std::min((quads_cta * QK + pb.G - 1) / pb.G + 1, (pb.K + pb.G - 1) / pb.G);
         q.xs_tok_stride = rows_cta * EPS * 2 + 16;
-        q.nst = QW > SQ ? 2 : 1;
+        q.nst = (QW > SQ && !one_slot) ? 2 : 1;
         size_t off = (size_t)WK * q.nst * stage_bytes<BITS>();
         q.off_bar = (uint32_t)off;
-        off += (size_t)WK * MAXST * 8;
+        off += (size_t)WK * MAXST * 8 + 8;  // per-warp stage barriers, then the s/z barrier
+        off = (off + 127) & ~(size_t)127;
+        q.sz_box = std::min(q.groups_cta, 256);
+        q.sz_rows = (q.groups_cta + q.sz_box - 1) / q.sz_box * q.sz_box;
+        q.off_sz = (uint32_t)off;
+        q.sz_stride = (uint32_t)(((size_t)q.sz_rows * COLS * 2 + 127) & ~(size_t)127);
+        off += (size_t)2 * q.sz_stride;
         q.off_x = (uint32_t)off;
         off += (size_t)pb.M * q.xs_tok_stride;
         off = (off + 15) & ~(size_t)15;
@@ -588,13 +607,34 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
         return off + 1024;  // slack for aligning the base to 1024 bytes
     };
 
-    // Among (warps per CTA, cluster size), pick the plan with the fewest waves x
-    // quads per warp; ties go to no cluster and larger CTAs.
     bool found = false;
     Params best{};
     size_t best_smem = 0;
     long best_score = 0;
+    // Products that overlap the previous one (WQ_FLAG_PDL_INPUTS_READY) gain
+    // most from small CTAs: 8 warps and one stage slot per warp keep shared
+    // memory low enough for three or more CTAs per SM, so several launches
+    // stream at once.  Used when there are enough column blocks to fill the SMs.
+    if (prm.late_wait && colblocks >= sms / 2) {
+        int QW = 1;
+        while (QW * 8 < prm.Q) QW <<= 1;
+        Params q = prm;
+        const size_t sm = layout(8, 1, QW, q, true);
+        int occ = 0;
+        if (sm <= 227 * 1024) {
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 8 * 32, sm);
+            cudaGetLastError();
+        }
+        if (occ >= 3) {
+            found = true;
+            best = q;
+            best_smem = sm;
+        }
+    }
+    // Otherwise, among (warps per CTA, cluster size), pick the plan with the
+    // fewest waves x quads per warp; ties go to no cluster and larger CTAs.
     for (int WK : {16, 8, 4}) {
+        if (found && best_score == 0) break;
         for (int CS : {1, 2, 4, 8}) {
             if (CS > 1 && WK * CS > prm.Q) continue;
             int QW = 1;
@@ -621,9 +661,13 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     }
     if (!found) return WQ_ERR_INVALID_ARG;  // shape too large for the shared-memory plan
 
-    CUtensorMap mw, ml;
+    CUtensorMap mw, ml, ms, mz;
     bool ok = make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, pb.w_q, pb.N, prm.Kw, (uint64_t)pb.N * 4, COLS, 4 * SQ,
                        CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && make_map(&ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, pb.scales, pb.N, prm.n_groups, (uint64_t)pb.N * 2, COLS,
+                        best.sz_box, CU_TENSOR_MAP_SWIZZLE_NONE);
+    ok = ok && make_map(&mz, CU_TENSOR_MAP_DATA_TYPE_UINT16, pb.zeros, pb.N, prm.n_groups, (uint64_t)pb.N * 2, COLS,
+                        best.sz_box, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (BITS == 3)
         ok = ok && make_map(&ml, CU_TENSOR_MAP_DATA_TYPE_UINT32, pb.w_lo, pb.N, pb.K / 32, (uint64_t)pb.N * 4, COLS,
                             2 * SQ, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -650,7 +694,7 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     }
     cfg.attrs = attrs;
     cfg.numAttrs = na;
-    return from_cuda(cudaLaunchKernelEx(&cfg, kern, mw, ml, best));
+    return from_cuda(cudaLaunchKernelEx(&cfg, kern, mw, ml, ms, mz, best));
 }
 
 }  // namespace

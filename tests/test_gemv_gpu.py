@@ -146,7 +146,11 @@ def test_inputs_ready_orders_the_writes_of_y(cuda, libwq):
     cases = [wq_inputs.custom(4, 4096, 4096, 4, 128, seed=20 + i) for i in range(3)]
     ds = [to_dev(c, cuda) for c in cases]
     packed = [libwq.pack_kmajor(d["codes"], 4) for d in ds]
-    ref = [run_gemv(libwq, d, 4, 128) for d in ds]
+    ref = []
+    for d, (w_q, _) in zip(ds, packed):  # same launch flag as below, so the same plan
+        torch.cuda.synchronize()
+        ref.append(libwq.gemv(d["x"], w_q, None, d["scales"], d["zeros"], 4, 128,
+                              inputs_ready=True).cpu().numpy())
     buf = ds[0]["x"].clone()                       # call 0 reads buf ...
     y0 = torch.empty((4, 4096), dtype=torch.float16, device=cuda)
     out = torch.empty((4, 4096), dtype=torch.float16, device=cuda)
@@ -165,6 +169,22 @@ def test_inputs_ready_orders_the_writes_of_y(cuda, libwq):
         assert np.array_equal(y0.cpu().numpy(), ref[0])
         assert np.array_equal(buf.cpu().numpy(), ref[1])
         assert np.array_equal(out.cpu().numpy(), ref[1])
+
+
+@pytest.mark.parametrize("name", ["decode_gemv_m1", "decode_gemv_m4", "decode_gemv_m16", "gemv_3bit",
+                                  "sweep_1bit", "sweep_8bit_perchannel"])
+def test_inputs_ready_plan_matches_oracle(cuda, libwq, orc, name):
+    """WQ_FLAG_PDL_INPUTS_READY selects its own CTA shape; every output against the oracle."""
+    import torch
+    case = wq_inputs.draw(wq_inputs.WORKLOADS[name], seed=0)
+    d = to_dev(case, cuda)
+    w_q, w_lo = libwq.pack_kmajor(d["codes"], case.wl.bits)
+    torch.cuda.synchronize()
+    y = libwq.gemv(d["x"], w_q, w_lo, d["scales"], d["zeros"], case.wl.bits, case.wl.group_size,
+                   inputs_ready=True).cpu().numpy()
+    y_ref, b = oracle_product(orc, case)
+    check_product(y, y_ref, b, name)
+    assert libwq.device_status() == 0
 
 
 def test_deterministic(cuda, libwq):
