@@ -214,22 +214,49 @@ def layers_for(wl, L2):
     return min(1024, max(2, int(2 * L2 // algo_bytes(wl)) + 2))
 
 
+def cpu_model() -> str:
+    try:
+        for line in Path("/proc/cpuinfo").read_text().splitlines():
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(seconds: float = 10.0):
-    """The CPU oracle (plain C fp64, OpenMP) on full decode GEMVs, for ~`seconds`."""
+    """The CPU oracle (plain C fp64) on full decode GEMVs: OpenMP over all host
+    threads for ~`seconds`, then one thread for ~`seconds` / 4."""
     import oracle
     wl = wq_inputs.WORKLOADS[HEADLINE]
     case = wq_inputs.draw(wl, 0)
     wq_, wlo = oracle.pack(case.codes, wl.bits)
-    reps, t0 = 0, time.perf_counter()
-    while True:
-        oracle.wq_matmul(case.x, wq_, wlo, case.scales, case.zeros, wl.bits, wl.group_size)
-        reps += 1
-        el = time.perf_counter() - t0
-        if el >= seconds or reps >= 2000:
-            break
-    return {"value": round(algo_bytes(wl) * reps / el / 1e9, 3), "unit": "GB/s", "cores": oracle.threads(),
-            "kind": "oracle",
-            "sample": f"{reps} full decode GEMVs (M=1, K=N=4096, 4-bit, g128) in {el:.1f} s, fp64 C"}
+
+    def run(limit):
+        reps, t0 = 0, time.perf_counter()
+        while True:
+            oracle.wq_matmul(case.x, wq_, wlo, case.scales, case.zeros, wl.bits, wl.group_size)
+            reps += 1
+            el = time.perf_counter() - t0
+            if el >= limit or reps >= 2000:
+                return reps, el
+
+    cores = oracle.threads()
+    reps, el = run(seconds)
+    single = None
+    try:
+        oracle.set_threads(1)
+        r1, e1 = run(seconds / 4)
+        single = {"value": round(algo_bytes(wl) * r1 / e1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                  "sample": f"{r1} full decode GEMVs in {e1:.1f} s"}
+    except AttributeError:
+        pass
+    finally:
+        if hasattr(oracle, "set_threads"):
+            oracle.set_threads(cores)
+    return {"value": round(algo_bytes(wl) * reps / el / 1e9, 3), "unit": "GB/s", "cores": cores,
+            "kind": "oracle", "cpu": cpu_model(), "single_thread": single,
+            "sample": f"{reps} full decode GEMVs (M=1, K=N=4096, 4-bit, g128) in {el:.1f} s, fp64 C, OpenMP"}
 
 
 # ------------------------------------------------------------------ reference arm

@@ -59,6 +59,8 @@ def lib():
         p = ctypes.c_void_p
         i = ctypes.c_int
         L.orc_threads.restype = i
+        L.orc_set_threads.argtypes = [i]
+        L.orc_set_threads.restype = None
         L.orc_half_to_double.argtypes = [ctypes.c_uint16]
         L.orc_half_to_double.restype = ctypes.c_double
         L.orc_pack_kmajor.argtypes = [p, i, i, i, p, p]
@@ -67,8 +69,9 @@ def lib():
         L.orc_matmul.argtypes = [p, p, i, i, i, p, p]
         L.orc_wq_matmul.argtypes = [p, p, p, p, p, i, i, i, i, i, p, p]
         L.orc_wq_matmul_sampled.argtypes = [p, p, p, p, p, i, i, i, i, i, p, p, i, p, p]
+        L.orc_add_bias.argtypes = [p, p, p, i, i]
         for f in ("orc_pack_kmajor", "orc_unpack_kmajor", "orc_dequant", "orc_matmul",
-                  "orc_wq_matmul", "orc_wq_matmul_sampled"):
+                  "orc_wq_matmul", "orc_wq_matmul_sampled", "orc_add_bias"):
             getattr(L, f).restype = i
         _lib = L
     return _lib
@@ -92,6 +95,11 @@ def words_shape(K: int, N: int, bits: int):
 
 def threads() -> int:
     return int(lib().orc_threads())
+
+
+def set_threads(n: int) -> None:
+    """Threads of the OpenMP loops from now on (for timing; results do not depend on it)."""
+    lib().orc_set_threads(int(n))
 
 
 def half_to_double(h: int) -> float:
@@ -139,8 +147,9 @@ def matmul(x, w_kn):
     return y, b
 
 
-def wq_matmul(x, wq, wlo, scales, zeros, bits: int, group_size: int, N: int | None = None):
-    """``(y_ref, bound)`` in fp64 for the packed problem (unpack, dequant, matmul)."""
+def wq_matmul(x, wq, wlo, scales, zeros, bits: int, group_size: int, N: int | None = None, bias=None):
+    """``(y_ref, bound)`` in fp64 for the packed problem (unpack, dequant, matmul,
+    then the optional fp16 ``bias`` of shape (N,))."""
     x = np.ascontiguousarray(x, dtype=np.float16).view(np.uint16)
     M, K = x.shape
     wq = np.ascontiguousarray(wq, dtype=np.uint32)
@@ -152,11 +161,22 @@ def wq_matmul(x, wq, wlo, scales, zeros, bits: int, group_size: int, N: int | No
     b = np.zeros((M, N), dtype=np.float64)
     _check(lib().orc_wq_matmul(_ptr(x), _ptr(wq), _ptr(wlo), _ptr(s), _ptr(z), M, K, N, bits,
                                group_size, _ptr(y), _ptr(b)), "wq_matmul")
+    if bias is not None:
+        add_bias(y, b, bias)
     return y, b
 
 
-def wq_matmul_sampled(x, wq, wlo, scales, zeros, bits: int, group_size: int, ms, ns):
-    """``(y_ref, bound)`` for the single outputs ``(ms[i], ns[i])``."""
+def add_bias(y, bound, bias):
+    """In place: ``y[m][n] += bias[n]``, ``bound[m][n] += |bias[n]|`` (fp64)."""
+    bias = np.ascontiguousarray(bias, dtype=np.float16).view(np.uint16)
+    M, N = y.shape
+    if bias.shape != (N,) or y.dtype != np.float64 or not y.flags.c_contiguous:
+        raise OracleError("add_bias: y (M, N) fp64 contiguous and bias (N,) expected")
+    _check(lib().orc_add_bias(_ptr(y), _ptr(bound), _ptr(bias), M, N), "add_bias")
+
+
+def wq_matmul_sampled(x, wq, wlo, scales, zeros, bits: int, group_size: int, ms, ns, bias=None):
+    """``(y_ref, bound)`` for the single outputs ``(ms[i], ns[i])`` (+ ``bias[ns[i]]``)."""
     x = np.ascontiguousarray(x, dtype=np.float16).view(np.uint16)
     M, K = x.shape
     wq = np.ascontiguousarray(wq, dtype=np.uint32)
@@ -171,4 +191,8 @@ def wq_matmul_sampled(x, wq, wlo, scales, zeros, bits: int, group_size: int, ms,
     _check(lib().orc_wq_matmul_sampled(_ptr(x), _ptr(wq), _ptr(wlo), _ptr(s), _ptr(z), M, K, N,
                                        bits, group_size, _ptr(ms), _ptr(ns), len(ms), _ptr(y),
                                        _ptr(b)), "wq_matmul_sampled")
+    if bias is not None:
+        bv = np.asarray(bias, dtype=np.float16).astype(np.float64)[ns]
+        y += bv
+        b += np.abs(bv)
     return y, b

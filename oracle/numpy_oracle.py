@@ -73,9 +73,15 @@ def dequant(wq, wlo, scales, zeros, K: int, N: int, bits: int, group_size: int) 
     return (q - z) * s
 
 
-def wq_matmul(x, wq, wlo, scales, zeros, bits: int, group_size: int, N: int | None = None):
+def wq_matmul(x, wq, wlo, scales, zeros, bits: int, group_size: int, N: int | None = None, bias=None):
+    """y = x @ w (+ bias[n], one fp16 value per output column, as the module's
+    forward adds it), and the bound sum |x w| (+ |bias|)."""
     x = np.asarray(x, dtype=np.float16).astype(np.float64)
     K = x.shape[1]
     N = np.asarray(wq).shape[1] if N is None else N
     w = dequant(wq, wlo, scales, zeros, K, N, bits, group_size)
-    return x @ w, np.abs(x) @ np.abs(w)
+    y, b = x @ w, np.abs(x) @ np.abs(w)
+    if bias is not None:
+        bv = np.asarray(bias, dtype=np.float16).astype(np.float64).reshape(1, N)
+        y, b = y + bv, b + np.abs(bv)
+    return y, b

@@ -55,6 +55,15 @@ int orc_threads(void) {
 #endif
 }
 
+/* Threads the OpenMP loops use from now on (timing only; results do not depend on it). */
+void orc_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /* IEEE 754 binary16 -> double, exact. */
 double orc_half_to_double(uint16_t h) {
     int sign = (h >> 15) & 1;
@@ -196,6 +205,23 @@ int orc_wq_matmul(const uint16_t* x, const uint32_t* wq, const uint32_t* wlo, co
     if (rc == ORC_OK) rc = orc_matmul(x, w, M, K, N, y, bound);
     free(w);
     return rc;
+}
+
+/*
+ * Fused bias ("dashq_kernel.py" `TritonQuantLinear.forward`: the output of
+ * the product plus `bias`, one fp16 value per output column):
+ * y[m][n] += bias[n], and the bias is one more addend of the error bound,
+ * bound[m][n] += |bias[n]|.
+ */
+int orc_add_bias(double* y, double* bound, const uint16_t* bias, int M, int N) {
+    if (M <= 0 || N <= 0 || !bias) return ORC_EARG;
+    for (int m = 0; m < M; ++m)
+        for (int n = 0; n < N; ++n) {
+            double b = orc_half_to_double(bias[n]);
+            y[(size_t)m * N + n] += b;
+            if (bound) bound[(size_t)m * N + n] += fabs(b);
+        }
+    return ORC_OK;
 }
 
 /*

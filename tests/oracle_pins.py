@@ -218,6 +218,32 @@ def pin_group_index(impl):
     assert np.array_equal(y[:, 0], expect), y[:, 0]
 
 
+def pin_bias(impl):
+    """The fused bias (one fp16 value per output column, added after the
+    product): with x = 0, or with every q == z, y is the bias exactly in every
+    row and the bound is |bias|; with x = e_k, row k is w[k] + bias, exact in
+    fp64 since both addends are exact."""
+    for bits in (1, 3, 4, 8):
+        kd = _kdiv(bits)
+        K, N, M, G = 4 * kd, 9, 3, 2 * kd
+        x, codes, s, z = _problem(bits, M, K, N, G, 300 + bits, int_zeros=False)
+        bias = _rng(400 + bits).uniform(-3, 3, size=N).astype(np.float16)
+        bias64 = bias.astype(np.float64)
+        wq, wlo = impl.pack(codes, bits)
+        y, b = impl.wq_matmul(np.zeros_like(x), wq, wlo, s, z, bits, G, bias=bias)
+        assert np.array_equal(y, np.tile(bias64, (M, 1))), (bits, "x = 0")
+        assert np.array_equal(b, np.tile(np.abs(bias64), (M, 1))), (bits, "bound, x = 0")
+        zq = _rng(bits + 60).integers(0, 1 << bits, size=(K // G, N))
+        wq0, wlo0 = impl.pack(np.repeat(zq, G, axis=0).astype(np.uint8), bits)
+        y, _ = impl.wq_matmul(x, wq0, wlo0, s, zq.astype(np.float16), bits, G, bias=bias)
+        assert np.array_equal(y, np.tile(bias64, (M, 1))), (bits, "q == z")
+        y, _ = impl.wq_matmul(np.eye(K, dtype=np.float16), wq, wlo, s, z, bits, G, bias=bias)
+        for k in range(K):
+            g = k // G
+            row = (codes[k].astype(np.float64) - z[g].astype(np.float64)) * s[g].astype(np.float64)
+            assert np.array_equal(y[k], row + bias64), (bits, "one-hot", k)
+
+
 PINS = [
     pin_golden_pack,
     pin_golden_products,
@@ -229,4 +255,5 @@ PINS = [
     pin_integer_matmul_special_case,
     pin_group_equivalences,
     pin_group_index,
+    pin_bias,
 ]

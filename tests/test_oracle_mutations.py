@@ -20,14 +20,34 @@ def _mutant(**overrides):
     return m
 
 
-def _matmul_with(dequant_fn):
-    def wq_matmul(x, wq, wlo, s, z, bits, G, N=None):
+def _with_bias(y, b, bias, N, sign=1.0, by_row=False):
+    if bias is None:
+        return y, b
+    bv = np.asarray(bias, np.float16).astype(np.float64)
+    if by_row:  # indexed by the token instead of the output column
+        bv = np.resize(bv, y.shape[0]).reshape(-1, 1)
+    else:
+        bv = bv.reshape(1, N)
+    return y + sign * bv, b + np.abs(bv)
+
+
+def _matmul_with(dequant_fn, bias_sign=1.0, bias_by_row=False, bias_used=True):
+    def wq_matmul(x, wq, wlo, s, z, bits, G, N=None, bias=None):
         x = np.asarray(x, np.float16).astype(np.float64)
         K = x.shape[1]
         N = np.asarray(wq).shape[1] if N is None else N
         w = dequant_fn(wq, wlo, s, z, K, N, bits, G)
-        return x @ w, np.abs(x) @ np.abs(w)
+        return _with_bias(x @ w, np.abs(x) @ np.abs(w), bias if bias_used else None, N,
+                          bias_sign, bias_by_row)
     return wq_matmul
+
+
+def _transposed(x, wq, wlo, s, z, bits, G, N=None, bias=None):
+    xx = np.asarray(x, np.float16).astype(np.float64)
+    N = np.asarray(wq).shape[1] if N is None else N
+    w = tw.dequant(wq, wlo, s, z, xx.shape[1], N, bits, G)
+    y = xx @ (w.T if w.shape[0] == w.shape[1] else w[::-1])
+    return _with_bias(y, np.abs(xx) @ np.abs(w), bias, N)
 
 
 def _dq(q_fn=None, combine=lambda q, z, s: (q - z) * s, expand=np.repeat):
@@ -101,13 +121,10 @@ MUTANTS = {
                                        wq_matmul=_matmul_with(_dq(q_fn=_unpack_no_mask))),
     "lo_plane_bit_index_3bit": _mutant(unpack=_unpack_3bit_lo_index,
                                        wq_matmul=_matmul_with(_dq(q_fn=_unpack_3bit_lo_index))),
-    "operand_transposed": _mutant(
-        wq_matmul=lambda x, wq, wlo, s, z, bits, G, N=None: (
-            lambda xx, w: (xx @ (w.T if w.shape[0] == w.shape[1] else w[::-1]),
-                           np.abs(xx) @ np.abs(w)))(
-            np.asarray(x, np.float16).astype(np.float64),
-            tw.dequant(wq, wlo, s, z, np.asarray(x).shape[1],
-                       np.asarray(wq).shape[1] if N is None else N, bits, G))),
+    "operand_transposed": _mutant(wq_matmul=_transposed),
+    "bias_dropped": _mutant(wq_matmul=_matmul_with(tw.dequant, bias_used=False)),
+    "bias_sign_flipped": _mutant(wq_matmul=_matmul_with(tw.dequant, bias_sign=-1.0)),
+    "bias_indexed_by_token": _mutant(wq_matmul=_matmul_with(tw.dequant, bias_by_row=True)),
     "bound_signed": _mutant(
         wq_matmul=lambda *a, **k: (lambda r: (r[0], np.abs(r[0])))(tw.wq_matmul(*a, **k))),
 }
