@@ -9,9 +9,10 @@ Entry points (same names as the C ABI, without the ``wq_`` prefix):
 
 * ``pack_kmajor(codes_kn, bits) -> (w_q, w_lo)``
 * ``unpack_kmajor(w_q, w_lo, K, bits) -> codes_kn``
-* ``gemv(x, w_q, w_lo, scales, zeros, bits, group_size, out=None, pdl=False) -> y``
+* ``gemv(x, w_q, w_lo, scales, zeros, bits, group_size, out=None, pdl=False,
+  inputs_ready=False, bias=None) -> y``
 * ``gemm(x, w_q, w_lo, scales, zeros, bits, group_size, out=None, pdl=False,
-  workspace=None) -> y``
+  workspace=None, inputs_ready=False, bias=None) -> y``
 * ``gemm_workspace_size(M, K, N, bits, group_size) -> bytes``
 * ``gemm_noalloc(x, w_q, w_lo, scales, zeros, bits, group_size, out) -> out``
 """
@@ -62,11 +63,11 @@ def lib() -> ctypes.CDLL:
         L.wq_status_string.restype = ctypes.c_char_p
         L.wq_pack_kmajor.argtypes = [p, i, i, i, p, p, p, p]
         L.wq_unpack_kmajor.argtypes = [p, p, i, i, i, p, p]
-        L.wq_gemv.argtypes = [p, p, p, p, p, p, i, i, i, i, i, u, p]
-        L.wq_gemm.argtypes = [p, p, p, p, p, p, i, i, i, i, i, u, p, ctypes.c_size_t, p]
+        L.wq_gemv.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, u, p]
+        L.wq_gemm.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, u, p, ctypes.c_size_t, p]
         L.wq_gemm_workspace_size.argtypes = [i, i, i, i, i]
         L.wq_gemm_workspace_size.restype = ctypes.c_size_t
-        L.wq_gemm_noalloc.argtypes = [p, p, p, p, p, p, i, i, i, i, i, u, p]
+        L.wq_gemm_noalloc.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, u, p]
         L.wq_gemm_noalloc.restype = i
         L.wq_device_status.argtypes = [i]
         for f in ("wq_pack_kmajor", "wq_unpack_kmajor", "wq_gemv", "wq_gemm", "wq_device_status"):
@@ -151,7 +152,7 @@ def unpack_kmajor(w_q, w_lo, K: int, bits: int):
 
 
 def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, workspace=False,
-             inputs_ready=False):
+             inputs_ready=False, bias=None):
     torch = _torch()
     _need(x, torch.float16, "x")
     _need(w_q, torch.int32, "w_q")
@@ -159,6 +160,8 @@ def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, worksp
         _need(w_lo, torch.int32, "w_lo")
     _need(scales, torch.float16, "scales")
     _need(zeros, torch.float16, "zeros")
+    if bias is not None:
+        _need(bias, torch.float16, "bias", ndim=1)
     M, K = x.shape
     N = w_q.shape[1]
     if out is None:
@@ -166,7 +169,7 @@ def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, worksp
     else:
         _need(out, torch.float16, "out")
     flags = (WQ_FLAG_PDL if pdl else 0) | (WQ_FLAG_PDL_INPUTS_READY if inputs_ready else 0)
-    args = [_ptr(x), _ptr(w_q), _ptr(w_lo), _ptr(scales), _ptr(zeros), _ptr(out),
+    args = [_ptr(x), _ptr(w_q), _ptr(w_lo), _ptr(scales), _ptr(zeros), _ptr(bias), _ptr(out),
             M, K, N, bits, group_size, flags]
     if workspace is not False:  # wq_gemm: (workspace, bytes)
         if workspace is None:
@@ -178,13 +181,14 @@ def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, worksp
 
 
 def gemv(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl: bool = False,
-         inputs_ready: bool = False):
+         inputs_ready: bool = False, bias=None):
     """y (M, N) fp16 = x (M, K) @ dequant(w_q), 1 <= M <= 16 (``wq_gemv``).
 
     ``pdl``: WQ_FLAG_PDL; ``inputs_ready``: WQ_FLAG_PDL_INPUTS_READY (the previous
-    kernel on the stream writes none of this call's inputs)."""
+    kernel on the stream writes none of this call's inputs); ``bias``: optional (N,)
+    fp16 tensor added to every row of the output."""
     return _product("wq_gemv", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl,
-                    inputs_ready=inputs_ready)
+                    inputs_ready=inputs_ready, bias=bias)
 
 
 def gemm_workspace_size(M: int, K: int, N: int, bits: int, group_size: int) -> int:
@@ -218,7 +222,7 @@ def _cached_workspace(device, nbytes: int):
 
 
 def gemm(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl: bool = False,
-         workspace=None, inputs_ready: bool = False):
+         workspace=None, inputs_ready: bool = False, bias=None):
     """y (M, N) fp16 = x (M, K) @ dequant(w_q), any M >= 1 (``wq_gemm``).
 
     ``workspace``: a CUDA uint8 tensor of at least ``gemm_workspace_size(...)``
@@ -228,7 +232,7 @@ def gemm(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl:
         torch = _torch()
         _need(workspace, torch.uint8, "workspace", ndim=1)
     return _product("wq_gemm", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, workspace,
-                    inputs_ready=inputs_ready)
+                    inputs_ready=inputs_ready, bias=bias)
 
 
 def device_status(reset: bool = False) -> int:
@@ -236,10 +240,12 @@ def device_status(reset: bool = False) -> int:
     return int(lib().wq_device_status(1 if reset else 0))
 
 
-def gemm_noalloc(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out, pdl: bool = False):
+def gemm_noalloc(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out, pdl: bool = False,
+                 bias=None):
     """``wq_gemm_noalloc``: the product into the caller's ``out`` with the
     library's fixed split-K scratch; neither the call nor this wrapper
     allocates device memory."""
     torch = _torch()
     _need(out, torch.float16, "out")
-    return _product("wq_gemm_noalloc", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl)
+    return _product("wq_gemm_noalloc", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl,
+                    bias=bias)

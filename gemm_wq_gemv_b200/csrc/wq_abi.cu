@@ -111,30 +111,32 @@ wq_status wq_unpack_kmajor(const uint32_t* w_q, const uint32_t* w_lo, int K, int
 }
 
 wq_status wq_gemv(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
-                  const uint16_t* scales, const uint16_t* zeros, uint16_t* y, int M, int K, int N,
-                  int bits, int group_size, unsigned flags, void* stream) {
+                  const uint16_t* scales, const uint16_t* zeros, const uint16_t* bias, uint16_t* y,
+                  int M, int K, int N, int bits, int group_size, unsigned flags, void* stream) {
     int G = 0;
     wq_status st = check_product(x, w_q, w_lo, scales, zeros, y, M, K, N, bits, group_size, G);
     if (st != WQ_OK) return st;
+    if (bias && !aligned(bias, 2)) return WQ_ERR_ALIGNMENT;
     if (M > 16) return WQ_ERR_INVALID_ARG;
     if (G != K && G % (4 * main_eps(bits)) != 0) return WQ_ERR_UNSUPPORTED;
     if ((st = check_device()) != WQ_OK) return st;
-    wq::Problem p{x, w_q, w_lo, scales, zeros, y, M, K, N, bits, G, flags, nullptr, 0};
+    wq::Problem p{x, w_q, w_lo, scales, zeros, bias, y, M, K, N, bits, G, flags, nullptr, 0};
     return wq::launch_gemv(p, (cudaStream_t)stream);
 }
 
 wq_status wq_gemm(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
-                  const uint16_t* scales, const uint16_t* zeros, uint16_t* y, int M, int K, int N,
-                  int bits, int group_size, unsigned flags, void* workspace, size_t workspace_bytes,
-                  void* stream) {
+                  const uint16_t* scales, const uint16_t* zeros, const uint16_t* bias, uint16_t* y,
+                  int M, int K, int N, int bits, int group_size, unsigned flags, void* workspace,
+                  size_t workspace_bytes, void* stream) {
     int G = 0;
     wq_status st = check_product(x, w_q, w_lo, scales, zeros, y, M, K, N, bits, group_size, G);
     if (st != WQ_OK) return st;
+    if (bias && !aligned(bias, 2)) return WQ_ERR_ALIGNMENT;
     if (K % 64 != 0) return WQ_ERR_INVALID_ARG;
     if (G % 64 != 0 && 64 % G != 0) return WQ_ERR_UNSUPPORTED;
     if (workspace && !aligned(workspace, 16)) return WQ_ERR_ALIGNMENT;
     if ((st = check_device()) != WQ_OK) return st;
-    wq::Problem p{x, w_q, w_lo, scales, zeros, y, M, K, N, bits, G, flags, workspace,
+    wq::Problem p{x, w_q, w_lo, scales, zeros, bias, y, M, K, N, bits, G, flags, workspace,
                   workspace ? workspace_bytes : 0};
     return wq::launch_gemm(p, (cudaStream_t)stream);
 }

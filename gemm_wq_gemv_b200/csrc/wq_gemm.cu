@@ -51,6 +51,7 @@ constexpr uint64_t WAIT_NS = 2000000000ull;
 
 struct GemmParams {
     uint16_t* y;
+    const uint16_t* bias;  // (N,) fp16 or null
     int M, K, N, G;
     int TN;              // tokens per tile (MMA N)
     int CS;              // CTAs per cluster along K
@@ -317,10 +318,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
                 }
             }
             if (ncol < p.N) {
+                const float bv = p.bias ? __half2float(__ushort_as_half(p.bias[ncol])) : 0.0f;
 #pragma unroll
                 for (int cc = 0; cc < 32; ++cc) {
                     const int m = m0 + 32 * j + cc;
-                    if (m < p.M) p.y[(size_t)m * p.N + ncol] = __half_as_ushort(__float2half_rn(acc[cc]));
+                    if (m < p.M) p.y[(size_t)m * p.N + ncol] = __half_as_ushort(__float2half_rn(acc[cc] + bv));
                 }
             }
         }
@@ -376,6 +378,7 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
 
     GemmParams p{};
     p.y = pb.y;
+    p.bias = pb.bias;
     p.M = pb.M; p.K = pb.K; p.N = pb.N; p.G = pb.G;
     // s/z rows per 64-deep block: 1 if a group covers whole blocks, else 64 / G
     if (pb.G % BK == 0) p.GPB = 1;

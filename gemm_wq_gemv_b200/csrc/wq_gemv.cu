@@ -53,6 +53,7 @@ struct Params {
     const uint32_t* w_lo;
     const uint16_t* s;
     const uint16_t* z;
+    const uint16_t* bias;  // (N,) fp16 or null
     uint16_t* y;
     int M, K, N, G;
     int Kw;        // word rows of the main plane
@@ -528,14 +529,20 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
             float sacc = 0.0f;
             for (int r = 0; r < p.CS; ++r) sacc += ld_shared_cluster_f32(map_shared_rank(part_addr + 4u * i, r));
             const int m = i / COLS, col = col0 + i % COLS;
-            if (col < p.N) p.y[(size_t)m * p.N + col] = __half_as_ushort(__float2half_rn(sacc));
+            if (col < p.N) {
+                const float b = p.bias ? __half2float(__ushort_as_half(p.bias[col])) : 0.0f;
+                p.y[(size_t)m * p.N + col] = __half_as_ushort(__float2half_rn(sacc + b));
+            }
         }
         cluster_sync();  // peers keep their shared memory until every read is done
     } else {
         for (int i = threadIdx.x; i < p.M * COLS; i += blockDim.x) {
             const float sacc = sum_warps(red, p.WK, p.M * COLS, i);
             const int m = i / COLS, col = col0 + i % COLS;
-            if (col < p.N) p.y[(size_t)m * p.N + col] = __half_as_ushort(__float2half_rn(sacc));
+            if (col < p.N) {
+                const float b = p.bias ? __half2float(__ushort_as_half(p.bias[col])) : 0.0f;
+                p.y[(size_t)m * p.N + col] = __half_as_ushort(__float2half_rn(sacc + b));
+            }
         }
     }
 }
@@ -563,6 +570,7 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     }
     Params prm{};
     prm.x = pb.x; prm.w_q = pb.w_q; prm.w_lo = pb.w_lo; prm.s = pb.scales; prm.z = pb.zeros;
+    prm.bias = pb.bias;
     prm.y = pb.y; prm.M = pb.M; prm.K = pb.K; prm.N = pb.N; prm.G = pb.G;
     prm.late_wait = (pb.flags & WQ_FLAG_PDL_INPUTS_READY) ? 1 : 0;
     prm.Kw = pb.K / EPS;

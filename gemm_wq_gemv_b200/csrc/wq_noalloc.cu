@@ -47,9 +47,9 @@ wq_status scratch_address(void** out) {
 }  // namespace
 
 extern "C" wq_status wq_gemm_noalloc(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
-                                     const uint16_t* scales, const uint16_t* zeros, uint16_t* y,
-                                     int M, int K, int N, int bits, int group_size, unsigned flags,
-                                     void* stream) {
+                                     const uint16_t* scales, const uint16_t* zeros,
+                                     const uint16_t* bias, uint16_t* y, int M, int K, int N,
+                                     int bits, int group_size, unsigned flags, void* stream) {
     // 0 for shapes that do not split K and for invalid arguments, which wq_gemm
     // then rejects without the scratch.
     const size_t need = wq_gemm_workspace_size(M, K, N, bits, group_size);
@@ -59,6 +59,6 @@ extern "C" wq_status wq_gemm_noalloc(const uint16_t* x, const uint32_t* w_q, con
         const wq_status st = scratch_address(&scratch);
         if (st != WQ_OK) return st;
     }
-    return wq_gemm(x, w_q, w_lo, scales, zeros, y, M, K, N, bits, group_size, flags, scratch,
+    return wq_gemm(x, w_q, w_lo, scales, zeros, bias, y, M, K, N, bits, group_size, flags, scratch,
                    scratch ? (size_t)WQ_GEMM_NOALLOC_SCRATCH_BYTES : 0, stream);
 }

@@ -50,7 +50,7 @@
 extern "C" {
 #endif
 
-#define WQ_ABI_VERSION 1
+#define WQ_ABI_VERSION 2
 
 typedef enum {
     WQ_OK = 0,
@@ -122,15 +122,20 @@ wq_status wq_unpack_kmajor(const uint32_t* w_q, const uint32_t* w_lo, int K, int
  * (3-bit: K % 32 == 0) and N % 8 == 0.
  * One launch: the split-K partial sums are reduced on chip (thread-block
  * cluster shared memory); no workspace and no zero-initialised output needed.
+ *   bias  optional (N,) binary16 device array, 2-byte aligned, or NULL: then
+ *         y[m][n] = RN_fp16(sum_k x[m][k] w[k][n] + bias[n]), the sum in fp32
+ *         (dashq_kernel.py `TritonQuantLinear.forward` adds its bias to the
+ *         product's output).
  */
 wq_status wq_gemv(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
-                  const uint16_t* scales, const uint16_t* zeros, uint16_t* y,
-                  int M, int K, int N, int bits, int group_size, unsigned flags, void* stream);
+                  const uint16_t* scales, const uint16_t* zeros, const uint16_t* bias,
+                  uint16_t* y, int M, int K, int N, int bits, int group_size, unsigned flags,
+                  void* stream);
 
 /*
  * Batched product for any M >= 1 ("GPTQModel-Compatible Triton Kernel"
  * README, `gptqmodel_quantized_matmul`; dashq_kernel.py `forward`, batched
- * branch).  Same arguments as wq_gemv, plus a workspace.  group_size: -1, or a
+ * branch).  Same arguments as wq_gemv (bias included), plus a workspace.  group_size: -1, or a
  * positive divisor of K that is a multiple of eps (3-bit: of 32) and either a
  * multiple or a divisor of 64.  Requires K % 64 == 0 and N % 8 == 0.
  * Packed tiles are dequantised to fp16 into tensor memory and multiplied on the
@@ -145,8 +150,8 @@ wq_status wq_gemv(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
  *                    is correct but uses fewer SMs for small M x N.
  */
 wq_status wq_gemm(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
-                  const uint16_t* scales, const uint16_t* zeros, uint16_t* y,
-                  int M, int K, int N, int bits, int group_size, unsigned flags,
+                  const uint16_t* scales, const uint16_t* zeros, const uint16_t* bias,
+                  uint16_t* y, int M, int K, int N, int bits, int group_size, unsigned flags,
                   void* workspace, size_t workspace_bytes, void* stream);
 
 /* Workspace bytes wq_gemm uses for this shape (0 when it does not split K, or
@@ -176,9 +181,9 @@ size_t wq_gemm_workspace_size(int M, int K, int N, int bits, int group_size);
  */
 #define WQ_GEMM_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 wq_status wq_gemm_noalloc(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
-                          const uint16_t* scales, const uint16_t* zeros, uint16_t* y,
-                          int M, int K, int N, int bits, int group_size, unsigned flags,
-                          void* stream);
+                          const uint16_t* scales, const uint16_t* zeros, const uint16_t* bias,
+                          uint16_t* y, int M, int K, int N, int bits, int group_size,
+                          unsigned flags, void* stream);
 
 /*
  * Device-side status of the current device: WQ_OK, or WQ_ERR_TIMEOUT when a

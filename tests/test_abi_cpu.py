@@ -30,7 +30,7 @@ def test_every_declared_symbol_is_exported(libwq):
 
 def test_version_and_strings(libwq):
     L = libwq.lib()
-    assert L.wq_abi_version() == 1
+    assert L.wq_abi_version() == 2
     for s in range(7):
         assert L.wq_status_string(s)
     assert L.wq_status_string(99) == b"unknown status"
@@ -40,11 +40,11 @@ P = 0x10000  # a 16-byte aligned fake device address: never dereferenced on the 
 
 
 def gemv(L, fn="wq_gemv", x=P, wq=P, wlo=None, s=P, z=P, y=P, M=1, K=512, N=256, bits=4, G=128,
-         flags=0, ws=None, ws_bytes=0):
+         flags=0, ws=None, ws_bytes=0, bias=None):
     if fn == "wq_gemm":
-        return L.wq_gemm(x, wq, wlo, s, z, y, M, K, N, bits, G, flags, ws, ctypes.c_size_t(ws_bytes),
-                         None)
-    return getattr(L, fn)(x, wq, wlo, s, z, y, M, K, N, bits, G, flags, None)
+        return L.wq_gemm(x, wq, wlo, s, z, bias, y, M, K, N, bits, G, flags, ws,
+                         ctypes.c_size_t(ws_bytes), None)
+    return getattr(L, fn)(x, wq, wlo, s, z, bias, y, M, K, N, bits, G, flags, None)
 
 
 @pytest.mark.parametrize("fn", ["wq_gemv", "wq_gemm"])
@@ -67,6 +67,7 @@ def test_product_argument_checks(libwq, fn):
     assert gemv(L, fn, N=252) == ALI                      # N % 8
     assert gemv(L, fn, x=P + 8) == ALI
     assert gemv(L, fn, wq=P + 4) == ALI
+    assert gemv(L, fn, bias=P + 1) == ALI                 # bias: 2-byte aligned fp16
     # valid arguments: the host checks pass and the call reaches CUDA, which has no device here
     import torch
     if not torch.cuda.is_available():

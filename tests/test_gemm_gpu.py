@@ -159,3 +159,24 @@ def test_pdl_flags(cuda, libwq):
     assert np.array_equal(y0.cpu().numpy(), ref0)
     assert np.array_equal(buf.cpu().numpy(), ref1)
     assert libwq.device_status() == 0
+
+
+@pytest.mark.parametrize("M,K,N,bits,G", [(512, 4096, 2048, 4, 128), (33, 512, 264, 8, 16),
+                                         (200, 2048, 384, 3, 128)])
+def test_bias_matches_oracle(cuda, libwq, orc, M, K, N, bits, G):
+    """y = x @ w + bias through the split-K and single-CTA epilogues, against the oracle;
+    wq_gemm_noalloc gives the same bits."""
+    import torch
+    case = wq_inputs.custom(M, K, N, bits, G, seed=M + bits)
+    d = to_dev(case, cuda)
+    bias_np = wq_inputs.bias_vector(N, seed=9)
+    bias = torch.from_numpy(bias_np).to(cuda)
+    w_q, w_lo = libwq.pack_kmajor(d["codes"], bits)
+    y = libwq.gemm(d["x"], w_q, w_lo, d["scales"], d["zeros"], bits, G, bias=bias)
+    y2 = torch.empty_like(y)
+    libwq.gemm_noalloc(d["x"], w_q, w_lo, d["scales"], d["zeros"], bits, G, out=y2, bias=bias)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2)
+    wq_, wlo_ = orc.pack(case.codes, bits)
+    y_ref, b = orc.wq_matmul(case.x, wq_, wlo_, case.scales, case.zeros, bits, G, bias=bias_np)
+    check_product(y.cpu().numpy(), y_ref, b, f"gemm {M}x{K}x{N} + bias")

@@ -187,6 +187,24 @@ def test_inputs_ready_plan_matches_oracle(cuda, libwq, orc, name):
     assert libwq.device_status() == 0
 
 
+@pytest.mark.parametrize("name,ready", [("tiny_gemv", False), ("decode_gemv_m1", True),
+                                        ("decode_gemv_m16", False), ("gemv_3bit", True)])
+def test_bias_matches_oracle(cuda, libwq, orc, name, ready):
+    """y = x @ w + bias, every output against the oracle (bound includes |bias|)."""
+    import torch
+    case = wq_inputs.draw(wq_inputs.WORKLOADS[name], seed=0)
+    d = to_dev(case, cuda)
+    bias = wq_inputs.bias_vector(case.wl.N, seed=5)
+    w_q, w_lo = libwq.pack_kmajor(d["codes"], case.wl.bits)
+    torch.cuda.synchronize()
+    y = libwq.gemv(d["x"], w_q, w_lo, d["scales"], d["zeros"], case.wl.bits, case.wl.group_size,
+                   bias=torch.from_numpy(bias).to(cuda), inputs_ready=ready).cpu().numpy()
+    wq_, wlo_ = orc.pack(case.codes, case.wl.bits)
+    y_ref, b = orc.wq_matmul(case.x, wq_, wlo_, case.scales, case.zeros, case.wl.bits,
+                             case.wl.group_size, bias=bias)
+    check_product(y, y_ref, b, name + " + bias")
+
+
 def test_deterministic(cuda, libwq):
     case = wq_inputs.draw(wq_inputs.WORKLOADS["decode_gemv_m4"], seed=1)
     d = to_dev(case, cuda)

@@ -32,7 +32,7 @@ def test_rejects_shapes_beyond_the_scratch(libwq):
     19 MiB (148 SMs, also assumed without a device): rejected before launch."""
     L = libwq.lib()
     assert L.wq_gemm_workspace_size(256, 4096, 9472, 4, 128) > SCRATCH_BYTES
-    st = L.wq_gemm_noalloc(P, P, None, P, P, P, 256, 4096, 9472, 4, 128, 0, None)
+    st = L.wq_gemm_noalloc(P, P, None, P, P, None, P, 256, 4096, 9472, 4, 128, 0, None)
     assert st == SCRATCH_LIMIT
     assert L.wq_status_string(SCRATCH_LIMIT)
 

@@ -92,3 +92,9 @@ def x_batch(M: int, K: int, seed: int) -> np.ndarray:
     """A fresh fp16 ``(M, K)`` activation block ~ N(0, 1)."""
     rng = np.random.default_rng(seed)
     return np.ascontiguousarray(rng.standard_normal((M, K)).astype(np.float16))
+
+
+def bias_vector(N: int, seed: int) -> np.ndarray:
+    """A fused-bias vector: fp16 ``(N,)`` ~ U[-1, 1]."""
+    rng = np.random.default_rng(seed)
+    return np.ascontiguousarray(rng.uniform(-1.0, 1.0, size=N).astype(np.float16))
