@@ -92,14 +92,22 @@ def _torch():
 
 def _stream():
     torch = _torch()
-    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+    if raw is not None:  # the handle without building a Stream object per call
+        return raw(torch.cuda.current_device())
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    return None if t is None else t.data_ptr()
 
 
 def _need(t, dtype, name, ndim=2):
+    try:  # the common case in one expression; the messages below only on failure
+        if t.is_cuda and t.dtype == dtype and t.dim() == ndim and t.is_contiguous():
+            return
+    except AttributeError:
+        pass
     torch = _torch()
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
@@ -173,7 +181,11 @@ def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, worksp
             M, K, N, bits, group_size, flags]
     if workspace is not False:  # wq_gemm: (workspace, bytes)
         if workspace is None:
-            workspace = _cached_workspace(x.device, gemm_workspace_size(M, K, N, bits, group_size))
+            key = (x.device.index, M, K, N, bits, group_size)
+            need = _ws_sizes.get(key)
+            if need is None:
+                need = _ws_sizes[key] = gemm_workspace_size(M, K, N, bits, group_size)
+            workspace = _cached_workspace(x.device, need)
         args += [_ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size()]
     st = getattr(lib(), fn)(*args, _stream())
     _check(fn, st)
@@ -197,6 +209,7 @@ def gemm_workspace_size(M: int, K: int, N: int, bits: int, group_size: int) -> i
 
 
 _workspaces = {}
+_ws_sizes = {}
 
 
 def _cached_workspace(device, nbytes: int):

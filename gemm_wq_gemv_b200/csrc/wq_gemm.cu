@@ -460,11 +460,13 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     cfg.stream = stream;
     cudaLaunchAttribute attrs[2];
     int na = 0;
-    attrs[na].id = cudaLaunchAttributeClusterDimension;
-    attrs[na].val.clusterDim.x = 1;
-    attrs[na].val.clusterDim.y = 1;
-    attrs[na].val.clusterDim.z = CS;
-    ++na;
+    if (CS > 1) {  // a cluster of one CTA is no cluster: launch without the attribute
+        attrs[na].id = cudaLaunchAttributeClusterDimension;
+        attrs[na].val.clusterDim.x = 1;
+        attrs[na].val.clusterDim.y = 1;
+        attrs[na].val.clusterDim.z = CS;
+        ++na;
+    }
     if (pb.flags & (WQ_FLAG_PDL | WQ_FLAG_PDL_INPUTS_READY)) {
         attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attrs[na].val.programmaticStreamSerializationAllowed = 1;

@@ -28,6 +28,9 @@
 //    x values of that group slice, so fractional zero points are exact and
 //    q == z gives exactly 0.
 #include <algorithm>
+#include <array>
+#include <map>
+#include <mutex>
 #include <type_traits>
 
 #include "wq_dequant.cuh"
@@ -579,95 +582,121 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     prm.qpg_shift = (prm.qpg & (prm.qpg - 1)) == 0 ? ilog2(prm.qpg) : -1;
     prm.n_groups = (pb.K + pb.G - 1) / pb.G;
     const int colblocks = (pb.N + COLS - 1) / COLS;
-    const int sms = sm_count();
 
-    auto layout = [&](int WK, int CS, int QW, Params& q, bool one_slot = false) -> size_t {
-        q.WK = WK; q.CS = CS; q.QW = QW;
-        const int rows_cta = WK * QW * 4;
-        const int quads_cta = WK * QW;
-        const int ch = EPS >= 8 ? EPS : 8;
-        q.cpt_shift = ilog2(rows_cta * EPS / ch);
-        q.qc_shift = ilog2(quads_cta);
-        q.groups_cta = std::min((quads_cta * QK + pb.G - 1) / pb.G + 1, (pb.K + pb.G - 1) / pb.G);
-        q.xs_tok_stride = rows_cta * EPS * 2 + 16;
-        q.nst = (QW > SQ && !one_slot) ? 2 : 1;
-        size_t off = (size_t)WK * q.nst * stage_bytes<BITS>();
-        q.off_bar = (uint32_t)off;
-        off += (size_t)WK * MAXST * 8 + 8;  // per-warp stage barriers, then the s/z barrier
-        off = (off + 127) & ~(size_t)127;
-        q.sz_box = std::min(q.groups_cta, 256);
-        q.sz_rows = (q.groups_cta + q.sz_box - 1) / q.sz_box * q.sz_box;
-        q.off_sz = (uint32_t)off;
-        q.sz_stride = (uint32_t)(((size_t)q.sz_rows * COLS * 2 + 127) & ~(size_t)127);
-        off += (size_t)2 * q.sz_stride;
-        q.off_x = (uint32_t)off;
-        off += (size_t)pb.M * q.xs_tok_stride;
-        off = (off + 15) & ~(size_t)15;
-        q.off_xq = (uint32_t)off;
-        off += (size_t)pb.M * quads_cta * 4;
-        off = (off + 15) & ~(size_t)15;
-        q.off_tab = (uint32_t)off;
-        off += (size_t)q.groups_cta * COLS * sizeof(Rec<BITS>);
-        q.off_red = (uint32_t)off;
-        off += (size_t)WK * pb.M * COLS * 4;
-        q.off_part = (uint32_t)off;
-        off += (size_t)pb.M * COLS * 4;
-        return off + 1024;  // slack for aligning the base to 1024 bytes
+    // The plan depends on the shape and flags only: computed once per device and
+    // kept (its occupancy queries would otherwise cost more than the launch).
+    struct Plan {
+        Params q;
+        size_t smem;
     };
-
+    static std::mutex plan_mu;
+    static std::map<std::array<int, 6>, Plan> plans;
+    const std::array<int, 6> key{dev, pb.M, pb.K, pb.N, pb.G, prm.late_wait};
     bool found = false;
     Params best{};
     size_t best_smem = 0;
-    long best_score = 0;
-    // Products that overlap the previous one (WQ_FLAG_PDL_INPUTS_READY) gain
-    // most from small CTAs: 8 warps and one stage slot per warp keep shared
-    // memory low enough for three or more CTAs per SM, so several launches
-    // stream at once.  Used when there are enough column blocks to fill the SMs.
-    if (prm.late_wait && colblocks >= sms / 2) {
-        int QW = 1;
-        while (QW * 8 < prm.Q) QW <<= 1;
-        Params q = prm;
-        const size_t sm = layout(8, 1, QW, q, true);
-        int occ = 0;
-        if (sm <= 227 * 1024) {
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 8 * 32, sm);
-            cudaGetLastError();
-        }
-        if (occ >= 3) {
+    {
+        std::lock_guard<std::mutex> lk(plan_mu);
+        const auto it = plans.find(key);
+        if (it != plans.end()) {
+            best = it->second.q;
+            best_smem = it->second.smem;
             found = true;
-            best = q;
-            best_smem = sm;
         }
     }
-    // Otherwise, among (warps per CTA, cluster size), pick the plan with the
-    // fewest waves x quads per warp; ties go to no cluster and larger CTAs.
-    for (int WK : {16, 8, 4}) {
-        if (found && best_score == 0) break;
-        for (int CS : {1, 2, 4, 8}) {
-            if (CS > 1 && WK * CS > prm.Q) continue;
+    if (!found) {
+        const int sms = sm_count();
+
+        auto layout = [&](int WK, int CS, int QW, Params& q, bool one_slot = false) -> size_t {
+            q.WK = WK; q.CS = CS; q.QW = QW;
+            const int rows_cta = WK * QW * 4;
+            const int quads_cta = WK * QW;
+            const int ch = EPS >= 8 ? EPS : 8;
+            q.cpt_shift = ilog2(rows_cta * EPS / ch);
+            q.qc_shift = ilog2(quads_cta);
+            q.groups_cta = std::min((quads_cta * QK + pb.G - 1) / pb.G + 1, (pb.K + pb.G - 1) / pb.G);
+            q.xs_tok_stride = rows_cta * EPS * 2 + 16;
+            q.nst = (QW > SQ && !one_slot) ? 2 : 1;
+            size_t off = (size_t)WK * q.nst * stage_bytes<BITS>();
+            q.off_bar = (uint32_t)off;
+            off += (size_t)WK * MAXST * 8 + 8;  // per-warp stage barriers, then the s/z barrier
+            off = (off + 127) & ~(size_t)127;
+            q.sz_box = std::min(q.groups_cta, 256);
+            q.sz_rows = (q.groups_cta + q.sz_box - 1) / q.sz_box * q.sz_box;
+            q.off_sz = (uint32_t)off;
+            q.sz_stride = (uint32_t)(((size_t)q.sz_rows * COLS * 2 + 127) & ~(size_t)127);
+            off += (size_t)2 * q.sz_stride;
+            q.off_x = (uint32_t)off;
+            off += (size_t)pb.M * q.xs_tok_stride;
+            off = (off + 15) & ~(size_t)15;
+            q.off_xq = (uint32_t)off;
+            off += (size_t)pb.M * quads_cta * 4;
+            off = (off + 15) & ~(size_t)15;
+            q.off_tab = (uint32_t)off;
+            off += (size_t)q.groups_cta * COLS * sizeof(Rec<BITS>);
+            q.off_red = (uint32_t)off;
+            off += (size_t)WK * pb.M * COLS * 4;
+            q.off_part = (uint32_t)off;
+            off += (size_t)pb.M * COLS * 4;
+            return off + 1024;  // slack for aligning the base to 1024 bytes
+        };
+
+        long best_score = 0;
+        // Products that overlap the previous one (WQ_FLAG_PDL_INPUTS_READY) gain
+        // most from small CTAs: 8 warps and one stage slot per warp keep shared
+        // memory low enough for three or more CTAs per SM, so several launches
+        // stream at once.  Used when there are enough column blocks to fill the SMs.
+        if (prm.late_wait && colblocks >= sms / 2) {
             int QW = 1;
-            while (QW * WK * CS < prm.Q) QW <<= 1;
+            while (QW * 8 < prm.Q) QW <<= 1;
             Params q = prm;
-            const size_t sm = layout(WK, CS, QW, q);
-            if (sm > 227 * 1024) continue;
+            const size_t sm = layout(8, 1, QW, q, true);
             int occ = 0;
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, WK * 32, sm);
-            cudaGetLastError();
-            if (occ <= 0) continue;
-            const long ctas = (long)colblocks * CS;
-            const long waves = (ctas + (long)occ * sms - 1) / ((long)occ * sms);
-            // per-warp serial work (quads, at least a full ring of them) x waves,
-            // plus a penalty for the cluster reduction
-            const long score = waves * std::max(QW, SQ) * 64 + (CS > 1 ? 96 : 0) + (16 / WK);
-            if (!found || score < best_score) {
+            if (sm <= 227 * 1024) {
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 8 * 32, sm);
+                cudaGetLastError();
+            }
+            if (occ >= 3) {
                 found = true;
                 best = q;
                 best_smem = sm;
-                best_score = score;
             }
         }
+        // Otherwise, among (warps per CTA, cluster size), pick the plan with the
+        // fewest waves x quads per warp; ties go to no cluster and larger CTAs.
+        for (int WK : {16, 8, 4}) {
+            if (found && best_score == 0) break;
+            for (int CS : {1, 2, 4, 8}) {
+                if (CS > 1 && WK * CS > prm.Q) continue;
+                int QW = 1;
+                while (QW * WK * CS < prm.Q) QW <<= 1;
+                Params q = prm;
+                const size_t sm = layout(WK, CS, QW, q);
+                if (sm > 227 * 1024) continue;
+                int occ = 0;
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, WK * 32, sm);
+                cudaGetLastError();
+                if (occ <= 0) continue;
+                const long ctas = (long)colblocks * CS;
+                const long waves = (ctas + (long)occ * sms - 1) / ((long)occ * sms);
+                // per-warp serial work (quads, at least a full ring of them) x waves,
+                // plus a penalty for the cluster reduction
+                const long score = waves * std::max(QW, SQ) * 64 + (CS > 1 ? 96 : 0) + (16 / WK);
+                if (!found || score < best_score) {
+                    found = true;
+                    best = q;
+                    best_smem = sm;
+                    best_score = score;
+                }
+            }
+        }
+        if (!found) return WQ_ERR_INVALID_ARG;  // shape too large for the shared-memory plan
+        std::lock_guard<std::mutex> lk(plan_mu);
+        plans.emplace(key, Plan{best, best_smem});
     }
-    if (!found) return WQ_ERR_INVALID_ARG;  // shape too large for the shared-memory plan
+    // this call's arrays
+    best.x = pb.x; best.w_q = pb.w_q; best.w_lo = pb.w_lo; best.s = pb.scales; best.z = pb.zeros;
+    best.bias = pb.bias; best.y = pb.y;
 
     CUtensorMap mw, ml, ms, mz;
     bool ok = make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, pb.w_q, pb.N, prm.Kw, (uint64_t)pb.N * 4, COLS, 4 * SQ,
@@ -690,11 +719,13 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     cfg.stream = stream;
     cudaLaunchAttribute attrs[2];
     int na = 0;
-    attrs[na].id = cudaLaunchAttributeClusterDimension;
-    attrs[na].val.clusterDim.x = 1;
-    attrs[na].val.clusterDim.y = best.CS;
-    attrs[na].val.clusterDim.z = 1;
-    ++na;
+    if (best.CS > 1) {  // a cluster of one CTA is no cluster: launch without the attribute
+        attrs[na].id = cudaLaunchAttributeClusterDimension;
+        attrs[na].val.clusterDim.x = 1;
+        attrs[na].val.clusterDim.y = best.CS;
+        attrs[na].val.clusterDim.z = 1;
+        ++na;
+    }
     if (pb.flags & (WQ_FLAG_PDL | WQ_FLAG_PDL_INPUTS_READY)) {
         attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attrs[na].val.programmaticStreamSerializationAllowed = 1;
