@@ -14,6 +14,7 @@ Entry points (same names as the C ABI, without the ``wq_`` prefix):
 * ``gemm(x, w_q, w_lo, scales, zeros, bits, group_size, out=None, pdl=False,
   workspace=None, inputs_ready=False, bias=None) -> y``
 * ``gemm_workspace_size(M, K, N, bits, group_size) -> bytes``
+* ``matmul(...)``: same arguments as ``gemm``; ``wq_gemv`` or ``wq_gemm`` by M
 * ``gemm_noalloc(x, w_q, w_lo, scales, zeros, bits, group_size, out) -> out``
 """
 from __future__ import annotations
@@ -68,6 +69,12 @@ def lib() -> ctypes.CDLL:
         L.wq_gemm_workspace_size.argtypes = [i, i, i, i, i]
         L.wq_gemm_workspace_size.restype = ctypes.c_size_t
         L.wq_gemm_noalloc.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, u, p]
+        L.wq_matmul.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, u, p, ctypes.c_size_t, p]
+        L.wq_matmul.restype = i
+        L.wq_matmul_uses_gemv.argtypes = [i, i, i, i, i]
+        L.wq_matmul_uses_gemv.restype = i
+        L.wq_matmul_workspace_size.argtypes = [i, i, i, i, i]
+        L.wq_matmul_workspace_size.restype = ctypes.c_size_t
         L.wq_gemm_noalloc.restype = i
         L.wq_device_status.argtypes = [i]
         for f in ("wq_pack_kmajor", "wq_unpack_kmajor", "wq_gemv", "wq_gemm", "wq_device_status"):
@@ -181,10 +188,11 @@ def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, worksp
             M, K, N, bits, group_size, flags]
     if workspace is not False:  # wq_gemm: (workspace, bytes)
         if workspace is None:
-            key = (x.device.index, M, K, N, bits, group_size)
+            key = (fn, x.device.index, M, K, N, bits, group_size)
             need = _ws_sizes.get(key)
-            if need is None:
-                need = _ws_sizes[key] = gemm_workspace_size(M, K, N, bits, group_size)
+            if need is None:  # wq_matmul's size is wq_gemm's on that route, else 0
+                query = lib().wq_matmul_workspace_size if fn == "wq_matmul" else lib().wq_gemm_workspace_size
+                need = _ws_sizes[key] = int(query(M, K, N, bits, group_size))
             workspace = _cached_workspace(x.device, need)
         args += [_ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size()]
     st = getattr(lib(), fn)(*args, _stream())
@@ -262,3 +270,18 @@ def gemm_noalloc(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out, p
     _need(out, torch.float16, "out")
     return _product("wq_gemm_noalloc", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl,
                     bias=bias)
+
+
+def matmul(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl: bool = False,
+           workspace=None, inputs_ready: bool = False, bias=None):
+    """``wq_matmul``: the product for any M, on ``wq_gemv`` or ``wq_gemm`` by the
+    library's measured M crossover (``uses_gemv`` tells which)."""
+    if workspace is not None:
+        torch = _torch()
+        _need(workspace, torch.uint8, "workspace", ndim=1)
+    return _product("wq_matmul", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, workspace,
+                    inputs_ready=inputs_ready, bias=bias)
+
+
+def uses_gemv(M: int, K: int, N: int, bits: int, group_size: int) -> bool:
+    return bool(lib().wq_matmul_uses_gemv(M, K, N, bits, group_size))

@@ -148,6 +148,29 @@ size_t wq_gemm_workspace_size(int M, int K, int N, int bits, int group_size) {
     return wq::gemm_workspace_bytes(M, K, N, bits, G);
 }
 
+int wq_matmul_uses_gemv(int M, int K, int N, int bits, int group_size) {
+    if (!supported_bits(bits) || M < 1 || K < 1 || N < 1) return 0;
+    const int G = group_size == -1 ? K : group_size;
+    const bool gemv_group = G == K || (G > 0 && G % (4 * main_eps(bits)) == 0);
+    const bool small_m = M <= 8 || (M <= 16 && (long long)M * K < 65536);
+    return (gemv_group && small_m) ? 1 : 0;
+}
+
+size_t wq_matmul_workspace_size(int M, int K, int N, int bits, int group_size) {
+    return wq_matmul_uses_gemv(M, K, N, bits, group_size) ? 0
+                                                         : wq_gemm_workspace_size(M, K, N, bits, group_size);
+}
+
+wq_status wq_matmul(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
+                    const uint16_t* scales, const uint16_t* zeros, const uint16_t* bias, uint16_t* y,
+                    int M, int K, int N, int bits, int group_size, unsigned flags, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+    if (wq_matmul_uses_gemv(M, K, N, bits, group_size))
+        return wq_gemv(x, w_q, w_lo, scales, zeros, bias, y, M, K, N, bits, group_size, flags, stream);
+    return wq_gemm(x, w_q, w_lo, scales, zeros, bias, y, M, K, N, bits, group_size, flags, workspace,
+                   workspace_bytes, stream);
+}
+
 wq_status wq_device_status(int reset) {
     const wq_status a = wq::gemm_device_status(reset);
     const wq_status b = wq::gemv_device_status(reset);

@@ -130,7 +130,6 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     // group of quad q (G = qpg * QK): a shift for the usual power-of-two group sizes
     auto gdiv = [&](int q) { return p.qpg_shift >= 0 ? (q >> p.qpg_shift) : q / p.qpg; };
     const int g_cta0 = gdiv(min(cta_q0, p.Q - 1));
-    const int n_groups = p.n_groups;
     const int nrec = p.groups_cta * COLS;
     Rec<BITS>* tab = reinterpret_cast<Rec<BITS>*>(smem + p.off_tab);
     bool any_frac = false;
@@ -356,7 +355,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
         constexpr uint32_t CS8 = 8 * RS;  // record stride between the lane's columns
         // bias constants of the lane's 4 columns, in registers for narrow records
         constexpr bool CREG = NC <= 2;
-        uint32_t creg[4][CREG ? NC : 1];
+        [[maybe_unused]] uint32_t creg[4][CREG ? NC : 1];
         auto load_creg = [&]() {
             if constexpr (CREG) {
 #pragma unroll
@@ -374,7 +373,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
         const uint32_t off_odd = (uint32_t)t * 128 + (((uint32_t)cg ^ (uint32_t)(t + 4)) << 4);
         // 3-bit lo plane: row R >> 1 = 2 iq + (t >> 1), swizzled with ((R >> 1) & 7)
         const uint32_t tl = (uint32_t)(t >> 1);
-        const uint32_t lo_off[4] = {tl * 128 + (((uint32_t)cg ^ tl) << 4), tl * 128 + (((uint32_t)cg ^ (tl + 2)) << 4),
+        [[maybe_unused]] const uint32_t lo_off[4] = {tl * 128 + (((uint32_t)cg ^ tl) << 4), tl * 128 + (((uint32_t)cg ^ (tl + 2)) << 4),
                                     tl * 128 + (((uint32_t)cg ^ (tl + 4)) << 4), tl * 128 + (((uint32_t)cg ^ (tl + 6)) << 4)};
 
         auto quad = [&](uint32_t stage, int iq, int i) {

@@ -154,6 +154,25 @@ wq_status wq_gemm(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
                   uint16_t* y, int M, int K, int N, int bits, int group_size, unsigned flags,
                   void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * The product for any M, routed to wq_gemv or wq_gemm by a measured crossover
+ * (the M-crossover of the "next" list; not in the pages): wq_gemv when
+ * M <= 8, or M <= 16 with M * K < 65536 (x then fits its on-chip staging),
+ * and the group size is one wq_gemv takes; wq_gemm otherwise.  Same arguments
+ * and rules as wq_gemm; the workspace is used only on the wq_gemm route
+ * (wq_matmul_workspace_size() reports 0 on the other).
+ */
+wq_status wq_matmul(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
+                    const uint16_t* scales, const uint16_t* zeros, const uint16_t* bias,
+                    uint16_t* y, int M, int K, int N, int bits, int group_size, unsigned flags,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* 1 if wq_matmul takes the wq_gemv route for this shape, 0 if wq_gemm (host-only). */
+int wq_matmul_uses_gemv(int M, int K, int N, int bits, int group_size);
+
+/* Workspace bytes wq_matmul uses for this shape (host-only). */
+size_t wq_matmul_workspace_size(int M, int K, int N, int bits, int group_size);
+
 /* Workspace bytes wq_gemm uses for this shape (0 when it does not split K, or
  * when the arguments are invalid).  Host-only; needs no device. */
 size_t wq_gemm_workspace_size(int M, int K, int N, int bits, int group_size);

@@ -114,3 +114,24 @@ def test_pack_argument_checks(libwq):
     assert L.wq_pack_kmajor(None, 32, 4, 4, P, None, None, None) == 1
     assert L.wq_pack_kmajor(P, 32, 4, 4, P + 2, None, None, None) == 3
     assert L.wq_unpack_kmajor(P, P, 32, 4, 4, P, None) == 1          # w_lo with 4-bit
+
+
+def test_matmul_route(libwq):
+    """wq_matmul's crossover: wq_gemv for M <= 8, or M <= 16 with M * K < 65536,
+    when the group size is one wq_gemv takes; wq_gemm otherwise."""
+    L = libwq.lib()
+    route = lambda *a: int(L.wq_matmul_uses_gemv(*a))
+    assert route(1, 4096, 4096, 4, 128) == 1
+    assert route(8, 8192, 8192, 4, 128) == 1
+    assert route(12, 4096, 4096, 4, 128) == 1
+    assert route(12, 8192, 4096, 4, 128) == 0      # 12 x 8192 >= 65536
+    assert route(16, 4096, 4096, 4, 128) == 0      # 16 x 4096 = 65536
+    assert route(17, 512, 256, 4, 128) == 0
+    assert route(1, 4096, 4096, 4, 16) == 0        # group 16 is wq_gemm's only
+    assert route(1, 4096, 4096, 4, -1) == 1
+    assert route(1, 4096, 4096, 5, 128) == 0
+    assert int(L.wq_matmul_workspace_size(1, 4096, 4096, 4, 128)) == 0
+    assert int(L.wq_matmul_workspace_size(512, 4096, 2048, 4, 128)) == \
+        int(L.wq_gemm_workspace_size(512, 4096, 2048, 4, 128))
+    # argument checks pass through: M = 0 is rejected before anything runs
+    assert L.wq_matmul(P, P, None, P, P, None, P, 0, 512, 256, 4, 128, 0, None, ctypes.c_size_t(0), None) == 1

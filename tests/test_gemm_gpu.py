@@ -180,3 +180,16 @@ def test_bias_matches_oracle(cuda, libwq, orc, M, K, N, bits, G):
     wq_, wlo_ = orc.pack(case.codes, bits)
     y_ref, b = orc.wq_matmul(case.x, wq_, wlo_, case.scales, case.zeros, bits, G, bias=bias_np)
     check_product(y.cpu().numpy(), y_ref, b, f"gemm {M}x{K}x{N} + bias")
+
+
+@pytest.mark.parametrize("M", [1, 12, 16, 64])
+def test_matmul_either_route_matches_oracle(cuda, libwq, orc, M):
+    """wq_matmul over the crossover: both routes against the oracle."""
+    K, N = 4096, 512
+    case = wq_inputs.custom(M, K, N, 4, 128, seed=40 + M)
+    d = to_dev(case, cuda)
+    w_q, w_lo = libwq.pack_kmajor(d["codes"], 4)
+    y = libwq.matmul(d["x"], w_q, w_lo, d["scales"], d["zeros"], 4, 128).cpu().numpy()
+    assert libwq.uses_gemv(M, K, N, 4, 128) == (M <= 12)
+    y_ref, b = oracle_product(orc, case)
+    check_product(y, y_ref, b, f"matmul M={M}")
