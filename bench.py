@@ -116,6 +116,24 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+# ------------------------------------------------------------------ replicas
+def replica_max(v: float, dist=None, device=None) -> float:
+    """The largest of every rank's `v` (a time: the job ends with its slowest
+    replica); `v` itself without a process group."""
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_step: float, steps: int, world: int, elapsed_s: float) -> float:
+    """Whole-job throughput: every replica processes `units_per_step` per step
+    (weak scaling), timed by the slowest replica's `elapsed_s`."""
+    return units_per_step * steps * world / elapsed_s
+
+
 # ------------------------------------------------------------------ helpers
 def src_digest() -> str:
     h = hashlib.sha1()
@@ -357,11 +375,7 @@ def main(argv=None):
             dist.barrier()
 
     def max_over_ranks(v):
-        if not dist:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replica_max(v, dist, dev)
 
     from gemm_wq_gemv_b200 import build as wq_build
     wq_build.build()
@@ -380,7 +394,7 @@ def main(argv=None):
     el = time_graph(torch, g, s, args.steps, args.warmup, barrier, sampler)
     el = max_over_ranks(el)
     bytes_step = algo_bytes(wl) * L
-    value = bytes_step * args.steps * world / el / 1e9
+    value = job_rate(bytes_step, args.steps, world, el) / 1e9
     per_launch_s = el / (args.steps * L)
     achieved = algo_bytes(wl) / per_launch_s / 1e9
     traffic = ncu_traffic("gemv_kernel<4,_1>", HEADLINE)
@@ -419,7 +433,7 @@ def main(argv=None):
     for _ in range(e2e_steps):
         e2e_step()
     e2e_el = max_over_ranks(time.perf_counter() - t0)
-    e2e_value = bytes_step * e2e_steps * world / e2e_el / 1e9
+    e2e_value = job_rate(bytes_step, e2e_steps, world, e2e_el) / 1e9
     del stack, g
 
     # ---- GEMM: M=512 prefill product
