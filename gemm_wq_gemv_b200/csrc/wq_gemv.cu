@@ -11,7 +11,7 @@
 //    thread-block cluster split K further and reduce their fp32 partial sums
 //    through distributed shared memory.  One launch, no workspace, no atomics.
 //  * Loads.  Each warp streams its K range with 2-D TMA boxes of 32 word rows
-//    x 32 columns (8 quads, 128-byte swizzle) into two shared-memory stages,
+//    x 32 columns (8 quads, 128-byte swizzle) into one or two shared-memory stages,
 //    completing on an mbarrier: the bytes in flight cost neither registers nor
 //    L1 request slots.  Lane (g, t) (g = lane / 4, t = lane % 4) then reads one
 //    16-byte vector per quad (4 adjacent columns of one word row); the column
@@ -27,6 +27,9 @@
 //  * Per group, acc += s * (D - (z - round(z)) * X) in fp32, X = the sum of the
 //    x values of that group slice, so fractional zero points are exact and
 //    q == z gives exactly 0.
+//  * s and z of the CTA's groups arrive with one TMA copy each and become
+//    per-(group, column) records in shared memory; the optional bias is added
+//    to the fp32 sum before the fp16 rounding.
 #include <algorithm>
 #include <array>
 #include <map>
