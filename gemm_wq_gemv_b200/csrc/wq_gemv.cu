@@ -508,9 +508,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     else
         main_loop(std::false_type{});
 
-    // ---- reduce over the warps of the CTA (and write y: with late_wait, only
+    // ---- reduce over the warps of the CTA, then write y (with late_wait, only
     // once the previous kernel on the stream has completed)
-    if (p.late_wait) grid_dependency_wait();
     float* red = reinterpret_cast<float*>(smem + p.off_red);  // [WK][M][COLS]
 #pragma unroll
     for (int c = 0; c < 4; ++c)
@@ -529,6 +528,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
         }
         // reduce over the CTAs of the cluster through distributed shared memory
         cluster_sync();
+        if (p.late_wait) grid_dependency_wait();
         const uint32_t part_addr = smem_u32(part);
         for (int i = rank + p.CS * (int)threadIdx.x; i < p.M * COLS; i += p.CS * blockDim.x) {
             float sacc = 0.0f;
@@ -541,6 +541,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
         }
         cluster_sync();  // peers keep their shared memory until every read is done
     } else {
+        if (p.late_wait) grid_dependency_wait();
         for (int i = threadIdx.x; i < p.M * COLS; i += blockDim.x) {
             const float sacc = sum_warps(red, p.WK, p.M * COLS, i);
             const int m = i / COLS, col = col0 + i % COLS;
