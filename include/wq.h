@@ -64,7 +64,7 @@ typedef enum {
 } wq_status;
 
 /*
- * Launch flags for wq_gemv / wq_gemm.
+ * Launch flags for wq_gemv, wq_gemm, wq_matmul and wq_gemm_noalloc.
  * WQ_FLAG_PDL: launch as a programmatic dependent of the previous kernel on
  *   the stream.  The kernel may start while that kernel still runs: it streams
  *   w_q, w_lo, scales and zeros at once and reads x only after the previous
@@ -174,7 +174,8 @@ int wq_matmul_uses_gemv(int M, int K, int N, int bits, int group_size);
 size_t wq_matmul_workspace_size(int M, int K, int N, int bits, int group_size);
 
 /* Workspace bytes wq_gemm uses for this shape (0 when it does not split K, or
- * when the arguments are invalid).  Host-only; needs no device. */
+ * when the arguments are invalid).  Host-only: it reads the current device's
+ * SM count (148 when there is no device). */
 size_t wq_gemm_workspace_size(int M, int K, int N, int bits, int group_size);
 
 /*
@@ -194,7 +195,8 @@ size_t wq_gemm_workspace_size(int M, int K, int N, int bits, int group_size);
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
  *   - Calls that may run at the same time on one device (other streams, other
- *     host threads) share the array and race; calls in one stream do not.
+ *     host threads) share the array and race; calls in one stream do not,
+ *     WQ_FLAG_PDL_INPUTS_READY included (it waits before the scratch is used).
  *   - A shape whose wq_gemm_workspace_size() exceeds the array is rejected
  *     with WQ_ERR_SCRATCH_LIMIT before anything is launched.
  */
