@@ -1,0 +1,34 @@
+"""Host-side behaviour of the Python binding that needs no GPU: it refuses CPU
+tensors (there is no CPU path) and fails loudly when libwq.so is missing."""
+from pathlib import Path
+
+import pytest
+import torch
+
+
+def test_cpu_tensors_are_refused(libwq):
+    x = torch.zeros((1, 64), dtype=torch.float16)
+    w = torch.zeros((8, 8), dtype=torch.int32)
+    s = torch.zeros((1, 8), dtype=torch.float16)
+    for fn in (libwq.gemv, libwq.gemm, libwq.matmul):
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            fn(x, w, None, s, s, 4, 64)
+
+
+def test_non_tensor_is_refused(libwq):
+    with pytest.raises(TypeError, match="torch.Tensor"):
+        libwq.gemv([[0.0]], None, None, None, None, 4, 64)
+
+
+def test_missing_library_fails_loudly(libwq, monkeypatch):
+    monkeypatch.setattr(libwq, "_lib", None)
+    monkeypatch.setattr(libwq, "LIB_PATH", Path("/nonexistent/libwq.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        libwq.lib()
+
+
+def test_status_names(libwq):
+    assert libwq.STATUS[7] == "WQ_ERR_SCRATCH_LIMIT"
+    assert "scratch" in libwq.describe(7)
+    err = libwq.WQError("wq_gemv", 3)
+    assert err.status == 3 and "WQ_ERR_ALIGNMENT" in str(err)
