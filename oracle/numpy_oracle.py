@@ -15,6 +15,10 @@ check each other.  It follows the same passages:
   is one group per output channel.
 
 The matmul step is NumPy's fp64 matmul (a library primitive).
+
+Floating-point inputs are fp16 (NumPy ``float16``) or bf16 (``uint16`` bit
+patterns): a bf16 value is the upper half of the binary32 with the same top 16
+bits, so it widens through NumPy's ``float32``.
 """
 from __future__ import annotations
 
@@ -65,23 +69,37 @@ def unpack(wq, wlo, K: int, N: int, bits: int) -> np.ndarray:
     return unpack_plane(wq, bits)[:K].astype(np.uint8)
 
 
-def dequant(wq, wlo, scales, zeros, K: int, N: int, bits: int, group_size: int) -> np.ndarray:
+def widen(a, dtype: str = "fp16") -> np.ndarray:
+    """fp16 / bf16 values as fp64."""
+    if dtype == "bf16":
+        u = np.asarray(a)
+        if u.dtype != np.uint16:
+            raise ValueError("bf16 arrays are passed as uint16 bit patterns")
+        return (u.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    if dtype != "fp16":
+        raise ValueError(f"unsupported dtype {dtype}")
+    return np.asarray(a, dtype=np.float16).astype(np.float64)
+
+
+def dequant(wq, wlo, scales, zeros, K: int, N: int, bits: int, group_size: int,
+            dtype: str = "fp16") -> np.ndarray:
     G = K if group_size == -1 else group_size
     q = unpack(wq, wlo, K, N, bits).astype(np.float64)
-    s = np.repeat(np.asarray(scales, dtype=np.float16).astype(np.float64), G, axis=0)
-    z = np.repeat(np.asarray(zeros, dtype=np.float16).astype(np.float64), G, axis=0)
+    s = np.repeat(widen(scales, dtype), G, axis=0)
+    z = np.repeat(widen(zeros, dtype), G, axis=0)
     return (q - z) * s
 
 
-def wq_matmul(x, wq, wlo, scales, zeros, bits: int, group_size: int, N: int | None = None, bias=None):
-    """y = x @ w (+ bias[n], one fp16 value per output column, as the module's
+def wq_matmul(x, wq, wlo, scales, zeros, bits: int, group_size: int, N: int | None = None, bias=None,
+              dtype: str = "fp16"):
+    """y = x @ w (+ bias[n], one value per output column, as the module's
     forward adds it), and the bound sum |x w| (+ |bias|)."""
-    x = np.asarray(x, dtype=np.float16).astype(np.float64)
+    x = widen(x, dtype)
     K = x.shape[1]
     N = np.asarray(wq).shape[1] if N is None else N
-    w = dequant(wq, wlo, scales, zeros, K, N, bits, group_size)
+    w = dequant(wq, wlo, scales, zeros, K, N, bits, group_size, dtype)
     y, b = x @ w, np.abs(x) @ np.abs(w)
     if bias is not None:
-        bv = np.asarray(bias, dtype=np.float16).astype(np.float64).reshape(1, N)
+        bv = widen(bias, dtype).reshape(1, N)
         y, b = y + bv, b + np.abs(bv)
     return y, b

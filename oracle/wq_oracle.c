@@ -24,8 +24,12 @@
  *                                dashq_kernel.py `forward`, batched branch)
  *   B[m][n]  = sum_k |x[m][k] * w[k][n]|   (the scale of the error bound)
  *
- * fp16 inputs are widened to double exactly, from the IEEE 754 binary16
- * definition (sign, 5-bit exponent with bias 15, 10-bit fraction).
+ * The floating-point inputs (x, s, z, bias) are all fp16 or all bf16 (the
+ * module's `out_dtype`, dashq_kernel.py `TritonQuantLinear.__init__`), chosen
+ * by the `dt` argument: ORC_FP16 (0) or ORC_BF16 (1).  Both are widened to
+ * double exactly from their definitions: IEEE 754 binary16 (sign, 5-bit
+ * exponent with bias 15, 10-bit fraction) and bfloat16 (sign, 8-bit exponent
+ * with bias 127, 7-bit fraction: the upper half of a binary32).
  *
  * Words are handled as uint32 bit patterns with logical shifts; the pages'
  * torch code uses int32 with arithmetic shifts and a mask, which gives the same
@@ -46,6 +50,9 @@
 #define ORC_EBITS (-2)       /* a bit width outside {1, 2, 3, 4, 8} */
 #define ORC_ERANGE (-3)      /* a code that does not fit in `bits` bits */
 #define ORC_ENOMEM (-4)
+
+#define ORC_FP16 0
+#define ORC_BF16 1
 
 int orc_threads(void) {
 #ifdef _OPENMP
@@ -78,6 +85,36 @@ double orc_half_to_double(uint16_t h) {
         v = ldexp((double)(1024 + f), e - 25);   /* (1 + f/1024) * 2^(e-15) */
     }
     return sign ? -v : v;
+}
+
+/* bfloat16 -> double, exact. */
+double orc_bf16_to_double(uint16_t h) {
+    int sign = (h >> 15) & 1;
+    int e = (h >> 7) & 0xff;
+    int f = h & 0x7f;
+    double v;
+    if (e == 0) {
+        v = ldexp((double)f, -133);              /* subnormal: f * 2^-126 * 2^-7 */
+    } else if (e == 255) {
+        v = f ? NAN : INFINITY;
+    } else {
+        v = ldexp((double)(128 + f), e - 134);   /* (1 + f/128) * 2^(e-127) */
+    }
+    return sign ? -v : v;
+}
+
+/* One stored value of type dt widened to double. */
+static double widen(uint16_t h, int dt) {
+    return dt == ORC_BF16 ? orc_bf16_to_double(h) : orc_half_to_double(h);
+}
+
+static int supported_dt(int dt) { return dt == ORC_FP16 || dt == ORC_BF16; }
+
+/* out[i] = the value of v[i] (type dt) as a double. */
+int orc_widen(const uint16_t* v, int n, int dt, double* out) {
+    if (n < 0 || !supported_dt(dt)) return ORC_EARG;
+    for (int i = 0; i < n; ++i) out[i] = widen(v[i], dt);
+    return ORC_OK;
 }
 
 static int supported_bits(int bits) {
@@ -153,18 +190,18 @@ static int resolve_group(int K, int group_size) {
 
 /* w_kn[k][n] = (q - z[g][n]) * s[g][n] in fp64, g = k / G. */
 int orc_dequant(const uint32_t* wq, const uint32_t* wlo, const uint16_t* s, const uint16_t* z,
-                int K, int N, int bits, int group_size, double* w_kn) {
+                int K, int N, int bits, int group_size, double* w_kn, int dt) {
     if (!supported_bits(bits)) return ORC_EBITS;
     int G = resolve_group(K, group_size);
-    if (G < 0 || N <= 0) return ORC_EARG;
+    if (G < 0 || N <= 0 || !supported_dt(dt)) return ORC_EARG;
     int kdiv = bits == 3 ? 32 : elems_per_word(bits);
     if (K % kdiv != 0) return ORC_EARG;
     for (int k = 0; k < K; ++k) {
         int g = k / G;
         for (int n = 0; n < N; ++n) {
             double q = (double)code_at(wq, wlo, N, bits, k, n);
-            double zz = orc_half_to_double(z[(size_t)g * N + n]);
-            double ss = orc_half_to_double(s[(size_t)g * N + n]);
+            double zz = widen(z[(size_t)g * N + n], dt);
+            double ss = widen(s[(size_t)g * N + n], dt);
             w_kn[(size_t)k * N + n] = (q - zz) * ss;
         }
     }
@@ -172,11 +209,12 @@ int orc_dequant(const uint32_t* wq, const uint32_t* wlo, const uint16_t* s, cons
 }
 
 /* y[m][n] = sum_k x[m][k] * w[k][n] (k ascending), bound[m][n] = sum_k |x w|. */
-int orc_matmul(const uint16_t* x, const double* w_kn, int M, int K, int N, double* y, double* bound) {
-    if (M <= 0 || K <= 0 || N <= 0) return ORC_EARG;
+int orc_matmul(const uint16_t* x, const double* w_kn, int M, int K, int N, double* y, double* bound,
+               int dt) {
+    if (M <= 0 || K <= 0 || N <= 0 || !supported_dt(dt)) return ORC_EARG;
     double* xd = (double*)malloc(sizeof(double) * (size_t)M * K);
     if (!xd) return ORC_ENOMEM;
-    for (size_t i = 0; i < (size_t)M * K; ++i) xd[i] = orc_half_to_double(x[i]);
+    for (size_t i = 0; i < (size_t)M * K; ++i) xd[i] = widen(x[i], dt);
 #pragma omp parallel for schedule(static)
     for (int n = 0; n < N; ++n) {
         for (int m = 0; m < M; ++m) {
@@ -197,27 +235,27 @@ int orc_matmul(const uint16_t* x, const double* w_kn, int M, int K, int N, doubl
 /* The whole product: unpack, dequantise, fp64 matmul. */
 int orc_wq_matmul(const uint16_t* x, const uint32_t* wq, const uint32_t* wlo, const uint16_t* s,
                   const uint16_t* z, int M, int K, int N, int bits, int group_size,
-                  double* y, double* bound) {
+                  double* y, double* bound, int dt) {
     if (M <= 0) return ORC_EARG;
     double* w = (double*)malloc(sizeof(double) * (size_t)K * N);
     if (!w) return ORC_ENOMEM;
-    int rc = orc_dequant(wq, wlo, s, z, K, N, bits, group_size, w);
-    if (rc == ORC_OK) rc = orc_matmul(x, w, M, K, N, y, bound);
+    int rc = orc_dequant(wq, wlo, s, z, K, N, bits, group_size, w, dt);
+    if (rc == ORC_OK) rc = orc_matmul(x, w, M, K, N, y, bound, dt);
     free(w);
     return rc;
 }
 
 /*
  * Fused bias ("dashq_kernel.py" `TritonQuantLinear.forward`: the output of
- * the product plus `bias`, one fp16 value per output column):
+ * the product plus `bias`, one value per output column, of type dt):
  * y[m][n] += bias[n], and the bias is one more addend of the error bound,
  * bound[m][n] += |bias[n]|.
  */
-int orc_add_bias(double* y, double* bound, const uint16_t* bias, int M, int N) {
-    if (M <= 0 || N <= 0 || !bias) return ORC_EARG;
+int orc_add_bias(double* y, double* bound, const uint16_t* bias, int M, int N, int dt) {
+    if (M <= 0 || N <= 0 || !bias || !supported_dt(dt)) return ORC_EARG;
     for (int m = 0; m < M; ++m)
         for (int n = 0; n < N; ++n) {
-            double b = orc_half_to_double(bias[n]);
+            double b = widen(bias[n], dt);
             y[(size_t)m * N + n] += b;
             if (bound) bound[(size_t)m * N + n] += fabs(b);
         }
@@ -232,10 +270,10 @@ int orc_add_bias(double* y, double* bound, const uint16_t* bias, int M, int N) {
 int orc_wq_matmul_sampled(const uint16_t* x, const uint32_t* wq, const uint32_t* wlo,
                           const uint16_t* s, const uint16_t* z, int M, int K, int N, int bits,
                           int group_size, const int32_t* ms, const int32_t* ns, int count,
-                          double* y, double* bound) {
+                          double* y, double* bound, int dt) {
     if (!supported_bits(bits)) return ORC_EBITS;
     int G = resolve_group(K, group_size);
-    if (G < 0 || M <= 0 || N <= 0) return ORC_EARG;
+    if (G < 0 || M <= 0 || N <= 0 || !supported_dt(dt)) return ORC_EARG;
     int kdiv = bits == 3 ? 32 : elems_per_word(bits);
     if (K % kdiv != 0) return ORC_EARG;
     for (int i = 0; i < count; ++i)
@@ -247,9 +285,8 @@ int orc_wq_matmul_sampled(const uint16_t* x, const uint32_t* wq, const uint32_t*
         for (int k = 0; k < K; ++k) {
             int g = k / G;
             double q = (double)code_at(wq, wlo, N, bits, k, n);
-            double w = (q - orc_half_to_double(z[(size_t)g * N + n])) *
-                       orc_half_to_double(s[(size_t)g * N + n]);
-            double p = orc_half_to_double(x[(size_t)m * K + k]) * w;
+            double w = (q - widen(z[(size_t)g * N + n], dt)) * widen(s[(size_t)g * N + n], dt);
+            double p = widen(x[(size_t)m * K + k], dt) * w;
             acc += p;
             b += fabs(p);
         }

@@ -13,7 +13,10 @@ under test or from the CUDA library:
   with NumPy's matmul); per-channel equals grouped when all groups share
   ``s, z``; ``group_size = -1`` equals ``group_size = K``;
 * brute force: every single-code matrix of a tiny shape packs to the one word
-  the layout rule predicts.
+  the layout rule predicts;
+* bf16 inputs: values that fp16 and bf16 both hold exactly give the same
+  product as fp16; powers of two beyond fp16's range (bit patterns written
+  from the bfloat16 field layout) give products known in closed form.
 """
 from __future__ import annotations
 
@@ -244,6 +247,65 @@ def pin_bias(impl):
             assert np.array_equal(y[k], row + bias64), (bits, "one-hot", k)
 
 
+def _bf16_exact(a):
+    """bf16 bit patterns of values that bfloat16 holds exactly (checked)."""
+    f = np.asarray(a, dtype=np.float64).astype(np.float32)
+    u = f.view(np.uint32)
+    assert np.all((u & np.uint32(0xFFFF)) == 0), "value not exact in bf16"
+    return (u >> np.uint32(16)).astype(np.uint16)
+
+
+def _bf16_pow2(e):
+    """bf16 pattern of 2**e from the field layout: exponent field e + 127 at bit 7
+    (normal), or fraction bit e + 133 (subnormal, e in [-133, -127))."""
+    if e >= -126:
+        return np.uint16((e + 127) << 7)
+    return np.uint16(1 << (e + 133))
+
+
+def pin_bf16_same_values_as_fp16(impl):
+    """Values that both formats hold exactly (8 significant bits, inside fp16's
+    normal range) give the same y and bound whether passed as fp16 or bf16."""
+    for bits in BITS:
+        kd = _kdiv(bits)
+        K, N, M, G = 4 * kd, 7, 3, 2 * kd
+        rng = _rng(500 + bits)
+        x = rng.integers(-255, 256, size=(M, K)) * 2.0 ** rng.integers(-9, 3, size=(M, K))
+        s = rng.integers(1, 256, size=(K // G, N)) * 2.0 ** -14
+        z = rng.integers(0, 2 * min(1 << bits, 128), size=(K // G, N)) / 2.0 - 0.5  # 8 bits
+        bias = rng.integers(-255, 256, size=N) * 2.0 ** -5
+        codes = rng.integers(0, 1 << bits, size=(K, N)).astype(np.uint8)
+        wq, wlo = impl.pack(codes, bits)
+        y16, b16 = impl.wq_matmul(x.astype(np.float16), wq, wlo, s.astype(np.float16),
+                                  z.astype(np.float16), bits, G, bias=bias.astype(np.float16))
+        yb, bb = impl.wq_matmul(_bf16_exact(x), wq, wlo, _bf16_exact(s), _bf16_exact(z), bits, G,
+                                bias=_bf16_exact(bias), dtype="bf16")
+        assert np.array_equal(y16, yb), bits
+        assert np.array_equal(b16, bb), bits
+        assert np.any(y16 != 0), bits
+
+
+def pin_bf16_beyond_fp16_range(impl):
+    """x = 2**e1 e_k, s = 2**e2 with e1, e2 outside fp16's range (one of them a
+    bf16 subnormal): row k is (q - z) * 2**(e1 + e2) exactly, plus the bias."""
+    bits, K, N, G = 4, 16, 5, 8
+    rng = _rng(600)
+    codes = rng.integers(0, 16, size=(K, N)).astype(np.uint8)
+    zq = rng.integers(0, 16, size=(K // G, N))
+    wq, wlo = impl.pack(codes, bits)
+    for e1, e2 in ((100, -110), (-120, 30), (60, -130), (-20, -20)):
+        x = np.zeros((K, K), dtype=np.uint16)
+        x[np.arange(K), np.arange(K)] = _bf16_pow2(e1)
+        s = np.full((K // G, N), _bf16_pow2(e2), dtype=np.uint16)
+        z = _bf16_exact(zq)
+        bias = np.full(N, _bf16_pow2(-3) | np.uint16(0x8000), dtype=np.uint16)  # -1/8
+        y, b = impl.wq_matmul(x, wq, wlo, s, z, bits, G, bias=bias, dtype="bf16")
+        for k in range(K):
+            row = (codes[k].astype(np.float64) - zq[k // G]) * 2.0 ** (e1 + e2)
+            assert np.array_equal(y[k], row - 0.125), (e1, e2, k)
+            assert np.array_equal(b[k], np.abs(row) + 0.125), (e1, e2, k)
+
+
 PINS = [
     pin_golden_pack,
     pin_golden_products,
@@ -256,4 +318,6 @@ PINS = [
     pin_group_equivalences,
     pin_group_index,
     pin_bias,
+    pin_bf16_same_values_as_fp16,
+    pin_bf16_beyond_fp16_range,
 ]

@@ -20,10 +20,10 @@ def _mutant(**overrides):
     return m
 
 
-def _with_bias(y, b, bias, N, sign=1.0, by_row=False):
+def _with_bias(y, b, bias, N, sign=1.0, by_row=False, dtype="fp16", widen=tw.widen):
     if bias is None:
         return y, b
-    bv = np.asarray(bias, np.float16).astype(np.float64)
+    bv = widen(bias, dtype)
     if by_row:  # indexed by the token instead of the output column
         bv = np.resize(bv, y.shape[0]).reshape(-1, 1)
     else:
@@ -31,31 +31,50 @@ def _with_bias(y, b, bias, N, sign=1.0, by_row=False):
     return y + sign * bv, b + np.abs(bv)
 
 
-def _matmul_with(dequant_fn, bias_sign=1.0, bias_by_row=False, bias_used=True):
-    def wq_matmul(x, wq, wlo, s, z, bits, G, N=None, bias=None):
-        x = np.asarray(x, np.float16).astype(np.float64)
+def _matmul_with(dequant_fn, bias_sign=1.0, bias_by_row=False, bias_used=True, widen=tw.widen):
+    def wq_matmul(x, wq, wlo, s, z, bits, G, N=None, bias=None, dtype="fp16"):
+        x = widen(x, dtype)
         K = x.shape[1]
         N = np.asarray(wq).shape[1] if N is None else N
-        w = dequant_fn(wq, wlo, s, z, K, N, bits, G)
+        w = dequant_fn(wq, wlo, s, z, K, N, bits, G, dtype)
         return _with_bias(x @ w, np.abs(x) @ np.abs(w), bias if bias_used else None, N,
-                          bias_sign, bias_by_row)
+                          bias_sign, bias_by_row, dtype, widen)
     return wq_matmul
 
 
-def _transposed(x, wq, wlo, s, z, bits, G, N=None, bias=None):
-    xx = np.asarray(x, np.float16).astype(np.float64)
+def _transposed(x, wq, wlo, s, z, bits, G, N=None, bias=None, dtype="fp16"):
+    xx = tw.widen(x, dtype)
     N = np.asarray(wq).shape[1] if N is None else N
-    w = tw.dequant(wq, wlo, s, z, xx.shape[1], N, bits, G)
+    w = tw.dequant(wq, wlo, s, z, xx.shape[1], N, bits, G, dtype)
     y = xx @ (w.T if w.shape[0] == w.shape[1] else w[::-1])
-    return _with_bias(y, np.abs(xx) @ np.abs(w), bias, N)
+    return _with_bias(y, np.abs(xx) @ np.abs(w), bias, N, dtype=dtype)
 
 
-def _dq(q_fn=None, combine=lambda q, z, s: (q - z) * s, expand=np.repeat):
-    def dequant(wq, wlo, s, z, K, N, bits, G):
+def _bf16_as_fp16(a, dtype="fp16"):  # bf16 patterns read as binary16
+    if dtype == "bf16":
+        return np.asarray(a, np.uint16).view(np.float16).astype(np.float64)
+    return tw.widen(a, dtype)
+
+
+def _bf16_bias_126(a, dtype="fp16"):  # bf16 exponent bias off by one
+    return tw.widen(a, dtype) * (2.0 if dtype == "bf16" else 1.0)
+
+
+def _bf16_fraction_8(a, dtype="fp16"):  # bf16 split as 7 exponent + 8 fraction bits
+    if dtype != "bf16":
+        return tw.widen(a, dtype)
+    u = np.asarray(a, np.uint16).astype(np.int64)
+    e, f = (u >> 8) & 0x7F, u & 0xFF
+    v = np.where(e == 0, f * 2.0 ** -70, (256 + f) * 2.0 ** (e - 63 - 8))
+    return np.where(u & 0x8000, -v, v)
+
+
+def _dq(q_fn=None, combine=lambda q, z, s: (q - z) * s, expand=np.repeat, widen=tw.widen):
+    def dequant(wq, wlo, s, z, K, N, bits, G, dtype="fp16"):
         Gr = K if G == -1 else G
         q = (q_fn or tw.unpack)(wq, wlo, K, N, bits).astype(np.float64)
-        s64 = np.asarray(s, np.float16).astype(np.float64)
-        z64 = np.asarray(z, np.float16).astype(np.float64)
+        s64 = widen(s, dtype)
+        z64 = widen(z, dtype)
         if expand is np.repeat:
             s64, z64 = np.repeat(s64, Gr, axis=0), np.repeat(z64, Gr, axis=0)
         else:
@@ -125,6 +144,12 @@ MUTANTS = {
     "bias_dropped": _mutant(wq_matmul=_matmul_with(tw.dequant, bias_used=False)),
     "bias_sign_flipped": _mutant(wq_matmul=_matmul_with(tw.dequant, bias_sign=-1.0)),
     "bias_indexed_by_token": _mutant(wq_matmul=_matmul_with(tw.dequant, bias_by_row=True)),
+    "bf16_read_as_fp16": _mutant(wq_matmul=_matmul_with(_dq(widen=_bf16_as_fp16), widen=_bf16_as_fp16)),
+    "bf16_exponent_bias_126": _mutant(wq_matmul=_matmul_with(_dq(widen=_bf16_bias_126),
+                                                             widen=_bf16_bias_126)),
+    "bf16_fraction_width_8": _mutant(wq_matmul=_matmul_with(_dq(widen=_bf16_fraction_8),
+                                                            widen=_bf16_fraction_8)),
+    "bf16_scale_read_as_fp16": _mutant(wq_matmul=_matmul_with(_dq(widen=_bf16_as_fp16))),
     "bound_signed": _mutant(
         wq_matmul=lambda *a, **k: (lambda r: (r[0], np.abs(r[0])))(tw.wq_matmul(*a, **k))),
 }

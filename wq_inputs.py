@@ -15,6 +15,11 @@ Recipe (one ``numpy.random.default_rng(seed)`` stream, PCG64, drawn in this
 order): ``x`` ~ N(0, 1) rounded to fp16; codes uniform integers in
 ``[0, 2**bits - 1]``; scales uniform in ``[s_lo, s_hi]`` rounded to fp16;
 zeros uniform integers in ``[0, 2**bits - 1]`` stored as fp16.
+
+bf16 problems (``dtype="bf16"``) take the same draws from the same stream and
+round x and the scales to bfloat16 instead (round to nearest, ties to even);
+their x, scales, zeros and bias are ``uint16`` bit patterns, NumPy having no
+bfloat16 type.
 """
 from __future__ import annotations
 
@@ -52,6 +57,7 @@ class Case:
     zeros: np.ndarray    # (groups, N) float16, integer-valued
     seed: int = 0
     extra: dict = field(default_factory=dict)
+    dtype: str = "fp16"  # "bf16": x, scales, zeros hold bfloat16 bit patterns (uint16)
 
 
 # The named workloads: the small parity case, the decode GEMV at three token
@@ -70,31 +76,48 @@ WORKLOADS = {
 }
 
 
-def draw(wl: Workload, seed: int = 0) -> Case:
+def bf16_bits(a) -> np.ndarray:
+    """Finite values rounded to bfloat16 (nearest, ties to even), as uint16 bit patterns."""
+    u = np.ascontiguousarray(np.asarray(a, dtype=np.float64).astype(np.float32)).view(np.uint32)
+    u = u.astype(np.uint64)
+    r = (u + np.uint64(0x7FFF) + ((u >> np.uint64(16)) & np.uint64(1))) >> np.uint64(16)
+    return np.ascontiguousarray(r.astype(np.uint16))
+
+
+def _as(a, dtype: str) -> np.ndarray:
+    if dtype == "bf16":
+        return bf16_bits(a)
+    if dtype != "fp16":
+        raise ValueError(f"dtype must be 'fp16' or 'bf16', not {dtype!r}")
+    return np.ascontiguousarray(np.asarray(a).astype(np.float16))
+
+
+def draw(wl: Workload, seed: int = 0, dtype: str = "fp16") -> Case:
     """Draw one problem for workload ``wl`` from ``default_rng(seed)``."""
     rng = np.random.default_rng(seed)
-    x = rng.standard_normal((wl.M, wl.K)).astype(np.float16)
+    x = rng.standard_normal((wl.M, wl.K))
     qmax = (1 << wl.bits) - 1
     codes = rng.integers(0, qmax + 1, size=(wl.K, wl.N), dtype=np.int64).astype(np.uint8)
-    scales = rng.uniform(wl.s_lo, wl.s_hi, size=(wl.groups, wl.N)).astype(np.float16)
-    zeros = rng.integers(0, qmax + 1, size=(wl.groups, wl.N), dtype=np.int64).astype(np.float16)
-    return Case(wl, np.ascontiguousarray(x), np.ascontiguousarray(codes),
-                np.ascontiguousarray(scales), np.ascontiguousarray(zeros), seed)
+    scales = rng.uniform(wl.s_lo, wl.s_hi, size=(wl.groups, wl.N))
+    zeros = rng.integers(0, qmax + 1, size=(wl.groups, wl.N), dtype=np.int64)
+    return Case(wl, _as(x, dtype), np.ascontiguousarray(codes), _as(scales, dtype),
+                _as(zeros, dtype), seed, dtype=dtype)
 
 
 def custom(M: int, K: int, N: int, bits: int, group_size: int, seed: int = 0,
-           s_lo: float = 0.005, s_hi: float = 0.02, name: str = "custom") -> Case:
+           s_lo: float = 0.005, s_hi: float = 0.02, name: str = "custom",
+           dtype: str = "fp16") -> Case:
     """Draw a problem of arbitrary shape with the same distributions."""
-    return draw(Workload(name, M, K, N, bits, group_size, s_lo, s_hi), seed)
+    return draw(Workload(name, M, K, N, bits, group_size, s_lo, s_hi), seed, dtype)
 
 
-def x_batch(M: int, K: int, seed: int) -> np.ndarray:
-    """A fresh fp16 ``(M, K)`` activation block ~ N(0, 1)."""
+def x_batch(M: int, K: int, seed: int, dtype: str = "fp16") -> np.ndarray:
+    """A fresh ``(M, K)`` activation block ~ N(0, 1)."""
     rng = np.random.default_rng(seed)
-    return np.ascontiguousarray(rng.standard_normal((M, K)).astype(np.float16))
+    return _as(rng.standard_normal((M, K)), dtype)
 
 
-def bias_vector(N: int, seed: int) -> np.ndarray:
-    """A fused-bias vector: fp16 ``(N,)`` ~ U[-1, 1]."""
+def bias_vector(N: int, seed: int, dtype: str = "fp16") -> np.ndarray:
+    """A fused-bias vector ``(N,)`` ~ U[-1, 1]."""
     rng = np.random.default_rng(seed)
-    return np.ascontiguousarray(rng.uniform(-1.0, 1.0, size=N).astype(np.float16))
+    return _as(rng.uniform(-1.0, 1.0, size=N), dtype)
