@@ -13,7 +13,8 @@ the products (packed words + s + z + x + y) per second, whole job.
 
 Also measured on the same box, in the same run:
 * ``gemm``: the batched product M=512, K=4096, N=2048 (4-bit, group 128) in TFLOP/s;
-* ``workloads``: every synthetic workload (bit-width sweep, 3-bit planes, M=4/16);
+* ``workloads``: every synthetic workload (bit-width sweep, 3-bit planes, M=4/16),
+  with fp16 and with bf16 x, scales, zeros and y;
 * ``e2e``: the headline metric through the Python API with host buffers (x copied
   in and y copied out every step);
 * ``cpu_baseline``: the CPU oracle (plain C, fp64) on a bounded sample.
@@ -159,19 +160,25 @@ def ncu_traffic(kernel: str, workload: str):
 class Stack:
     """L distinct weight sets of one workload on the device, plus x / y per set."""
 
-    def __init__(self, wq, torch, wl, L, dev, seed0=0):
+    def __init__(self, wq, torch, wl, L, dev, seed0=0, dtype="fp16"):
         import numpy as np
         self.wl, self.L = wl, L
-        base = wq_inputs.draw(wl, seed=seed0)
+        base = wq_inputs.draw(wl, seed=seed0, dtype=dtype)
         codes = torch.from_numpy(base.codes).to(dev)
         w_q, w_lo = wq.pack_kmajor(codes, wl.bits)
-        s = torch.from_numpy(base.scales).to(dev)
-        z = torch.from_numpy(base.zeros).to(dev)
+
+        def dev_array(a):  # bf16 inputs are uint16 bit patterns on the host
+            if dtype == "bf16":
+                return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+            return torch.from_numpy(a).to(dev)
+
+        s = dev_array(base.scales)
+        z = dev_array(base.zeros)
         del codes
         self.sets = []
         for i in range(L):
-            x = torch.from_numpy(wq_inputs.x_batch(wl.M, wl.K, seed=1000 + i)).to(dev)
-            y = torch.empty((wl.M, wl.N), dtype=torch.float16, device=dev)
+            x = dev_array(wq_inputs.x_batch(wl.M, wl.K, seed=1000 + i, dtype=dtype))
+            y = torch.empty((wl.M, wl.N), dtype=x.dtype, device=dev)
             self.sets.append((x, w_q.clone() if i else w_q, None if w_lo is None else (w_lo.clone() if i else w_lo),
                               s.clone() if i else s, z.clone() if i else z, y))
         self.np = np
@@ -397,7 +404,7 @@ def main(argv=None):
     value = job_rate(bytes_step, args.steps, world, el) / 1e9
     per_launch_s = el / (args.steps * L)
     achieved = algo_bytes(wl) / per_launch_s / 1e9
-    traffic = ncu_traffic("gemv_kernel<4,_1>", HEADLINE)
+    traffic = ncu_traffic("gemv_kernel<4,_1,_0>", HEADLINE)
 
     # ---- the same stack as a dependency chain (x of each product = y of the previous)
     cg, cs = capture(torch, lambda: stack.run_chain(wq))
@@ -467,7 +474,7 @@ def main(argv=None):
     gel = max_over_ranks(time_graph(torch, gg, gs, gsteps, args.warmup, barrier))
     g_launch_s = gel / (gsteps * GL)
     g_tflops = algo_flops(gwl) / g_launch_s / 1e12
-    g_traffic = ncu_traffic("gemm_kernel<4>", GEMM_WL)
+    g_traffic = ncu_traffic("gemm_kernel<4,_0>", GEMM_WL)
     del gstack, gg
 
     # ---- context: the same kernel on a large product (no split-K, many k blocks),
@@ -503,16 +510,16 @@ def main(argv=None):
     # ---- every workload once (rank-local, for the table)
     table = []
     if not args.no_secondary:
-        for name, w in wq_inputs.WORKLOADS.items():
+        for dtype, (name, w) in [(d, nw) for d in ("fp16", "bf16") for nw in wq_inputs.WORKLOADS.items()]:
             fn = wq.gemm if w.M > 16 else wq.gemv
             n_l = layers_for(w, L2)
-            stk = Stack(wq, torch, w, n_l, dev)
+            stk = Stack(wq, torch, w, n_l, dev, dtype=dtype)
             gr, st_ = capture(torch, lambda: stk.run(wq, fn, inputs_ready=True))
             reps = 20
             t = time_graph(torch, gr, st_, reps, 3)
             us = t / (reps * n_l) * 1e6
-            row = {"workload": name, "M": w.M, "K": w.K, "N": w.N, "bits": w.bits, "group": w.group_size,
-                   "kernel": "gemm" if fn is wq.gemm else "gemv", "us": round(us, 3)}
+            row = {"workload": name, "dtype": dtype, "M": w.M, "K": w.K, "N": w.N, "bits": w.bits,
+                   "group": w.group_size, "kernel": "gemm" if fn is wq.gemm else "gemv", "us": round(us, 3)}
             if fn is wq.gemm:
                 tfl = algo_flops(w) / (us * 1e-6) / 1e12
                 row.update({"TFLOPS": round(tfl, 1), "frac": round(tfl / tf_peak, 4)})

@@ -16,6 +16,9 @@ Entry points (same names as the C ABI, without the ``wq_`` prefix):
 * ``gemm_workspace_size(M, K, N, bits, group_size) -> bytes``
 * ``matmul(...)``: same arguments as ``gemm``; ``wq_gemv`` or ``wq_gemm`` by M
 * ``gemm_noalloc(x, w_q, w_lo, scales, zeros, bits, group_size, out) -> out``
+
+x, scales, zeros, bias and the output are all ``torch.float16`` or all
+``torch.bfloat16`` (the type of x decides; bfloat16 sets ``WQ_FLAG_BF16``).
 """
 from __future__ import annotations
 
@@ -37,6 +40,7 @@ STATUS = {
 }
 WQ_FLAG_PDL = 1
 WQ_FLAG_PDL_INPUTS_READY = 2
+WQ_FLAG_BF16 = 4
 
 _lib = None
 
@@ -166,24 +170,37 @@ def unpack_kmajor(w_q, w_lo, K: int, bits: int):
     return out
 
 
+def _elem_type(x):
+    """float16 or bfloat16: the type of x, which scales, zeros, bias and y share."""
+    torch = _torch()
+    dt = getattr(x, "dtype", None)
+    if dt is torch.float16 or dt is torch.bfloat16:
+        return dt
+    if isinstance(x, torch.Tensor):
+        raise TypeError(f"x must be torch.float16 or torch.bfloat16, got {dt}")
+    raise TypeError("x must be a torch.Tensor")
+
+
 def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, workspace=False,
              inputs_ready=False, bias=None):
     torch = _torch()
-    _need(x, torch.float16, "x")
+    dt = _elem_type(x)
+    _need(x, dt, "x")
     _need(w_q, torch.int32, "w_q")
     if w_lo is not None:
         _need(w_lo, torch.int32, "w_lo")
-    _need(scales, torch.float16, "scales")
-    _need(zeros, torch.float16, "zeros")
+    _need(scales, dt, "scales")
+    _need(zeros, dt, "zeros")
     if bias is not None:
-        _need(bias, torch.float16, "bias", ndim=1)
+        _need(bias, dt, "bias", ndim=1)
     M, K = x.shape
     N = w_q.shape[1]
     if out is None:
-        out = torch.empty((M, N), dtype=torch.float16, device=x.device)
+        out = torch.empty((M, N), dtype=dt, device=x.device)
     else:
-        _need(out, torch.float16, "out")
-    flags = (WQ_FLAG_PDL if pdl else 0) | (WQ_FLAG_PDL_INPUTS_READY if inputs_ready else 0)
+        _need(out, dt, "out")
+    flags = ((WQ_FLAG_PDL if pdl else 0) | (WQ_FLAG_PDL_INPUTS_READY if inputs_ready else 0)
+             | (WQ_FLAG_BF16 if dt is torch.bfloat16 else 0))
     args = [_ptr(x), _ptr(w_q), _ptr(w_lo), _ptr(scales), _ptr(zeros), _ptr(bias), _ptr(out),
             M, K, N, bits, group_size, flags]
     if workspace is not False:  # wq_gemm: (workspace, bytes)
@@ -202,11 +219,11 @@ def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, worksp
 
 def gemv(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl: bool = False,
          inputs_ready: bool = False, bias=None):
-    """y (M, N) fp16 = x (M, K) @ dequant(w_q), 1 <= M <= 16 (``wq_gemv``).
+    """y (M, N) = x (M, K) @ dequant(w_q), 1 <= M <= 16 (``wq_gemv``), in the type of x.
 
     ``pdl``: WQ_FLAG_PDL; ``inputs_ready``: WQ_FLAG_PDL_INPUTS_READY (the previous
     kernel on the stream writes none of this call's inputs); ``bias``: optional (N,)
-    fp16 tensor added to every row of the output."""
+    tensor of x's type added to every row of the output."""
     return _product("wq_gemv", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl,
                     inputs_ready=inputs_ready, bias=bias)
 
@@ -244,7 +261,7 @@ def _cached_workspace(device, nbytes: int):
 
 def gemm(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl: bool = False,
          workspace=None, inputs_ready: bool = False, bias=None):
-    """y (M, N) fp16 = x (M, K) @ dequant(w_q), any M >= 1 (``wq_gemm``).
+    """y (M, N) = x (M, K) @ dequant(w_q), any M >= 1 (``wq_gemm``), in the type of x.
 
     ``workspace``: a CUDA uint8 tensor of at least ``gemm_workspace_size(...)``
     bytes for splitting K over a cluster; by default one cached per stream.
@@ -266,8 +283,7 @@ def gemm_noalloc(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out, p
     """``wq_gemm_noalloc``: the product into the caller's ``out`` with the
     library's fixed split-K scratch; neither the call nor this wrapper
     allocates device memory."""
-    torch = _torch()
-    _need(out, torch.float16, "out")
+    _need(out, _elem_type(x), "out")
     return _product("wq_gemm_noalloc", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl,
                     bias=bias)
 

@@ -50,10 +50,11 @@ wq_status check_plane_shape(int K, int N, int bits, const void* w_lo, bool need_
 // Shared checks of wq_gemv / wq_gemm; resolves G.
 wq_status check_product(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
                         const uint16_t* s, const uint16_t* z, const uint16_t* y, int M, int K,
-                        int N, int bits, int group_size, int& G) {
+                        int N, int bits, int group_size, unsigned flags, int& G) {
     wq_status st = check_plane_shape(K, N, bits, w_lo, true);
     if (st != WQ_OK) return st;
     if (M < 1) return WQ_ERR_INVALID_ARG;
+    if (flags & ~WQ_FLAG_ALL) return WQ_ERR_INVALID_ARG;
     if (!x || !w_q || !s || !z || !y) return WQ_ERR_INVALID_ARG;
     if (group_size == -1) {
         G = K;
@@ -114,7 +115,7 @@ wq_status wq_gemv(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
                   const uint16_t* scales, const uint16_t* zeros, const uint16_t* bias, uint16_t* y,
                   int M, int K, int N, int bits, int group_size, unsigned flags, void* stream) {
     int G = 0;
-    wq_status st = check_product(x, w_q, w_lo, scales, zeros, y, M, K, N, bits, group_size, G);
+    wq_status st = check_product(x, w_q, w_lo, scales, zeros, y, M, K, N, bits, group_size, flags, G);
     if (st != WQ_OK) return st;
     if (bias && !aligned(bias, 2)) return WQ_ERR_ALIGNMENT;
     if (M > 16) return WQ_ERR_INVALID_ARG;
@@ -129,7 +130,7 @@ wq_status wq_gemm(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
                   int M, int K, int N, int bits, int group_size, unsigned flags, void* workspace,
                   size_t workspace_bytes, void* stream) {
     int G = 0;
-    wq_status st = check_product(x, w_q, w_lo, scales, zeros, y, M, K, N, bits, group_size, G);
+    wq_status st = check_product(x, w_q, w_lo, scales, zeros, y, M, K, N, bits, group_size, flags, G);
     if (st != WQ_OK) return st;
     if (bias && !aligned(bias, 2)) return WQ_ERR_ALIGNMENT;
     if (K % 64 != 0) return WQ_ERR_INVALID_ARG;

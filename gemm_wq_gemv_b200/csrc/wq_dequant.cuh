@@ -1,12 +1,19 @@
-// wq_dequant.cuh -- exact conversion of packed code pairs to fp16 (q - round(z)).
+// wq_dequant.cuh -- exact conversion of packed code pairs to fp16 or bf16 (q - round(z)).
 //
 // Shared by the GEMV and the GEMM.  Codes j and j + E/2 of a word (E codes per
 // word) sit at the same bit offset in the two 16-bit halves, so one LOP3 ORs
 // both into the mantissa of the fp16 constant 1024 (0x6400), and one exact
 // fp16x2 FMA brings them back to the integers q - zi, zi = round(z): every
 // value involved is an integer below 2048, so nothing rounds.
+//
+// bf16 has 7 fraction bits: the constant is 128 (0x4300), whose fraction holds
+// a code field only at bits 0-6, so each word is read through two to four
+// shifted copies; zi is kept in [0, 2^bits - 1] so that q - zi (|.| <= 255)
+// stays exact in bf16's 8 significant bits.  8-bit codes do not fit 7 bits:
+// they go through the fp32 constant 2^23 instead and are packed to bf16 pairs.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -16,20 +23,43 @@ namespace wq {
 
 // ----------------------------------------------------------------- formats
 // EPS: codes per word of the main plane (3-bit: the 2-bit plane).
-// NC:  number of distinct fp16 bias constants per (group, column).
+// NC:  number of distinct fp16 bias constants per (group, column); NCB: bf16.
 template <int BITS> struct Fmt;
-template <> struct Fmt<1> { static constexpr int EPS = 32, NC = 10; };
-template <> struct Fmt<2> { static constexpr int EPS = 16, NC = 5; };
-template <> struct Fmt<3> { static constexpr int EPS = 16, NC = 8; };
-template <> struct Fmt<4> { static constexpr int EPS = 8, NC = 2; };
-template <> struct Fmt<8> { static constexpr int EPS = 4, NC = 1; };
+template <> struct Fmt<1> { static constexpr int EPS = 32, NC = 10, NCB = 7; };
+template <> struct Fmt<2> { static constexpr int EPS = 16, NC = 5, NCB = 3; };
+template <> struct Fmt<3> { static constexpr int EPS = 16, NC = 8, NCB = 8; };
+template <> struct Fmt<4> { static constexpr int EPS = 8, NC = 2, NCB = 1; };
+template <> struct Fmt<8> { static constexpr int EPS = 4, NC = 1, NCB = 1; };
+
+template <int BITS, bool BF>
+constexpr int ncons() { return BF ? Fmt<BITS>::NCB : Fmt<BITS>::NC; }
 
 // Per (group, column) record in shared memory: fp32 scale, fp32 fractional zero
-// part, and NC bias constants as duplicated fp16 pairs.
-template <int BITS> struct alignas(16) Rec {
+// part, and the bias constants (duplicated fp16 / bf16 pairs; 8-bit bf16: one fp32).
+template <int BITS, bool BF> struct alignas(16) Rec {
     float s;
     float zr;
-    uint32_t c[Fmt<BITS>::NC];
+    uint32_t c[ncons<BITS, BF>()];
+};
+
+// ------------------------------------------------------------ element types
+// x, scales, zeros, bias and y share one 16-bit type: fp16 (BF = false) or bf16.
+template <bool BF> struct Dt;
+template <> struct Dt<false> {
+    static __device__ __forceinline__ float load(uint16_t v) { return __half2float(__ushort_as_half(v)); }
+    static __device__ __forceinline__ uint16_t store(float v) { return __half_as_ushort(__float2half_rn(v)); }
+    static __device__ __forceinline__ float2 pair(uint32_t u) {
+        return __half22float2(*reinterpret_cast<const __half2*>(&u));
+    }
+};
+template <> struct Dt<true> {
+    static __device__ __forceinline__ float load(uint16_t v) { return __uint_as_float((uint32_t)v << 16); }
+    static __device__ __forceinline__ uint16_t store(float v) {
+        return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    }
+    static __device__ __forceinline__ float2 pair(uint32_t u) {
+        return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+    }
 };
 
 // Bias constant for a code that sits at mantissa bit p of a 0x6400 word and is
@@ -56,11 +86,64 @@ __device__ __forceinline__ uint32_t dup_half(float v) {
     return (uint32_t)b | ((uint32_t)b << 16);
 }
 
+__device__ __forceinline__ uint32_t dup_bf16(float v) {
+    const uint16_t b = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    return (uint32_t)b | ((uint32_t)b << 16);
+}
+
+template <bool BF>
+__device__ __forceinline__ uint32_t dup_t(float v) { return BF ? dup_bf16(v) : dup_half(v); }
+
+// bf16 pair j of a 3-bit word: the hi field sits at bit PH3(j) of its shifted
+// copy, the lo bit at PL3(j).
+__device__ __forceinline__ constexpr int ph3_bf(int j) { return 2 * (j % 3) + 1; }
+__device__ __forceinline__ constexpr int pl3_bf(int j) { return j < 6 ? j + 1 : j - 5; }
+
+// bf16 bias magnitude of constant i: 128 * 2^-p for a code at bit p of 0x4300
+// (1-bit p = i; 2-bit p = 2 i; 4-bit p = 0).  3-bit: hi field at ph (multiplier
+// 2^(1-ph)) and lo bit at pl (multiplier 2^-pl): 2^(8-ph) + 2^(7-pl).  With
+// zi <= 2^bits - 1 every sum below has at most 8 significant bits.
+template <int BITS>
+__device__ __forceinline__ float bias_magnitude_bf(int i) {
+    if constexpr (BITS == 1) {
+        return (float)(128 >> i);
+    } else if constexpr (BITS == 2) {
+        return (float)(128 >> (2 * i));
+    } else if constexpr (BITS == 4) {
+        return 128.0f;
+    } else {
+        return (float)(1 << (8 - ph3_bf(i))) + (float)(1 << (7 - pl3_bf(i)));
+    }
+}
+
+// The integer zero point the exact conversion subtracts; the rest, z - zi, is
+// applied in fp32 (GEMV) or folded into the scale FMA (GEMM).
+template <int BITS, bool BF>
+__device__ __forceinline__ float zero_int(float z) {
+    if constexpr (BF) return fminf(fmaxf(rintf(z), 0.0f), (float)((1 << BITS) - 1));
+    else return fminf(fmaxf(rintf(z), -256.0f), 256.0f);
+}
+
+// Bias constant ci of a (group, column) whose integer zero point is zi.
+template <int BITS, bool BF>
+__device__ __forceinline__ uint32_t pair_const(int ci, float zi) {
+    if constexpr (!BF) {
+        return dup_half(-(bias_magnitude<BITS>(ci) + zi));
+    } else if constexpr (BITS == 8) {
+        return __float_as_uint(-(8388608.0f + zi));  // fp32: 2^23 + q minus 2^23 + zi
+    } else {
+        return dup_bf16(-(bias_magnitude_bf<BITS>(ci) + zi));
+    }
+}
+
 // fp16x2 constant with the same value in both lanes (compile-time exact values).
 __device__ __forceinline__ constexpr uint32_t h2c(uint32_t bits16) { return bits16 | (bits16 << 16); }
 
 // fp16 bit patterns of 2^-p, p = 0..10
 __device__ __forceinline__ constexpr uint32_t pow2neg_h(int p) { return (uint32_t)(15 - p) << 10; }
+
+// bf16 bit patterns of 2^-p, p = 0..7
+__device__ __forceinline__ constexpr uint32_t pow2neg_b(int p) { return (uint32_t)(127 - p) << 7; }
 
 // ------------------------------------------------------- pair dequantisation
 // Pair j of word w (codes j and j + EPS/2 in the low / high half) as fp16x2
@@ -120,5 +203,96 @@ __device__ __forceinline__ void prep_word(uint32_t& w, uint32_t& w_hi, uint32_t&
         w_hi = w;
     }
 }
+
+// ---------------------------------------------------- bf16 pair dequantisation
+// A word and the shifted copies of it that pair_bf reads.
+struct SrcB {
+    uint32_t a, b, c, d;  // main plane copies
+    uint32_t la, lb;      // 3-bit: lo plane copies
+};
+
+// 1-bit: w, w >> 7, w >> 14 (bits 0-6, 7-13, 14-15 of each half at bit 0);
+// 2-bit: w, w >> 6, w >> 12; 4-bit: w, w >> 4, w >> 8, w >> 12; 8-bit: w.
+// 3-bit: (hi << 1), hi >> 5, hi >> 11 put pair j's 2-bit field at bit
+// 2 (j % 3) + 1; the lo bits of the hi word's 16 codes (selected by lo_sel
+// as in prep_word) go to bit j + 1 (j < 6) or j - 5 (j >= 6).
+template <int BITS>
+__device__ __forceinline__ void prep_bf(uint32_t w, uint32_t lo_word, uint32_t lo_sel, SrcB& s) {
+    s.a = w;
+    s.b = s.c = s.d = s.la = s.lb = 0;
+    if constexpr (BITS == 1) {
+        s.b = w >> 7;
+        s.c = w >> 14;
+    } else if constexpr (BITS == 2) {
+        s.b = w >> 6;
+        s.c = w >> 12;
+    } else if constexpr (BITS == 4) {
+        s.b = w >> 4;
+        s.c = w >> 8;
+        s.d = w >> 12;
+    } else if constexpr (BITS == 3) {
+        s.a = w << 1;
+        s.b = w >> 5;
+        s.c = w >> 11;
+        const uint32_t ls = prmt(lo_word, 0u, lo_sel);
+        s.la = ls << 1;
+        s.lb = ls >> 5;
+    }
+}
+
+// Pair j (codes j and j + EPS/2 in the low / high half) as bf16x2 values q - zi.
+template <int BITS>
+__device__ __forceinline__ uint32_t pair_bf(const SrcB& s, const uint32_t (&c)[Fmt<BITS>::NCB], int j) {
+    constexpr uint32_t MAGIC = 0x43004300u;
+    if constexpr (BITS == 8) {
+        // bytes j and j + 2 into the low byte of the fp32 constant 2^23 (0x4B000000)
+        const float lo = __uint_as_float(prmt(s.a, 0x4B000000u, 0x7440u + j)) + __uint_as_float(c[0]);
+        const float hi = __uint_as_float(prmt(s.a, 0x4B000000u, 0x7442u + j)) + __uint_as_float(c[0]);
+        const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<const uint32_t*>(&v);
+    } else if constexpr (BITS == 4) {
+        const uint32_t src = j == 0 ? s.a : j == 1 ? s.b : j == 2 ? s.c : s.d;
+        return bfma2_u32(and_or(src, 0x000F000Fu, MAGIC), h2c(pow2neg_b(0)), c[0]);
+    } else if constexpr (BITS == 2) {
+        const uint32_t src = j < 3 ? s.a : j < 6 ? s.b : s.c;
+        const int i = j % 3;
+        return bfma2_u32(and_or(src, 0x00030003u << (2 * i), MAGIC), h2c(pow2neg_b(2 * i)), c[i]);
+    } else if constexpr (BITS == 1) {
+        const uint32_t src = j < 7 ? s.a : j < 14 ? s.b : s.c;
+        const int p = j % 7;
+        return bfma2_u32(and_or(src, 0x00010001u << p, MAGIC), h2c(pow2neg_b(p)), c[p]);
+    } else {
+        const uint32_t srch = j < 3 ? s.a : j < 6 ? s.b : s.c;
+        const uint32_t srcl = j < 6 ? s.la : s.lb;
+        const int ph = ph3_bf(j), pl = pl3_bf(j);
+        const uint32_t H = and_or(srch, 0x00030003u << ph, MAGIC);
+        const uint32_t L = and_or(srcl, 0x00010001u << pl, MAGIC);
+        const uint32_t T = bfma2_u32(H, h2c(pow2neg_b(ph - 1)), c[j]);
+        return bfma2_u32(L, h2c(pow2neg_b(pl)), T);
+    }
+}
+
+// ----------------------------------------------- one word, either element type
+template <int BITS, bool BF> struct Word;
+template <int BITS> struct Word<BITS, false> {
+    uint32_t w, wh, ls;
+    __device__ __forceinline__ void prep(uint32_t word, uint32_t lo_word, uint32_t lo_sel) {
+        w = word;
+        wh = ls = 0;
+        prep_word<BITS>(w, wh, ls, lo_word, lo_sel);
+    }
+    __device__ __forceinline__ uint32_t pair(const uint32_t (&c)[Fmt<BITS>::NC], int j) const {
+        return pair_q<BITS>(w, wh, ls, c, j);
+    }
+};
+template <int BITS> struct Word<BITS, true> {
+    SrcB s;
+    __device__ __forceinline__ void prep(uint32_t word, uint32_t lo_word, uint32_t lo_sel) {
+        prep_bf<BITS>(word, lo_word, lo_sel, s);
+    }
+    __device__ __forceinline__ uint32_t pair(const uint32_t (&c)[Fmt<BITS>::NCB], int j) const {
+        return pair_bf<BITS>(s, c, j);
+    }
+};
 
 }  // namespace wq

@@ -3,20 +3,22 @@
 // What is computed: "GPTQModel-Compatible Triton Kernel" README
 // (`gptqmodel_quantized_matmul`: output = x @ dequantize(qweight)) and the batched
 // branch of dashq_kernel.py `forward` (x @ dequantize_weight()), with fp32
-// accumulation and one fp16 rounding at the end.
+// accumulation and one rounding at the end.  x, s, z, the bias and y are all
+// fp16 or all bf16 (the module's `out_dtype`; the MMA takes both operands in it).
 //
 // How (sm_100a), per CTA = one tile of 128 weight columns x TN tokens x a K range:
 //  * The product is computed transposed (D = W^T x^T), so the 128 weight columns
 //    fill the MMA's M = 128 and the tokens are its N (16..256).  D lives in
 //    tensor memory: lane = weight column, column = token, fp32.
 //  * Warp 0 (one lane) streams each 64-deep k block with TMA into a ring of
-//    shared-memory stages: the x tile (TN x 64 fp16, 128-byte swizzle, which is
+//    shared-memory stages: the x tile (TN x 64 16-bit values, 128-byte swizzle, which is
 //    the MMA's K-major layout), the packed word tile (64 / eps rows x 128 columns),
 //    the 3-bit lo-plane tile and the s, z rows of the block's group(s).
 //  * Warps 2-9 (two threads per weight column, each taking half of the stage's
-//    word rows) turn that column's words into 32 fp16 values (q - z) * s each --
-//    code pairs become exact q - round(z) with one LOP3 + one FMA, are put in k
-//    order with PRMT and scaled with one more FMA -- and store them with
+//    word rows) turn that column's words into 32 values (q - z) * s each --
+//    code pairs become exact q - round(z) with one LOP3 + one FMA (bf16: see
+//    wq_dequant.cuh), are put in k order with PRMT and scaled with one more
+//    fp16x2 / bf16x2 FMA -- and store them with
 //    tcgen05.st into tensor memory, where the MMA reads its A operand.
 //  * Warp 1 (one lane) issues four tcgen05.mma (K = 16 each) per stage and
 //    frees the stage with tcgen05.commit when they have read it.
@@ -51,7 +53,7 @@ constexpr uint64_t WAIT_NS = 2000000000ull;
 
 struct GemmParams {
     uint16_t* y;
-    const uint16_t* bias;  // (N,) fp16 or null
+    const uint16_t* bias;  // (N,) fp16 / bf16 or null
     int M, K, N, G;
     int TN;              // tokens per tile (MMA N)
     int CS;              // CTAs per cluster along K
@@ -72,14 +74,15 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
 }
 
-template <int BITS>
+template <int BITS, bool BF>
 __global__ void __launch_bounds__(NWARPS * 32, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
             const __grid_constant__ CUtensorMap tm_lo, const __grid_constant__ CUtensorMap tm_s,
             const __grid_constant__ CUtensorMap tm_z, const GemmParams p) {
     using F = Fmt<BITS>;
+    using T16 = Dt<BF>;
     constexpr int EPS = F::EPS;          // codes per word of the main plane
-    constexpr int NC = F::NC;
+    constexpr int NC = ncons<BITS, BF>();
     constexpr int RW = BK / EPS;         // word rows per stage
 
     extern __shared__ uint8_t smem_raw[];
@@ -161,7 +164,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     } else if (warp == 1) {
         // ------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idesc = (1u << 4) | ((uint32_t)(p.TN >> 3) << 17) | (8u << 24);
+            // D fp32 (bit 4), A and B both fp16 (format 0) or both bf16 (format 1,
+            // bits 7 and 10), N = TN (bits 17-22, N / 8), M = 128 (bits 24-28, M / 16)
+            constexpr uint32_t ab_fmt = BF ? ((1u << 7) | (1u << 10)) : 0u;
+            const uint32_t idesc = (1u << 4) | ab_fmt | ((uint32_t)(p.TN >> 3) << 17) | (8u << 24);
             int s = 0;
             uint32_t ph = 0;
             const uint64_t bdesc0 = sw128_desc(smem_u32(base));
@@ -193,27 +199,28 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
         auto word = [&](const uint8_t* st, int rw, const uint32_t (&c)[NC], uint32_t s2, uint32_t zs2,
                         uint32_t* out) {
             const uint32_t* wt = reinterpret_cast<const uint32_t*>(st + p.off_w);
-            uint32_t w = wt[rw * BMW + nl], wh = 0, ls = 0, lw = 0;
+            uint32_t lw = 0;
             if constexpr (BITS == 3) lw = reinterpret_cast<const uint32_t*>(st + p.off_lo)[(rw >> 1) * BMW + nl];
-            prep_word<BITS>(w, wh, ls, lw, (rw & 1) ? lo_sel1 : lo_sel0);
+            Word<BITS, BF> wd;
+            wd.prep(wt[rw * BMW + nl], lw, (rw & 1) ? lo_sel1 : lo_sel0);
             uint32_t P[EPS / 2];
 #pragma unroll
-            for (int j = 0; j < EPS / 2; ++j) P[j] = pair_q<BITS>(w, wh, ls, c, j);
+            for (int j = 0; j < EPS / 2; ++j) P[j] = wd.pair(c, j);
 #pragma unroll
             for (int i = 0; i < EPS / 4; ++i) {
-                out[i] = hfma2_u32(prmt(P[2 * i], P[2 * i + 1], 0x5410u), s2, zs2);
-                out[i + EPS / 4] = hfma2_u32(prmt(P[2 * i], P[2 * i + 1], 0x7632u), s2, zs2);
+                out[i] = fma2_u32<BF>(prmt(P[2 * i], P[2 * i + 1], 0x5410u), s2, zs2);
+                out[i + EPS / 4] = fma2_u32<BF>(prmt(P[2 * i], P[2 * i + 1], 0x7632u), s2, zs2);
             }
         };
         // per-(group, column) constants from the stage's s, z rows
         auto consts = [&](const uint8_t* st, int gi, uint32_t (&c)[NC], uint32_t& s2, uint32_t& zs2) {
-            const float sv = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(st + p.off_s)[gi * BMW + nl]));
-            const float zv = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(st + p.off_z)[gi * BMW + nl]));
-            const float zi = fminf(fmaxf(rintf(zv), -256.0f), 256.0f);
+            const float sv = T16::load(reinterpret_cast<const uint16_t*>(st + p.off_s)[gi * BMW + nl]);
+            const float zv = T16::load(reinterpret_cast<const uint16_t*>(st + p.off_z)[gi * BMW + nl]);
+            const float zi = zero_int<BITS, BF>(zv);
 #pragma unroll
-            for (int ci = 0; ci < NC; ++ci) c[ci] = dup_half(-(bias_magnitude<BITS>(ci) + zi));
-            s2 = dup_half(sv);
-            zs2 = dup_half(-(zv - zi) * sv);
+            for (int ci = 0; ci < NC; ++ci) c[ci] = pair_const<BITS, BF>(ci, zi);
+            s2 = dup_t<BF>(sv);
+            zs2 = dup_t<BF>(-(zv - zi) * sv);
         };
 
         int s = 0;
@@ -224,7 +231,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
                 if (*abort_flag) break;
                 const uint8_t* st = base + (size_t)s * p.stage_bytes;
                 uint32_t c[NC], s2, zs2;
-                uint32_t a32[32];  // this thread's 64 k values (32 fp16 pairs) of the stage's A row
+                uint32_t a32[32];  // this thread's 64 k values (32 pairs) of the stage's A row
                 if (p.GPB == 1) {  // one group covers the whole k block
                     consts(st, 0, c, s2, zs2);
 #pragma unroll
@@ -318,11 +325,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
                 }
             }
             if (ncol < p.N) {
-                const float bv = p.bias ? __half2float(__ushort_as_half(p.bias[ncol])) : 0.0f;
+                const float bv = p.bias ? T16::load(p.bias[ncol]) : 0.0f;
 #pragma unroll
                 for (int cc = 0; cc < 32; ++cc) {
                     const int m = m0 + 32 * j + cc;
-                    if (m < p.M) p.y[(size_t)m * p.N + ncol] = __half_as_ushort(__float2half_rn(acc[cc] + bv));
+                    if (m < p.M) p.y[(size_t)m * p.N + ncol] = T16::store(acc[cc] + bv);
                 }
             }
         }
@@ -369,12 +376,12 @@ Tiling plan(int M, int K, int N, size_t ws_bytes) {
     return t;
 }
 
-template <int BITS>
+template <int BITS, bool BF>
 wq_status run(const Problem& pb, cudaStream_t stream) {
     constexpr int EPS = Fmt<BITS>::EPS;
     constexpr int RW = BK / EPS;
     constexpr int RL = (BITS == 3) ? BK / 32 : 0;
-    auto kern = gemm_kernel<BITS>;
+    auto kern = gemm_kernel<BITS, BF>;
 
     GemmParams p{};
     p.y = pb.y;
@@ -410,7 +417,7 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     int stages = (int)((limit - 1024 - bar_bytes) / p.stage_bytes);
     stages = std::min(stages, 6);
     stages = std::min(stages, std::max(2, p.kb_cta));
-    // tensor memory: the fp32 accumulator (TN columns), then 32 columns of fp16 A pairs per stage
+    // tensor memory: the fp32 accumulator (TN columns), then 32 columns of 16-bit A pairs per stage
     p.a_col = (uint32_t)((TN + 31) / 32 * 32);
     if (p.a_col + 32u * (uint32_t)stages > 512u) stages = (int)((512u - p.a_col) / 32u);
     p.tmem_cols = 32;
@@ -429,8 +436,8 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
 
     CUtensorMap mx, mw, ml, ms, mz;
     const int groups = (pb.K + pb.G - 1) / pb.G;
-    bool ok = make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, pb.x, pb.K, pb.M, (uint64_t)pb.K * 2, BK, TN,
-                       CU_TENSOR_MAP_SWIZZLE_128B);
+    bool ok = make_map(&mx, BF ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, pb.x, pb.K,
+                       pb.M, (uint64_t)pb.K * 2, BK, TN, CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, pb.w_q, pb.N, pb.K / EPS, (uint64_t)pb.N * 4, BMW, RW,
                         CU_TENSOR_MAP_SWIZZLE_NONE);
     if (BITS == 3)
@@ -477,17 +484,22 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     return from_cuda(cudaLaunchKernelEx(&cfg, kern, mx, mw, ml, ms, mz, p));
 }
 
+template <bool BF>
+wq_status launch_typed(const Problem& p, cudaStream_t s) {
+    switch (p.bits) {
+        case 1: return run<1, BF>(p, s);
+        case 2: return run<2, BF>(p, s);
+        case 3: return run<3, BF>(p, s);
+        case 4: return run<4, BF>(p, s);
+        case 8: return run<8, BF>(p, s);
+        default: return WQ_ERR_UNSUPPORTED;
+    }
+}
+
 }  // namespace
 
 wq_status launch_gemm(const Problem& p, cudaStream_t s) {
-    switch (p.bits) {
-        case 1: return run<1>(p, s);
-        case 2: return run<2>(p, s);
-        case 3: return run<3>(p, s);
-        case 4: return run<4>(p, s);
-        case 8: return run<8>(p, s);
-        default: return WQ_ERR_UNSUPPORTED;
-    }
+    return (p.flags & WQ_FLAG_BF16) ? launch_typed<true>(p, s) : launch_typed<false>(p, s);
 }
 
 size_t gemm_workspace_bytes(int M, int K, int N, int bits, int G) {

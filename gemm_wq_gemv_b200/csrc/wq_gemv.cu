@@ -2,7 +2,8 @@
 //
 // What is computed: dashq_kernel.py `_dashq_gemv_kernel` (one token there; up to
 // 16 here): each output column n is sum_k x[k] * (q[k][n] - z[g][n]) * s[g][n],
-// g = k / G, with fp32 accumulation and one fp16 rounding at the end.
+// g = k / G, with fp32 accumulation and one rounding at the end.  x, s, z, the
+// bias and y are all fp16 or all bf16 (the module's `out_dtype`).
 //
 // How (sm_100a):
 //  * Work split.  A CTA owns 32 output columns and a contiguous K range, split
@@ -19,9 +20,10 @@
 //    conflicts.
 //  * Dequant.  A code pair (code j, code j + eps/2) sits at the same offset in
 //    the two 16-bit halves of a word: one LOP3 ORs both into the mantissa of
-//    fp16 1024 and one exact fp16x2 FMA gives the integers q - round(z).
+//    fp16 1024 and one exact fp16x2 FMA gives the integers q - round(z) (bf16:
+//    the same with bf16 128 on shifted copies of the word; see wq_dequant.cuh).
 //  * Dot product.  Those exact values are the A operand of a warp MMA m16n8k16
-//    (fp16 in, fp32 accumulate) with x as B: A rows are 16 output columns and
+//    (fp16 or bf16 in, fp32 accumulate) with x as B: A rows are 16 output columns and
 //    the 16 k-slots are 4 word rows x 4 codes, a permutation of k; x is staged
 //    once per CTA in shared memory in the same permuted order.
 //  * Per group, acc += s * (D - (z - round(z)) * X) in fp32, X = the sum of the
@@ -29,7 +31,7 @@
 //    q == z gives exactly 0.
 //  * s and z of the CTA's groups arrive with one TMA copy each and become
 //    per-(group, column) records in shared memory; the optional bias is added
-//    to the fp32 sum before the fp16 rounding.
+//    to the fp32 sum before the final rounding.
 #include <algorithm>
 #include <array>
 #include <map>
@@ -59,7 +61,7 @@ struct Params {
     const uint32_t* w_lo;
     const uint16_t* s;
     const uint16_t* z;
-    const uint16_t* bias;  // (N,) fp16 or null
+    const uint16_t* bias;  // (N,) fp16 / bf16 or null
     uint16_t* y;
     int M, K, N, G;
     int Kw;        // word rows of the main plane
@@ -100,13 +102,15 @@ __device__ __forceinline__ float sum_warps(const float* red, int wk, int stride,
     return v[0];
 }
 
-template <int BITS, int NT>
+template <int BITS, int NT, bool BF>
 __global__ void __launch_bounds__(MAXW * 32, (NT == 1 && BITS != 1) ? 2 : 1)
 gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_lo,
             const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_z, const Params p) {
     using F = Fmt<BITS>;
+    using T16 = Dt<BF>;
+    using R = Rec<BITS, BF>;
     constexpr int EPS = F::EPS;
-    constexpr int NC = F::NC;
+    constexpr int NC = ncons<BITS, BF>();
     constexpr int QK = 4 * EPS;  // k values per quad
     constexpr int MMAS = EPS / 4;
     constexpr int SB = stage_bytes<BITS>();
@@ -134,7 +138,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     auto gdiv = [&](int q) { return p.qpg_shift >= 0 ? (q >> p.qpg_shift) : q / p.qpg; };
     const int g_cta0 = gdiv(min(cta_q0, p.Q - 1));
     const int nrec = p.groups_cta * COLS;
-    Rec<BITS>* tab = reinterpret_cast<Rec<BITS>*>(smem + p.off_tab);
+    R* tab = reinterpret_cast<R*>(smem + p.off_tab);
     bool any_frac = false;
     // Record slot sl of a group holds column 4 (sl % 8) + sl / 8: the eight lanes
     // reading one column offset c of their chunks then read consecutive records.
@@ -146,15 +150,15 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
         for (int i = threadIdx.x; i < nrec; i += blockDim.x) {
             const int sl = i & (COLS - 1);
             const int o = (i & ~(COLS - 1)) + 4 * (sl & 7) + (sl >> 3);
-            const float sv = __half2float(__ushort_as_half(s_raw[o]));
-            const float zv = __half2float(__ushort_as_half(z_raw[o]));
-            const float zi = fminf(fmaxf(rintf(zv), -256.0f), 256.0f);
-            Rec<BITS> rec;
+            const float sv = T16::load(s_raw[o]);
+            const float zv = T16::load(z_raw[o]);
+            const float zi = zero_int<BITS, BF>(zv);
+            R rec;
             rec.s = sv;
             rec.zr = zv - zi;
             any_frac |= (rec.zr != 0.0f);
 #pragma unroll
-            for (int ci = 0; ci < NC; ++ci) rec.c[ci] = dup_half(-(bias_magnitude<BITS>(ci) + zi));
+            for (int ci = 0; ci < NC; ++ci) rec.c[ci] = pair_const<BITS, BF>(ci, zi);
             tab[i] = rec;
         }
     };
@@ -300,7 +304,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
                 const uint32_t e[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
-                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&e[h]));
+                    const float2 f = T16::pair(e[h]);
                     a0 += f.x;
                     a1 += f.y;
                 }
@@ -324,7 +328,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     // The main loop, specialised on whether fractional zero-point terms are needed.
     auto main_loop = [&](auto frac_tag) {
         constexpr bool FRAC = decltype(frac_tag)::value;
-        constexpr uint32_t RS = sizeof(Rec<BITS>);
+        constexpr uint32_t RS = sizeof(R);
         float dsum[2][NT][4];
         float xs_sum[NT][2];
 #pragma unroll
@@ -424,18 +428,18 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
                         cB[ci] = lds32_u32(rc + cb * CS8 + 8 + 4 * ci);
                     }
                 }
-                uint32_t wA = wv[ca], wB = wv[cb], wAh = 0, wBh = 0, lA = 0, lB = 0;
-                prep_word<BITS>(wA, wAh, lA, lw[ca], lo_sel);
-                prep_word<BITS>(wB, wBh, lB, lw[cb], lo_sel);
+                Word<BITS, BF> WA, WB;
+                WA.prep(wv[ca], lw[ca], lo_sel);
+                WB.prep(wv[cb], lw[cb], lo_sel);
 #pragma unroll
                 for (int h = 0; h < MMAS; ++h) {
                     uint32_t a[4];
-                    a[0] = pair_q<BITS>(wA, wAh, lA, cA, 2 * h);
-                    a[1] = pair_q<BITS>(wB, wBh, lB, cB, 2 * h);
-                    a[2] = pair_q<BITS>(wA, wAh, lA, cA, 2 * h + 1);
-                    a[3] = pair_q<BITS>(wB, wBh, lB, cB, 2 * h + 1);
+                    a[0] = WA.pair(cA, 2 * h);
+                    a[1] = WB.pair(cB, 2 * h);
+                    a[2] = WA.pair(cA, 2 * h + 1);
+                    a[3] = WB.pair(cB, 2 * h + 1);
 #pragma unroll
-                    for (int n = 0; n < NT; ++n) mma_16816(dsum[T][n], a, bx[n][2 * h], bx[n][2 * h + 1]);
+                    for (int n = 0; n < NT; ++n) mma_16816<BF>(dsum[T][n], a, bx[n][2 * h], bx[n][2 * h + 1]);
                 }
             }
 
@@ -535,8 +539,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
             for (int r = 0; r < p.CS; ++r) sacc += ld_shared_cluster_f32(map_shared_rank(part_addr + 4u * i, r));
             const int m = i / COLS, col = col0 + i % COLS;
             if (col < p.N) {
-                const float b = p.bias ? __half2float(__ushort_as_half(p.bias[col])) : 0.0f;
-                p.y[(size_t)m * p.N + col] = __half_as_ushort(__float2half_rn(sacc + b));
+                const float b = p.bias ? T16::load(p.bias[col]) : 0.0f;
+                p.y[(size_t)m * p.N + col] = T16::store(sacc + b);
             }
         }
         cluster_sync();  // peers keep their shared memory until every read is done
@@ -546,8 +550,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
             const float sacc = sum_warps(red, p.WK, p.M * COLS, i);
             const int m = i / COLS, col = col0 + i % COLS;
             if (col < p.N) {
-                const float b = p.bias ? __half2float(__ushort_as_half(p.bias[col])) : 0.0f;
-                p.y[(size_t)m * p.N + col] = __half_as_ushort(__float2half_rn(sacc + b));
+                const float b = p.bias ? T16::load(p.bias[col]) : 0.0f;
+                p.y[(size_t)m * p.N + col] = T16::store(sacc + b);
             }
         }
     }
@@ -560,12 +564,12 @@ int ilog2(int v) {
     return r;
 }
 
-template <int BITS, int NT>
+template <int BITS, int NT, bool BF>
 wq_status run(const Problem& pb, cudaStream_t stream) {
     using F = Fmt<BITS>;
     constexpr int EPS = F::EPS;
     constexpr int QK = 4 * EPS;
-    auto kern = gemv_kernel<BITS, NT>;
+    auto kern = gemv_kernel<BITS, NT, BF>;
     static unsigned long long attr_done = 0;  // one bit per device
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return WQ_ERR_CUDA;
@@ -588,6 +592,7 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
 
     // The plan depends on the shape and flags only: computed once per device and
     // kept (its occupancy queries would otherwise cost more than the launch).
+    // One map per instantiation (bit width, tokens per MMA, element type).
     struct Plan {
         Params q;
         size_t smem;
@@ -636,7 +641,7 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
             off += (size_t)pb.M * quads_cta * 4;
             off = (off + 15) & ~(size_t)15;
             q.off_tab = (uint32_t)off;
-            off += (size_t)q.groups_cta * COLS * sizeof(Rec<BITS>);
+            off += (size_t)q.groups_cta * COLS * sizeof(Rec<BITS, BF>);
             q.off_red = (uint32_t)off;
             off += (size_t)WK * pb.M * COLS * 4;
             q.off_part = (uint32_t)off;
@@ -752,16 +757,25 @@ wq_status gemv_device_status(int reset) {
     return v ? WQ_ERR_TIMEOUT : WQ_OK;
 }
 
-wq_status launch_gemv(const Problem& p, cudaStream_t s) {
+namespace {
+
+template <bool BF>
+wq_status launch_typed(const Problem& p, cudaStream_t s) {
     const bool two = p.M > 8;
     switch (p.bits) {
-        case 1: return two ? run<1, 2>(p, s) : run<1, 1>(p, s);
-        case 2: return two ? run<2, 2>(p, s) : run<2, 1>(p, s);
-        case 3: return two ? run<3, 2>(p, s) : run<3, 1>(p, s);
-        case 4: return two ? run<4, 2>(p, s) : run<4, 1>(p, s);
-        case 8: return two ? run<8, 2>(p, s) : run<8, 1>(p, s);
+        case 1: return two ? run<1, 2, BF>(p, s) : run<1, 1, BF>(p, s);
+        case 2: return two ? run<2, 2, BF>(p, s) : run<2, 1, BF>(p, s);
+        case 3: return two ? run<3, 2, BF>(p, s) : run<3, 1, BF>(p, s);
+        case 4: return two ? run<4, 2, BF>(p, s) : run<4, 1, BF>(p, s);
+        case 8: return two ? run<8, 2, BF>(p, s) : run<8, 1, BF>(p, s);
         default: return WQ_ERR_UNSUPPORTED;
     }
+}
+
+}  // namespace
+
+wq_status launch_gemv(const Problem& p, cudaStream_t s) {
+    return (p.flags & WQ_FLAG_BF16) ? launch_typed<true>(p, s) : launch_typed<false>(p, s);
 }
 
 }  // namespace wq

@@ -16,7 +16,7 @@ struct Problem {
     const uint32_t* w_lo;
     const uint16_t* scales;
     const uint16_t* zeros;
-    const uint16_t* bias;  // (N,) fp16 or null
+    const uint16_t* bias;  // (N,) fp16 or bf16 (WQ_FLAG_BF16), or null
     uint16_t* y;
     int M, K, N, bits, G;  // G resolved: group_size == -1 -> K
     unsigned flags;

@@ -50,7 +50,7 @@
 extern "C" {
 #endif
 
-#define WQ_ABI_VERSION 2
+#define WQ_ABI_VERSION 3
 
 typedef enum {
     WQ_OK = 0,
@@ -82,6 +82,20 @@ typedef enum {
  *   activation, expert weights of one token) use it to overlap completely.
  */
 #define WQ_FLAG_PDL_INPUTS_READY 2u
+/*
+ * WQ_FLAG_BF16: x, scales, zeros, bias and y hold bfloat16 instead of
+ *   binary16 (dashq_kernel.py `TritonQuantLinear`: scale, zero and bias are
+ *   stored in its `out_dtype`, and the product is computed in the dtype of x).
+ *   The accumulation stays fp32 and y is rounded once to bfloat16 (nearest
+ *   even).  wq_gemm dequantises each weight to bfloat16 for the tensor cores
+ *   with one bf16 FMA, (q - zi) * s + bf16(-(z - zi) * s), zi = round(z)
+ *   clamped to [0, 2^bits - 1] (the module's batched branch dequantises in
+ *   the dtype of x); wq_gemv keeps q - zi exact and applies s and z - zi in
+ *   fp32.  With either type the layouts, shapes and other rules are the same.
+ */
+#define WQ_FLAG_BF16 4u
+/* Every flag bit the products accept; any other bit gives WQ_ERR_INVALID_ARG. */
+#define WQ_FLAG_ALL (WQ_FLAG_PDL | WQ_FLAG_PDL_INPUTS_READY | WQ_FLAG_BF16)
 
 /* Version of this ABI (WQ_ABI_VERSION). */
 int wq_abi_version(void);
@@ -115,15 +129,16 @@ wq_status wq_unpack_kmajor(const uint32_t* w_q, const uint32_t* w_lo, int K, int
 /*
  * Decode-time product for a few rows of x: 1 <= M <= 16
  * (dashq_kernel.py `_dashq_gemv_kernel` and `forward` for one token; here any
- * M up to 16 reads W_q once).  x (M, K), y (M, N), binary16.
+ * M up to 16 reads W_q once).  x (M, K), y (M, N), binary16 (bfloat16 with
+ * WQ_FLAG_BF16, which then also applies to scales, zeros and bias).
  * group_size: -1, or a positive divisor of K that is a multiple of 4 * eps
  * (1-bit: 128, 2-bit: 64, 3-bit: 64, 4-bit: 32, 8-bit: 16); other group sizes
  * give WQ_ERR_UNSUPPORTED here (wq_gemm takes them).  Requires K % eps == 0
  * (3-bit: K % 32 == 0) and N % 8 == 0.
  * One launch: the split-K partial sums are reduced on chip (thread-block
  * cluster shared memory); no workspace and no zero-initialised output needed.
- *   bias  optional (N,) binary16 device array, 2-byte aligned, or NULL: then
- *         y[m][n] = RN_fp16(sum_k x[m][k] w[k][n] + bias[n]), the sum in fp32
+ *   bias  optional (N,) device array of the same type as x, 2-byte aligned,
+ *         or NULL: then y[m][n] = RN(sum_k x[m][k] w[k][n] + bias[n]), the sum in fp32
  *         (dashq_kernel.py `TritonQuantLinear.forward` adds its bias to the
  *         product's output).
  */
@@ -138,8 +153,9 @@ wq_status wq_gemv(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
  * branch).  Same arguments as wq_gemv (bias included), plus a workspace.  group_size: -1, or a
  * positive divisor of K that is a multiple of eps (3-bit: of 32) and either a
  * multiple or a divisor of 64.  Requires K % 64 == 0 and N % 8 == 0.
- * Packed tiles are dequantised to fp16 into tensor memory and multiplied on the
- * tensor cores (tcgen05, fp32 accumulators in tensor memory).
+ * Packed tiles are dequantised to fp16 (bf16 with WQ_FLAG_BF16) into tensor
+ * memory and multiplied on the tensor cores (tcgen05, fp32 accumulators in
+ * tensor memory).
  *   workspace        device scratch for splitting K over the CTAs of a cluster
  *                    (fp32 partial tiles, reduced through L2), owned by the
  *                    caller; it needs no initialisation and keeps no state

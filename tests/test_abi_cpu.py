@@ -30,7 +30,7 @@ def test_every_declared_symbol_is_exported(libwq):
 
 def test_version_and_strings(libwq):
     L = libwq.lib()
-    assert L.wq_abi_version() == 2
+    assert L.wq_abi_version() == 3
     for s in range(7):
         assert L.wq_status_string(s)
     assert L.wq_status_string(99) == b"unknown status"
@@ -67,12 +67,25 @@ def test_product_argument_checks(libwq, fn):
     assert gemv(L, fn, N=252) == ALI                      # N % 8
     assert gemv(L, fn, x=P + 8) == ALI
     assert gemv(L, fn, wq=P + 4) == ALI
-    assert gemv(L, fn, bias=P + 1) == ALI                 # bias: 2-byte aligned fp16
+    assert gemv(L, fn, bias=P + 1) == ALI                 # bias: 2-byte aligned fp16 / bf16
+    assert gemv(L, fn, flags=8) == INV                    # unknown flag bit
+    assert gemv(L, fn, flags=0x80000000 | 4) == INV
     # valid arguments: the host checks pass and the call reaches CUDA, which has no device here
     import torch
     if not torch.cuda.is_available():
         assert gemv(L, fn) == CUDA
         assert gemv(L, fn, bits=3, wlo=P, K=512, G=128) == CUDA
+        assert gemv(L, fn, flags=4) == CUDA               # WQ_FLAG_BF16
+        assert gemv(L, fn, flags=1 | 4) == CUDA
+        assert gemv(L, fn, flags=2 | 4) == CUDA
+
+
+def test_flag_values_match_the_header(libwq):
+    text = (ROOT / "include" / "wq.h").read_text()
+    vals = dict(re.findall(r"#define (WQ_FLAG_\w+) (\d+)u", text))
+    assert vals == {"WQ_FLAG_PDL": str(libwq.WQ_FLAG_PDL),
+                    "WQ_FLAG_PDL_INPUTS_READY": str(libwq.WQ_FLAG_PDL_INPUTS_READY),
+                    "WQ_FLAG_BF16": str(libwq.WQ_FLAG_BF16)}
 
 
 def test_gemv_specific_limits(libwq):

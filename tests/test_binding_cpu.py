@@ -15,6 +15,24 @@ def test_cpu_tensors_are_refused(libwq):
             fn(x, w, None, s, s, 4, 64)
 
 
+def test_cpu_tensors_are_refused_in_bf16_too(libwq):
+    x = torch.zeros((1, 64), dtype=torch.bfloat16)
+    w = torch.zeros((8, 8), dtype=torch.int32)
+    s = torch.zeros((1, 8), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        libwq.gemv(x, w, None, s, s, 4, 64)
+
+
+def test_element_types(libwq):
+    """x must be float16 or bfloat16; scales, zeros and bias must match it."""
+    w = torch.zeros((8, 8), dtype=torch.int32)
+    x32 = torch.zeros((1, 64), dtype=torch.float32)
+    with pytest.raises(TypeError, match="float16 or torch.bfloat16"):
+        libwq.gemv(x32, w, None, x32, x32, 4, 64)
+    assert libwq._elem_type(torch.zeros(1, dtype=torch.bfloat16)) is torch.bfloat16
+    assert libwq._elem_type(torch.zeros(1, dtype=torch.float16)) is torch.float16
+
+
 def test_non_tensor_is_refused(libwq):
     with pytest.raises(TypeError, match="torch.Tensor"):
         libwq.gemv([[0.0]], None, None, None, None, 4, 64)
