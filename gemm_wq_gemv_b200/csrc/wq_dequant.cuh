@@ -34,11 +34,24 @@ template <> struct Fmt<8> { static constexpr int EPS = 4, NC = 1, NCB = 1; };
 template <int BITS, bool BF>
 constexpr int ncons() { return BF ? Fmt<BITS>::NCB : Fmt<BITS>::NC; }
 
-// Per (group, column) record in shared memory: fp32 scale, fp32 fractional zero
-// part, and the bias constants (duplicated fp16 / bf16 pairs; 8-bit bf16: one fp32).
-template <int BITS, bool BF> struct alignas(16) Rec {
+// Per (group, column) record in shared memory: the bias constants (duplicated
+// fp16 / bf16 pairs; 8-bit bf16: one fp32), preceded by the fp32 scale and
+// fractional zero part.  8-bit keeps "slim" records, the constant alone: the
+// GEMV reads s and z from the raw s/z rows when a group ends, so the table is
+// a quarter of the size.  On B200 that takes the 8192 x 8192 8-bit group-128
+// decode plan from two CTAs per SM to three (25 us -> 14 us); the same for
+// 4-bit would take the 4096 x 4096 decode plan from three to four CTAs per SM,
+// which measured 4 % slower, so 4-bit keeps full records.
+template <int BITS, bool BF>
+constexpr bool slim_rec() { return BITS == 8; }
+
+template <int BITS, bool BF, bool SLIM = slim_rec<BITS, BF>()> struct Rec;
+template <int BITS, bool BF> struct alignas(16) Rec<BITS, BF, false> {
     float s;
     float zr;
+    uint32_t c[ncons<BITS, BF>()];
+};
+template <int BITS, bool BF> struct Rec<BITS, BF, true> {
     uint32_t c[ncons<BITS, BF>()];
 };
 

@@ -109,6 +109,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     using F = Fmt<BITS>;
     using T16 = Dt<BF>;
     using R = Rec<BITS, BF>;
+    constexpr bool SLIM = slim_rec<BITS, BF>();
+    constexpr uint32_t COFF = SLIM ? 0u : 8u;  // byte offset of the constants in a record
     constexpr int EPS = F::EPS;
     constexpr int NC = ncons<BITS, BF>();
     constexpr int QK = 4 * EPS;  // k values per quad
@@ -154,9 +156,11 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
             const float zv = T16::load(z_raw[o]);
             const float zi = zero_int<BITS, BF>(zv);
             R rec;
-            rec.s = sv;
-            rec.zr = zv - zi;
-            any_frac |= (rec.zr != 0.0f);
+            if constexpr (!SLIM) {
+                rec.s = sv;
+                rec.zr = zv - zi;
+            }
+            any_frac |= (zv - zi != 0.0f);
 #pragma unroll
             for (int ci = 0; ci < NC; ++ci) rec.c[ci] = pair_const<BITS, BF>(ci, zi);
             tab[i] = rec;
@@ -360,6 +364,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
         int left = p.qpg - (q_begin - g_first * p.qpg);  // quads left in the current group
         uint32_t rc = smem_u32(tab) + RS * (uint32_t)((g_first - g_cta0) * COLS + cg);
         constexpr uint32_t CS8 = 8 * RS;  // record stride between the lane's columns
+        // slim records: the raw s row of the lane's 4 columns (z at + sz_stride)
+        [[maybe_unused]] uint32_t sz_row = smem_u32(s_raw) + 2u * (uint32_t)((g_first - g_cta0) * COLS + 4 * cg);
         // bias constants of the lane's 4 columns, in registers for narrow records
         constexpr bool CREG = NC <= 2;
         [[maybe_unused]] uint32_t creg[4][CREG ? NC : 1];
@@ -368,7 +374,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
 #pragma unroll
-                    for (int ci = 0; ci < NC; ++ci) creg[c][ci] = lds32_u32(rc + c * CS8 + 8 + 4 * ci);
+                    for (int ci = 0; ci < NC; ++ci) creg[c][ci] = lds32_u32(rc + c * CS8 + COFF + 4 * ci);
             }
         };
         if (nq > 0) load_creg();
@@ -424,8 +430,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
                         cA[ci] = creg[ca][ci];
                         cB[ci] = creg[cb][ci];
                     } else {
-                        cA[ci] = lds32_u32(rc + ca * CS8 + 8 + 4 * ci);
-                        cB[ci] = lds32_u32(rc + cb * CS8 + 8 + 4 * ci);
+                        cA[ci] = lds32_u32(rc + ca * CS8 + COFF + 4 * ci);
+                        cB[ci] = lds32_u32(rc + cb * CS8 + COFF + 4 * ci);
                     }
                 }
                 Word<BITS, BF> WA, WB;
@@ -445,10 +451,29 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
 
             // end of a group (or of this warp's range): scale and fold into acc
             if (--left == 0 || i == nq - 1) {
+                [[maybe_unused]] float s4[4], zr4[4];
+                if constexpr (SLIM) {  // columns 4 cg .. 4 cg + 3 of the raw rows: one 8-byte read each
+                    const uint2 su = lds64_u32(sz_row);
+                    const float2 s01 = T16::pair(su.x), s23 = T16::pair(su.y);
+                    s4[0] = s01.x; s4[1] = s01.y; s4[2] = s23.x; s4[3] = s23.y;
+                    if constexpr (FRAC) {
+                        const uint2 zu = lds64_u32(sz_row + p.sz_stride);
+                        const float2 z01 = T16::pair(zu.x), z23 = T16::pair(zu.y);
+                        const float zv[4] = {z01.x, z01.y, z23.x, z23.y};
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) zr4[c] = zv[c] - zero_int<BITS, BF>(zv[c]);
+                    }
+                }
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const float sc = __uint_as_float(lds32_u32(rc + c * CS8));
-                    const float zr = FRAC ? __uint_as_float(lds32_u32(rc + c * CS8 + 4)) : 0.0f;
+                    float sc, zr = 0.0f;
+                    if constexpr (SLIM) {
+                        sc = s4[c];
+                        if constexpr (FRAC) zr = zr4[c];
+                    } else {
+                        sc = __uint_as_float(lds32_u32(rc + c * CS8));
+                        if constexpr (FRAC) zr = __uint_as_float(lds32_u32(rc + c * CS8 + 4));
+                    }
                     const int T = c >> 1, half = c & 1;
 #pragma unroll
                     for (int n = 0; n < NT; ++n)
@@ -472,6 +497,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
                 if (left == 0) {
                     left = p.qpg;
                     rc += COLS * RS;
+                    sz_row += 2 * COLS;
                     if (i + 1 < nq) load_creg();
                 }
             }
