@@ -20,6 +20,10 @@ Floating-point inputs (x, scales, zeros, bias) are all fp16 or all bf16
 NumPy ``float16``, bf16 arrays as ``uint16`` bit patterns (NumPy has no
 bfloat16).
 
+``mse_observer`` (NumPy) is the oracle of the MSE-observer search of
+per-group scales and zero points (the "Benchmark for MSE observer grid
+search" page), pinned by ``tests/test_mse_oracle.py``.
+
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
 (hand-derived golden words and products, closed forms, brute force, library
 special cases); none is "parity unpinned".
