@@ -16,6 +16,7 @@ Entry points (same names as the C ABI, without the ``wq_`` prefix):
 * ``gemm_workspace_size(M, K, N, bits, group_size) -> bytes``
 * ``matmul(...)``: same arguments as ``gemm``; ``wq_gemv`` or ``wq_gemm`` by M
 * ``gemm_noalloc(x, w_q, w_lo, scales, zeros, bits, group_size, out) -> out``
+* ``selftest_wait_timeout(limit_ns) -> status`` (the bounded-wait failure path)
 
 x, scales, zeros, bias and the output are all ``torch.float16`` or all
 ``torch.bfloat16`` (the type of x decides; bfloat16 sets ``WQ_FLAG_BF16``).
@@ -81,7 +82,9 @@ def lib() -> ctypes.CDLL:
         L.wq_matmul_workspace_size.restype = ctypes.c_size_t
         L.wq_gemm_noalloc.restype = i
         L.wq_device_status.argtypes = [i]
-        for f in ("wq_pack_kmajor", "wq_unpack_kmajor", "wq_gemv", "wq_gemm", "wq_device_status"):
+        L.wq_selftest_wait_timeout.argtypes = [ctypes.c_uint64, p]
+        for f in ("wq_pack_kmajor", "wq_unpack_kmajor", "wq_gemv", "wq_gemm", "wq_device_status",
+                  "wq_selftest_wait_timeout"):
             getattr(L, f).restype = i
         _lib = L
     return _lib
@@ -286,6 +289,13 @@ def gemm_noalloc(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out, p
     _need(out, _elem_type(x), "out")
     return _product("wq_gemm_noalloc", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl,
                     bias=bias)
+
+
+def selftest_wait_timeout(limit_ns: int = 1_000_000) -> int:
+    """``wq_selftest_wait_timeout``: run the bounded-wait failure path on purpose
+    (a wait on a barrier nothing completes) on the current stream; returns the
+    status, 5 (WQ_ERR_TIMEOUT) when the wait gave up as it should."""
+    return int(lib().wq_selftest_wait_timeout(int(limit_ns), _stream()))
 
 
 def matmul(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl: bool = False,

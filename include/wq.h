@@ -229,6 +229,21 @@ wq_status wq_gemm_noalloc(const uint16_t* x, const uint32_t* w_q, const uint32_t
  */
 wq_status wq_device_status(int reset);
 
+/*
+ * Failure-detection self-test (the pages have no counterpart).  Every mbarrier
+ * wait in the products is bounded: on time-out the kernel records it in a
+ * device status word (read with wq_device_status as WQ_ERR_TIMEOUT), skips its
+ * remaining work and exits, so the context stays usable.  This call runs that
+ * path on purpose, without any fault: one CTA waits, with the products' bounded
+ * wait, on an mbarrier that nothing completes, gives up after limit_ns and
+ * records the time-out in a status word of its own.  It synchronises `stream`.
+ *   limit_ns  1e3 .. 1e9 (else WQ_ERR_INVALID_ARG, nothing launched)
+ * Returns WQ_ERR_TIMEOUT when the wait ran out (the expected result), WQ_OK if
+ * it did not, WQ_ERR_CUDA if the launch or the copies failed.  The products'
+ * status words are not touched.
+ */
+wq_status wq_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -148,3 +148,14 @@ def test_matmul_route(libwq):
         int(L.wq_gemm_workspace_size(512, 4096, 2048, 4, 128))
     # argument checks pass through: M = 0 is rejected before anything runs
     assert L.wq_matmul(P, P, None, P, P, None, P, 0, 512, 256, 4, 128, 0, None, ctypes.c_size_t(0), None) == 1
+
+
+def test_selftest_argument_checks(libwq):
+    """The failure-path self-test rejects limits outside 1 us .. 1 s before any launch."""
+    L = libwq.lib()
+    assert L.wq_selftest_wait_timeout(0, None) == 1
+    assert L.wq_selftest_wait_timeout(999, None) == 1
+    assert L.wq_selftest_wait_timeout(2_000_000_000, None) == 1
+    import torch
+    if not torch.cuda.is_available():
+        assert L.wq_selftest_wait_timeout(1_000_000, None) == 6   # reaches CUDA: no device here
