@@ -101,9 +101,11 @@ def group_error(w, w_hat, norm: float) -> np.ndarray:
 
 def search(w, bits: int, group_size: int, maxshrink: float = 0.2, grid: int = 100,
            norm: float = 2.4, patience: int | None = None) -> dict:
-    # defaults: the page's benchmark CLI (maxshrink 0.20, grid 100, norm 2.4; its
-    # patience default is 5, passed explicitly since None means every candidate)
     """The grid search for every group of W (rows x cols, fp32; cols % group_size == 0).
+
+    Defaults are the page's benchmark CLI (maxshrink 0.20, grid 100, norm 2.4);
+    its patience default, 5, is passed explicitly, since None means every
+    candidate is evaluated.
 
     Returns a dict of arrays of shape (rows, cols // group_size):
     ``step`` (best candidate index), ``err`` (its error), ``scale``, ``zero``
