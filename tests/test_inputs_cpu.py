@@ -1,0 +1,38 @@
+"""The seeded input generator: what DESIGN states about the draws holds."""
+import numpy as np
+import torch
+
+import wq_inputs
+
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(0)
+    v = np.concatenate([rng.standard_normal(10000) * 10.0 ** rng.integers(-20, 20, 10000),
+                        [0.0, -0.0, 1.0, 1.00390625, 1.01171875, -3.0, 65504.0, 1e30]])
+    ours = wq_inputs.bf16_bits(v)
+    ref = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_same_stream_for_both_types():
+    wl = wq_inputs.WORKLOADS["tiny_gemv"]
+    a = wq_inputs.draw(wl, seed=4)
+    b = wq_inputs.draw(wl, seed=4, dtype="bf16")
+    assert np.array_equal(a.codes, b.codes)
+    # the same draws, rounded to each type: zeros are integers (exact in both)
+    zb = (b.zeros.astype(np.uint32) << 16).view(np.float32)
+    assert np.array_equal(a.zeros.astype(np.float32), zb)
+    xb = (b.x.astype(np.uint32) << 16).view(np.float32)
+    assert np.all(np.abs(xb - a.x.astype(np.float32)) <= 2.0 ** -8 * np.abs(xb) + 2.0 ** -24)
+
+
+def test_deterministic_and_in_range():
+    for name, wl in wq_inputs.WORKLOADS.items():
+        if wl.K * wl.N > 1 << 24:
+            continue
+        a = wq_inputs.draw(wl, seed=0)
+        b = wq_inputs.draw(wl, seed=0)
+        assert np.array_equal(a.codes, b.codes) and np.array_equal(a.x, b.x), name
+        assert a.codes.max() <= (1 << wl.bits) - 1, name
+        assert a.scales.min() >= np.float16(wl.s_lo) and a.scales.max() <= np.float16(wl.s_hi), name
+        assert a.scales.shape == (wl.groups, wl.N) and a.x.shape == (wl.M, wl.K), name
