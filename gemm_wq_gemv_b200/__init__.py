@@ -140,6 +140,58 @@ def words_shape(K: int, N: int, bits: int):
     return (K // (32 // bits), N), None
 
 
+_BITS = (1, 2, 3, 4, 8)
+
+
+def _same_device(ref, **tensors):
+    for name, t in tensors.items():
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"{name} is on {t.device}, x on {ref.device}: all tensors must share one device")
+
+
+def _check_planes(w_q, w_lo, K: int, bits: int):
+    """w_q (and w_lo) must have the packed shape of a (K, N) code matrix, N = w_q.shape[1].
+
+    The library sizes its copies from K, N and bits, so a plane of another shape
+    would be read out of its bounds; a bit width it does not take is left to the
+    C call, which rejects it."""
+    if bits not in _BITS:
+        return
+    N = w_q.shape[1]
+    hs, ls = words_shape(K, N, bits)
+    if tuple(w_q.shape) != hs:
+        raise ValueError(f"w_q has shape {tuple(w_q.shape)}; K={K}, {bits}-bit words need {hs}")
+    if ls is None and w_lo is not None:
+        raise ValueError(f"w_lo must be None for {bits}-bit words")
+    if ls is not None:
+        if w_lo is None:
+            raise ValueError("3-bit words need the lo plane w_lo")
+        if tuple(w_lo.shape) != ls:
+            raise ValueError(f"w_lo has shape {tuple(w_lo.shape)}; K={K} 3-bit needs {ls}")
+
+
+def _check_product(x, w_q, w_lo, scales, zeros, bias, out, bits: int, group_size: int):
+    """Every tensor of a product has the shape its K, N, M, bits and group size
+    imply, and sits on x's device.  Raises ValueError before any C call.
+    Shapes the C rules reject anyway (a K that is not a multiple of the word
+    width, a group size that does not divide K) are left to the C call, which
+    names the rule."""
+    M, K = x.shape
+    N = w_q.shape[1]
+    _same_device(x, w_q=w_q, w_lo=w_lo, scales=scales, zeros=zeros, bias=bias, out=out)
+    _check_planes(w_q, w_lo, K, bits)
+    G = K if group_size == -1 else group_size
+    if G > 0 and K % G == 0:
+        for name, t in (("scales", scales), ("zeros", zeros)):
+            if tuple(t.shape) != (K // G, N):
+                raise ValueError(f"{name} has shape {tuple(t.shape)}; K={K}, group size {group_size} "
+                                 f"and N={N} need {(K // G, N)}")
+    if bias is not None and tuple(bias.shape) != (N,):
+        raise ValueError(f"bias has shape {tuple(bias.shape)}; N={N} needs ({N},)")
+    if out is not None and tuple(out.shape) != (M, N):
+        raise ValueError(f"out has shape {tuple(out.shape)}; M={M}, N={N} need {(M, N)}")
+
+
 def pack_kmajor(codes_kn, bits: int, check_range: bool = True):
     """(K, N) uint8 codes -> (w_q, w_lo) int32 words (w_lo is None unless bits == 3).
 
@@ -166,6 +218,8 @@ def unpack_kmajor(w_q, w_lo, K: int, bits: int):
     _need(w_q, torch.int32, "w_q")
     if w_lo is not None:
         _need(w_lo, torch.int32, "w_lo")
+    _same_device(w_q, w_lo=w_lo)
+    _check_planes(w_q, w_lo, K, bits)
     N = w_q.shape[1]
     out = torch.empty((K, N), dtype=torch.uint8, device=w_q.device)
     _check("wq_unpack_kmajor", lib().wq_unpack_kmajor(_ptr(w_q), _ptr(w_lo), K, N, bits,
@@ -196,12 +250,13 @@ def _product(fn, x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, worksp
     _need(zeros, dt, "zeros")
     if bias is not None:
         _need(bias, dt, "bias", ndim=1)
+    if out is not None:
+        _need(out, dt, "out")
+    _check_product(x, w_q, w_lo, scales, zeros, bias, out, bits, group_size)
     M, K = x.shape
     N = w_q.shape[1]
     if out is None:
         out = torch.empty((M, N), dtype=dt, device=x.device)
-    else:
-        _need(out, dt, "out")
     flags = ((WQ_FLAG_PDL if pdl else 0) | (WQ_FLAG_PDL_INPUTS_READY if inputs_ready else 0)
              | (WQ_FLAG_BF16 if dt is torch.bfloat16 else 0))
     args = [_ptr(x), _ptr(w_q), _ptr(w_lo), _ptr(scales), _ptr(zeros), _ptr(bias), _ptr(out),
@@ -272,6 +327,7 @@ def gemm(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl:
     if workspace is not None:
         torch = _torch()
         _need(workspace, torch.uint8, "workspace", ndim=1)
+        _same_device(x, workspace=workspace)
     return _product("wq_gemm", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, workspace,
                     inputs_ready=inputs_ready, bias=bias)
 
@@ -305,6 +361,7 @@ def matmul(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pd
     if workspace is not None:
         torch = _torch()
         _need(workspace, torch.uint8, "workspace", ndim=1)
+        _same_device(x, workspace=workspace)
     return _product("wq_matmul", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl, workspace,
                     inputs_ready=inputs_ready, bias=bias)
 

@@ -451,14 +451,10 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
                         CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return WQ_ERR_CUDA;
 
-    static unsigned long long attr_done = 0;
+    static std::atomic<uint64_t> attr_ctx[MAX_DEVICES];  // context the smem limit was raised in
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return WQ_ERR_CUDA;
-    if (dev < 64 && !(attr_done & (1ull << dev))) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)limit) != cudaSuccess)
-            return WQ_ERR_CUDA;
-        attr_done |= 1ull << dev;
-    }
+    if (const wq_status st = ensure_smem_attr((const void*)kern, (int)limit, attr_ctx, dev); st != WQ_OK) return st;
 
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(ntiles, mt, CS);

@@ -596,14 +596,10 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     constexpr int EPS = F::EPS;
     constexpr int QK = 4 * EPS;
     auto kern = gemv_kernel<BITS, NT, BF>;
-    static unsigned long long attr_done = 0;  // one bit per device
+    static std::atomic<uint64_t> attr_ctx[MAX_DEVICES];  // context the smem limit was raised in
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return WQ_ERR_CUDA;
-    if (dev < 64 && !(attr_done & (1ull << dev))) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
-            return WQ_ERR_CUDA;
-        attr_done |= 1ull << dev;
-    }
+    if (const wq_status st = ensure_smem_attr((const void*)kern, 227 * 1024, attr_ctx, dev); st != WQ_OK) return st;
     Params prm{};
     prm.x = pb.x; prm.w_q = pb.w_q; prm.w_lo = pb.w_lo; prm.s = pb.scales; prm.z = pb.zeros;
     prm.bias = pb.bias;

@@ -66,6 +66,53 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t 
     return true;
 }
 
+// Unique ID of the CUDA context current on this thread (0 when there is none or
+// the driver does not report one).  A context that is destroyed and created
+// again (cudaDeviceReset) gets a new ID, so per-context state keyed on it --
+// a kernel attribute, a symbol's device address -- is set up again.
+uint64_t current_ctx_id() {
+    using GetCurrent = CUresult (*)(CUcontext*);
+    using GetId = CUresult (*)(CUcontext, unsigned long long*);
+    static std::atomic<GetCurrent> get_current{nullptr};
+    static std::atomic<GetId> get_id{nullptr};
+    GetCurrent gc = get_current.load(std::memory_order_acquire);
+    GetId gi = get_id.load(std::memory_order_acquire);
+    if (!gc || !gi) {
+        void* p1 = nullptr;
+        void* p2 = nullptr;
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p1, cudaEnableDefault, &q1) != cudaSuccess ||
+            q1 != cudaDriverEntryPointSuccess ||
+            cudaGetDriverEntryPoint("cuCtxGetId", &p2, cudaEnableDefault, &q2) != cudaSuccess ||
+            q2 != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            return 0;
+        }
+        gc = reinterpret_cast<GetCurrent>(p1);
+        gi = reinterpret_cast<GetId>(p2);
+        get_current.store(gc, std::memory_order_release);
+        get_id.store(gi, std::memory_order_release);
+    }
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (gc(&ctx) != CUDA_SUCCESS || !ctx || gi(ctx, &id) != CUDA_SUCCESS) return 0;
+    return (uint64_t)id;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per context.  `done` is the
+// caller's per-device record of the context the attribute was last set in; a
+// concurrent first call may set it twice, which is harmless (the setting is
+// idempotent), and no call launches before its own thread has set it.
+wq_status ensure_smem_attr(const void* kern, int bytes, std::atomic<uint64_t>* done, int dev) {
+    if (dev < 0 || dev >= MAX_DEVICES) return WQ_ERR_UNSUPPORTED;
+    const uint64_t id = current_ctx_id();
+    if (id != 0 && done[dev].load(std::memory_order_acquire) == id) return WQ_OK;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return WQ_ERR_CUDA;
+    if (id != 0) done[dev].store(id, std::memory_order_release);
+    return WQ_OK;
+}
+
 // SM count of the current device, queried once per device (148 without a device).
 int sm_count() {
     static std::atomic<int> cached[64];

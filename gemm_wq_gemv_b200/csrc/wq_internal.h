@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/wq.h"
 
 namespace wq {
@@ -41,6 +43,10 @@ wq_status gemv_device_status(int reset);
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t outer,
               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
 int sm_count();
+
+constexpr int MAX_DEVICES = 64;
+uint64_t current_ctx_id();
+wq_status ensure_smem_attr(const void* kern, int bytes, std::atomic<uint64_t>* done, int dev);
 
 inline wq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? WQ_OK : WQ_ERR_CUDA; }
 

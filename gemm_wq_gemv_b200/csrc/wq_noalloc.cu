@@ -10,7 +10,7 @@
 // device.  Nothing in it needs to start at zero: within one launch every slice
 // the owners read was written first.  Calls that may run at the same time on
 // one device share the array and race.
-#include <atomic>
+#include <mutex>
 
 #include <cuda_runtime.h>
 
@@ -20,27 +20,39 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_gemm_scratch[WQ_GEMM_NOALLOC_SCRATCH_BYTES];
 
-constexpr int MAX_DEVICES = 64;
-std::atomic<void*> g_scratch_addr[MAX_DEVICES];
+// The array's device address in the context current on each device, and the ID
+// of that context.  A context that is destroyed and made again (cudaDeviceReset)
+// loads the library's device image afresh, and the array may move: a new
+// context ID makes the next call look the address up again.
+struct ScratchSlot {
+    std::mutex mu;
+    uint64_t ctx = 0;
+    void* addr = nullptr;
+};
+ScratchSlot g_slot[wq::MAX_DEVICES];
 
-// Device address of the array on the current device, looked up on the first
-// call per device (with that device current) and kept.
+// Device address of the array in the current context, looked up (with that
+// device current) on the first call in each context and kept.
 wq_status scratch_address(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
         return WQ_ERR_CUDA;
     }
-    if (dev < 0 || dev >= MAX_DEVICES) return WQ_ERR_UNSUPPORTED;
-    void* a = g_scratch_addr[dev].load(std::memory_order_acquire);
-    if (!a) {
+    if (dev < 0 || dev >= wq::MAX_DEVICES) return WQ_ERR_UNSUPPORTED;
+    const uint64_t id = wq::current_ctx_id();
+    ScratchSlot& sl = g_slot[dev];
+    std::lock_guard<std::mutex> lk(sl.mu);
+    if (id == 0 || sl.ctx != id || !sl.addr) {
+        void* a = nullptr;
         if (cudaGetSymbolAddress(&a, g_gemm_scratch) != cudaSuccess || !a) {
             cudaGetLastError();
             return WQ_ERR_CUDA;
         }
-        g_scratch_addr[dev].store(a, std::memory_order_release);
+        sl.addr = a;
+        sl.ctx = id;
     }
-    *out = a;
+    *out = sl.addr;
     return WQ_OK;
 }
 

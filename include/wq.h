@@ -207,14 +207,20 @@ size_t wq_gemm_workspace_size(int M, int K, int N, int bits, int group_size);
  * WQ_GEMM_NOALLOC_SCRATCH_BYTES in the library's device image, one per
  * device, so the call allocates nothing.  Nothing in it needs to start at zero
  * and no state is kept in it between calls.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *   - The first call in each CUDA context looks up the array's device
+ *     address (cudaGetSymbolAddress) with that device current and keeps it,
+ *     keyed on the context's ID; make that first call before any stream
+ *     capture.  A context created again after cudaDeviceReset has a new ID,
+ *     so its first call looks the address up afresh (and should likewise come
+ *     before any capture).
  *   - Calls that may run at the same time on one device (other streams, other
  *     host threads) share the array and race; calls in one stream do not,
  *     WQ_FLAG_PDL_INPUTS_READY included (it waits before the scratch is used).
  *   - A shape whose wq_gemm_workspace_size() exceeds the array is rejected
- *     with WQ_ERR_SCRATCH_LIMIT before anything is launched.
+ *     with WQ_ERR_SCRATCH_LIMIT before anything is launched.  That size, and
+ *     so which shapes fit, depends on the current device's SM count (the
+ *     split-K plan fills the SMs once); on a 148-SM B200 every shape with
+ *     M <= 256 and N <= 2048 fits, and M = 512, K = 4096, N = 2048 needs 16 MiB.
  */
 #define WQ_GEMM_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 wq_status wq_gemm_noalloc(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,

@@ -196,6 +196,9 @@ int orc_dequant(const uint32_t* wq, const uint32_t* wlo, const uint16_t* s, cons
     if (G < 0 || N <= 0 || !supported_dt(dt)) return ORC_EARG;
     int kdiv = bits == 3 ? 32 : elems_per_word(bits);
     if (K % kdiv != 0) return ORC_EARG;
+    /* Rows are independent: each element is the same fp64 expression whichever
+     * thread computes it. */
+#pragma omp parallel for schedule(static)
     for (int k = 0; k < K; ++k) {
         int g = k / G;
         for (int n = 0; n < N; ++n) {

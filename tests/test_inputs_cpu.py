@@ -1,4 +1,5 @@
-"""The seeded input generator: what DESIGN states about the draws holds."""
+"""The seeded input generator: bf16 rounding equals torch's, fp16 and bf16 problems share one
+stream of draws, and the draws are deterministic and inside their stated ranges."""
 import numpy as np
 import torch
 
