@@ -133,8 +133,8 @@ wq_status wq_gemm(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
     wq_status st = check_product(x, w_q, w_lo, scales, zeros, y, M, K, N, bits, group_size, flags, G);
     if (st != WQ_OK) return st;
     if (bias && !aligned(bias, 2)) return WQ_ERR_ALIGNMENT;
-    if (K % 64 != 0) return WQ_ERR_INVALID_ARG;
-    if (G % 64 != 0 && 64 % G != 0) return WQ_ERR_UNSUPPORTED;
+    // the tensor-memory copy engine reads x in rows of K values: 16-byte multiples
+    if (K % 8 != 0) return WQ_ERR_ALIGNMENT;
     if (workspace && !aligned(workspace, 16)) return WQ_ERR_ALIGNMENT;
     if ((st = check_device()) != WQ_OK) return st;
     wq::Problem p{x, w_q, w_lo, scales, zeros, bias, y, M, K, N, bits, G, flags, workspace,
@@ -143,9 +143,9 @@ wq_status wq_gemm(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
 }
 
 size_t wq_gemm_workspace_size(int M, int K, int N, int bits, int group_size) {
-    if (!supported_bits(bits) || M < 1 || N < 1 || K < 64 || K % 64 != 0) return 0;
+    if (!supported_bits(bits) || M < 1 || N < 1 || K < 1 || K % k_quantum(bits) != 0 || K % 8 != 0) return 0;
     const int G = group_size == -1 ? K : group_size;
-    if (G < 1 || K % G != 0) return 0;
+    if (G < 1 || K % G != 0 || G % k_quantum(bits) != 0) return 0;
     return wq::gemm_workspace_bytes(M, K, N, bits, G);
 }
 
@@ -175,8 +175,9 @@ wq_status wq_matmul(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo
 wq_status wq_device_status(int reset) {
     const wq_status a = wq::gemm_device_status(reset);
     const wq_status b = wq::gemv_device_status(reset);
-    if (a == WQ_ERR_CUDA || b == WQ_ERR_CUDA) return WQ_ERR_CUDA;
-    return (a != WQ_OK) ? a : b;
+    const wq_status c = wq::gemv_lean_device_status(reset);
+    if (a == WQ_ERR_CUDA || b == WQ_ERR_CUDA || c == WQ_ERR_CUDA) return WQ_ERR_CUDA;
+    return (a != WQ_OK) ? a : (b != WQ_OK) ? b : c;
 }
 
 }  // extern "C"

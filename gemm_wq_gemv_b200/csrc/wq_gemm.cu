@@ -59,6 +59,7 @@ struct GemmParams {
     int CS;              // CTAs per cluster along K
     int kb_cta;          // k blocks per CTA
     int GPB;             // s/z rows per stage
+    int gmode;           // 0: G a multiple of 64; 1: G a power of two below 64; 2: any other G
     int g_shift;         // log2(G) when G < 64
     int stages;
     uint32_t stage_bytes, off_w, off_lo, off_s, off_z;
@@ -153,10 +154,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
                 tma_load_2d(st + p.off_s, &tm_s, &full_tma[s], n0, grow);
                 tma_load_2d(st + p.off_z, &tm_z, &full_tma[s], n0, grow);
                 kg += BK;
-                if (p.GPB == 1) {  // a group spans whole k blocks: next row once kg reaches it
+                if (p.gmode == 0) {         // a group spans whole k blocks: next row once kg reaches it
                     if (kg >= gnext) { ++grow; gnext += p.G; }
-                } else {           // 64 / G rows per k block
+                } else if (p.gmode == 1) {  // 64 / G rows per k block
                     grow += p.GPB;
+                } else {                    // the group of the block's first k, then GPB rows
+                    grow = kg / p.G;
                 }
                 if (++s == p.stages) { s = 0; ph ^= 1u; }
             }
@@ -232,10 +235,27 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
                 const uint8_t* st = base + (size_t)s * p.stage_bytes;
                 uint32_t c[NC], s2, zs2;
                 uint32_t a32[32];  // this thread's 64 k values (32 pairs) of the stage's A row
-                if (p.GPB == 1) {  // one group covers the whole k block
+                if (p.gmode == 0) {  // one group covers the whole k block
                     consts(st, 0, c, s2, zs2);
 #pragma unroll
                     for (int rw = 0; rw < RW; ++rw) word(st, rw, c, s2, zs2, a32 + rw * (EPS / 2));
+                } else if (p.gmode == 2) {
+                    // Group boundaries anywhere in the block (G a multiple of the
+                    // codes per word, so never inside a word row): row gi of the
+                    // stage's s, z tile is group (block start) / G + gi.
+                    const int kbase = (kb0 + kb) * BK;
+                    int gi = 0;
+                    int next = (kbase / p.G + 1) * p.G - kbase;  // block offset of the next group start
+                    consts(st, 0, c, s2, zs2);
+#pragma unroll
+                    for (int rw = 0; rw < RW; ++rw) {
+                        if (rw * EPS >= next) {
+                            ++gi;
+                            next += p.G;
+                            consts(st, gi, c, s2, zs2);
+                        }
+                        word(st, rw, c, s2, zs2, a32 + rw * (EPS / 2));
+                    }
                 } else {
                     int cur = -1;
 #pragma unroll
@@ -364,7 +384,7 @@ Tiling plan(int M, int K, int N, size_t ws_bytes) {
     t.TN = std::max(32, (tn + 31) / 32 * 32);  // the epilogue reads tensor memory 32 columns at a time
     t.ntiles = (N + BMW - 1) / BMW;
     const int tiles = t.ntiles * t.mt;
-    const int KB = K / BK;
+    const int KB = (K + BK - 1) / BK;  // a ragged last block reads zeros past K
     const int sms = sm_count();
     t.CS = 1;
     for (int c = 8; c >= 2; c >>= 1) {
@@ -388,9 +408,16 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     p.bias = pb.bias;
     p.M = pb.M; p.K = pb.K; p.N = pb.N; p.G = pb.G;
     // s/z rows per 64-deep block: 1 if a group covers whole blocks, else 64 / G
-    if (pb.G % BK == 0) p.GPB = 1;
-    else if (BK % pb.G == 0) p.GPB = BK / pb.G;
-    else return WQ_ERR_UNSUPPORTED;
+    if (pb.G % BK == 0) {
+        p.GPB = 1;
+        p.gmode = 0;
+    } else if (BK % pb.G == 0) {
+        p.GPB = BK / pb.G;
+        p.gmode = 1;
+    } else {  // a 64-deep block meets at most ceil(63 / G) + 1 groups
+        p.GPB = (BK - 1 + pb.G - 1) / pb.G + 1;
+        p.gmode = 2;
+    }
     p.g_shift = 0;
     while ((1 << (p.g_shift + 1)) <= pb.G && p.g_shift < 6) ++p.g_shift;
 
@@ -399,7 +426,7 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     const int TN = t.TN, mt = t.mt, ntiles = t.ntiles, CS = t.CS;
     p.TN = TN;
     p.CS = CS;
-    p.kb_cta = pb.K / BK / CS;
+    p.kb_cta = (pb.K + BK - 1) / BK / CS;
     p.ws = static_cast<uint4*>(pb.ws);
     p.late_wait = (pb.flags & WQ_FLAG_PDL_INPUTS_READY) ? 1 : 0;
 
@@ -500,7 +527,7 @@ wq_status launch_gemm(const Problem& p, cudaStream_t s) {
 
 size_t gemm_workspace_bytes(int M, int K, int N, int bits, int G) {
     (void)bits;
-    if (G % BK != 0 && BK % G != 0) return 0;
+    (void)G;
     const Tiling t = plan(M, K, N, ~(size_t)0);
     return t.CS > 1 ? split_bytes(t, t.CS) : 0;
 }

@@ -797,6 +797,10 @@ wq_status launch_typed(const Problem& p, cudaStream_t s) {
 }  // namespace
 
 wq_status launch_gemv(const Problem& p, cudaStream_t s) {
+    if (gemv_lean_takes(p)) {
+        const wq_status st = launch_gemv_lean(p, s);
+        if (st != WQ_ERR_UNSUPPORTED) return st;  // else: its x stage does not fit; the kernel below takes it
+    }
     return (p.flags & WQ_FLAG_BF16) ? launch_typed<true>(p, s) : launch_typed<false>(p, s);
 }
 

@@ -31,6 +31,10 @@ wq_status launch_pack(const uint8_t* codes, int K, int N, int bits, uint32_t* w_
 wq_status launch_unpack(const uint32_t* w_q, const uint32_t* w_lo, int K, int N, int bits,
                         uint8_t* codes, cudaStream_t s);
 wq_status launch_gemv(const Problem& p, cudaStream_t s);
+// GEMV with a small shared-memory footprint for 4- and 8-bit words and M <= 8
+// (wq_gemv_lean.cu); launch_gemv routes the shapes it takes there.
+bool gemv_lean_takes(const Problem& p);
+wq_status launch_gemv_lean(const Problem& p, cudaStream_t s);
 wq_status launch_gemm(const Problem& p, cudaStream_t s);
 size_t gemm_workspace_bytes(int M, int K, int N, int bits, int G);
 
@@ -38,6 +42,7 @@ size_t gemm_workspace_bytes(int M, int K, int N, int bits, int G);
 // Reading synchronises the device; reset clears the word.
 wq_status gemm_device_status(int reset);
 wq_status gemv_device_status(int reset);
+wq_status gemv_lean_device_status(int reset);
 
 // 2-D tiled TMA descriptor for a row-major (outer, inner) array.
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t outer,

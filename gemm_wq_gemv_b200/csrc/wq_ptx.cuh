@@ -131,6 +131,31 @@ __device__ __forceinline__ uint32_t bfma2_u32(uint32_t a, uint32_t b, uint32_t c
     return r;
 }
 
+// fp16x2 add / subtract (round to nearest even), min and max.
+__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t hmin2_u32(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("min.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t hmax2_u32(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 template <bool BF>
 __device__ __forceinline__ uint32_t fma2_u32(uint32_t a, uint32_t b, uint32_t c) {
     return BF ? bfma2_u32(a, b, c) : hfma2_u32(a, b, c);
@@ -206,6 +231,16 @@ __device__ __forceinline__ void tma_load_2d_u32(uint32_t dst, const void* tmap, 
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
         "[%2];" ::"r"(dst),
         "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+// The same with a 64-bit L2 cache policy (createpolicy), e.g. evict-first for streamed data.
+__device__ __forceinline__ void tma_load_2d_u32_hint(uint32_t dst, const void* tmap, uint64_t* bar, int c0, int c1,
+                                                     uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+        "[%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+        "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "l"(pol)
         : "memory");
 }
 

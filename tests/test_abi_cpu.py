@@ -93,9 +93,17 @@ def test_gemv_specific_limits(libwq):
     assert gemv(L, "wq_gemv", M=17) == 1
     assert gemv(L, "wq_gemv", bits=4, G=16, K=512) == 2   # group not a multiple of 4*eps
     assert gemv(L, "wq_gemv", bits=1, G=64, K=512) == 2
-    assert gemv(L, "wq_gemm", K=544, G=-1) == 1           # gemm needs K % 64
-    assert gemv(L, "wq_gemm", K=576, G=96) == 2           # group neither a multiple nor a divisor of 64
     assert gemv(L, "wq_gemm", ws=P + 8, ws_bytes=1 << 20) == 3  # workspace alignment
+    assert gemv(L, "wq_gemm", bits=8, K=516, G=-1) == 3   # x rows of 516 values are not 16-byte multiples
+    import torch
+    if not torch.cuda.is_available():
+        # any K that is a multiple of eps (and of 8) and any group that divides K and is a
+        # multiple of eps pass the host checks and reach CUDA, which has no device here
+        assert gemv(L, "wq_gemm", K=544, G=-1) == 6       # a ragged 64-deep block
+        assert gemv(L, "wq_gemm", K=4160, N=264, M=48, G=-1) == 6
+        assert gemv(L, "wq_gemm", K=576, G=96) == 6       # groups straddle 64-deep blocks
+        assert gemv(L, "wq_gemm", bits=3, wlo=P, K=96 * 32, G=96) == 6
+        assert gemv(L, "wq_gemm", bits=8, K=520, G=40) == 6
 
 
 def test_gemm_workspace_size(libwq):
@@ -115,8 +123,9 @@ def test_gemm_workspace_size(libwq):
     assert size(1, 128, 4096, 4, 128) == 0       # two k blocks: no split
     assert size(0, 4096, 4096, 4, 128) == 0      # invalid arguments
     assert size(1, 4096, 4096, 5, 128) == 0
-    assert size(1, 4000, 4096, 4, 128) == 0
-    assert size(1, 4096, 4096, 4, 96) == 0
+    assert size(1, 4000, 4096, 4, 128) == 0      # the group does not divide K
+    assert size(1, 4092, 4096, 4, -1) == 0       # K not a multiple of 8
+    assert size(1, 4096, 4096, 4, 12) == 0       # group not a multiple of eps
 
 
 def test_pack_argument_checks(libwq):

@@ -4,14 +4,19 @@ import pytest
 
 import wq_inputs
 from gpu_cases import oracle_product, to_dev
+from guard import Guarded, Guarded1D
 from parity import check_product
 
 pytestmark = pytest.mark.gpu
 
 
 def run_gemm(libwq, d, bits, G, **kw):
+    """The product into an output with sentinel rows around it, which must survive."""
     w_q, w_lo = libwq.pack_kmajor(d["codes"], bits)
-    y = libwq.gemm(d["x"], w_q, w_lo, d["scales"], d["zeros"], bits, G, **kw)
+    M, N = d["x"].shape[0], w_q.shape[1]
+    out = Guarded((M, N), d["x"].dtype, d["x"].device)
+    y = libwq.gemm(d["x"], w_q, w_lo, d["scales"], d["zeros"], bits, G, out=out.view, **kw)
+    assert out.intact(), "a store landed outside y"
     return y.cpu().numpy()
 
 
@@ -49,6 +54,14 @@ SHAPES = [
     (512, 128, 8192, 8, 128),   # many tiles, no split
     (64, 8192, 136, 1, -1),
     (7, 4096, 2048, 2, 32),
+    # ragged last 64-deep block, and groups whose boundaries fall inside a block
+    (48, 4160, 264, 4, -1),     # K = 65 blocks: a ragged block, K split over clusters
+    (3, 544, 64, 4, -1),
+    (40, 576, 136, 4, 96),      # group 96 straddles blocks
+    (24, 3072, 128, 3, 96),     # 3-bit planes with group 96
+    (9, 520, 64, 8, 40),        # 8-bit, K = 8 blocks + 8, group 40
+    (96, 1088, 256, 2, 64),     # 17 blocks
+    (2, 96, 64, 4, 32),         # one and a half blocks
 ]
 
 
@@ -115,13 +128,29 @@ def test_deterministic_and_status(cuda, libwq):
 
 
 def test_rejected_calls(cuda, libwq):
-    import torch
-    case = wq_inputs.custom(4, 96, 64, 4, 32, seed=1)
+    """x must come in 16-byte rows for the tensor-memory copy engine: 8-bit
+    codes with K = 516 pass every format rule but are refused (WQ_ERR_ALIGNMENT)."""
+    case = wq_inputs.custom(4, 516, 64, 8, -1, seed=1)
     d = to_dev(case, cuda)
-    w_q, _ = libwq.pack_kmajor(d["codes"], 4)
-    with pytest.raises(libwq.WQError) as e:   # K % 64 != 0
-        libwq.gemm(d["x"], w_q, None, d["scales"], d["zeros"], 4, 32)
-    assert e.value.status == 1
+    w_q, _ = libwq.pack_kmajor(d["codes"], 8)
+    with pytest.raises(libwq.WQError) as e:
+        libwq.gemm(d["x"], w_q, None, d["scales"], d["zeros"], 8, -1)
+    assert e.value.status == 3
+
+
+def test_workspace_guards(cuda, libwq, orc):
+    """The split-K workspace: nothing is written outside the bytes the size query names."""
+    import torch
+    M, K, N, bits, G = 64, 4096, 512, 4, 128
+    case = wq_inputs.custom(M, K, N, bits, G, seed=11)
+    d = to_dev(case, cuda)
+    need = libwq.gemm_workspace_size(M, K, N, bits, G)
+    assert need > 0
+    ws = Guarded1D(need, torch.uint8, cuda)
+    y = run_gemm(libwq, d, bits, G, workspace=ws.view)
+    assert ws.intact(), "a store landed outside the workspace"
+    y_ref, b = oracle_product(orc, case)
+    check_product(y, y_ref, b, "workspace_guards")
 
 
 def test_pdl_flags(cuda, libwq):

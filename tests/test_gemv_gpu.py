@@ -4,14 +4,19 @@ import pytest
 
 import wq_inputs
 from gpu_cases import oracle_product, to_dev
+from guard import Guarded
 from parity import check_product
 
 pytestmark = pytest.mark.gpu
 
 
 def run_gemv(libwq, d, bits, G, **kw):
+    """The product into an output with sentinel rows around it, which must survive."""
     w_q, w_lo = libwq.pack_kmajor(d["codes"], bits)
-    y = libwq.gemv(d["x"], w_q, w_lo, d["scales"], d["zeros"], bits, G, **kw)
+    M, N = d["x"].shape[0], w_q.shape[1]
+    out = Guarded((M, N), d["x"].dtype, d["x"].device)
+    y = libwq.gemv(d["x"], w_q, w_lo, d["scales"], d["zeros"], bits, G, out=out.view, **kw)
+    assert out.intact(), "a store landed outside y"
     return y.cpu().numpy()
 
 
@@ -222,6 +227,15 @@ def test_rejected_calls(cuda, libwq):
     with pytest.raises(libwq.WQError) as e:
         libwq.gemv(x17, w_q, None, d["scales"], d["zeros"], 4, 128)
     assert e.value.status == 1
+    # group 16 is a legal 4-bit group size but not one wq_gemv takes (it needs a
+    # multiple of 4 * eps = 32): the library, not the binding, refuses it
+    s16 = torch.zeros((512 // 16, 256), dtype=torch.float16, device=cuda)
     with pytest.raises(libwq.WQError) as e:
-        libwq.gemv(d["x"], w_q, None, d["scales"], d["zeros"], 4, 16)
+        libwq.gemv(d["x"], w_q, None, s16, s16, 4, 16)
     assert e.value.status == 2
+    # tensors whose shapes disagree with K, N and the group size never reach the library
+    with pytest.raises(ValueError, match="scales"):
+        libwq.gemv(d["x"], w_q, None, d["scales"][:2], d["zeros"], 4, 128)
+    with pytest.raises(ValueError, match="out"):
+        libwq.gemv(d["x"], w_q, None, d["scales"], d["zeros"], 4, 128,
+                   out=torch.empty((1, 128), dtype=torch.float16, device=cuda))

@@ -79,3 +79,32 @@ def test_bad_arguments_raise_before_launch(cuda, libwq):
     with pytest.raises(libwq.WQError) as e:
         libwq.pack_kmajor(codes, 4)
     assert e.value.status == 1
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("K,N", [(32, 1), (96, 1000), (64, 5)])
+def test_packing_stays_inside_its_planes(cuda, libwq, orc, bits, K, N):
+    """Pack and unpack through the C ABI into buffers with sentinel rows around
+    them: every word and code lands inside its plane, none outside."""
+    import torch
+    from guard import Guarded
+    case = wq_inputs.custom(1, K, N, bits, -1, seed=7 * K + N + bits)
+    codes = torch.from_numpy(case.codes).to(cuda)
+    hs, ls = libwq.words_shape(K, N, bits)
+    gq = Guarded(hs, torch.int32, cuda)
+    glo = Guarded(ls, torch.int32, cuda) if ls else None
+    stream = torch.cuda.current_stream().cuda_stream
+    st = libwq.lib().wq_pack_kmajor(codes.data_ptr(), K, N, bits, gq.view.data_ptr(),
+                                    glo.view.data_ptr() if glo else None, None, stream)
+    assert st == 0
+    assert gq.intact() and (glo is None or glo.intact())
+    ref_q, ref_lo = orc.pack(case.codes, bits)
+    assert np.array_equal(_u32(gq.view), ref_q)
+    if bits == 3:
+        assert np.array_equal(_u32(glo.view), ref_lo)
+    back = Guarded((K, N), torch.uint8, cuda)
+    st = libwq.lib().wq_unpack_kmajor(gq.view.data_ptr(), glo.view.data_ptr() if glo else None, K, N, bits,
+                                      back.view.data_ptr(), stream)
+    assert st == 0
+    assert back.intact()
+    assert np.array_equal(back.view.cpu().numpy(), case.codes)

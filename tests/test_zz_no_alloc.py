@@ -85,6 +85,8 @@ def test_no_device_memory_taken_per_call(cuda, libwq):
 def test_rejected_on_the_device_too(cuda, libwq):
     """The scratch limit holds on a B200 (148 SMs): nothing is launched and y is untouched."""
     import torch
+    if torch.cuda.get_device_properties(cuda).multi_processor_count != 148:
+        pytest.skip("the split-K plan, and so which shapes exceed the scratch, follows the SM count")
     M, K, N = 256, 4096, 9472
     x = torch.zeros((M, K), dtype=torch.float16, device=cuda)
     w_q = torch.zeros((K // 8, N), dtype=torch.int32, device=cuda)
