@@ -39,6 +39,16 @@ and ``z = qmin - round(lo / s)`` clamped to the code range, so that 0 is
 exactly representable.  A zero scale becomes the fp32 machine epsilon, the
 replacement the page's kernels use (``_scale_round_config``, ``scale_eps``).
 
+Symmetric integers.  The page's search also takes symmetric arguments
+(``args.symmetric``: codes ``[-2**(bits-1), 2**(bits-1) - 1]`` in the fused
+kernel's launch, no zero point in its fake quantisation).  The page does not
+print their parameter rule either; ``qparams_symmetric`` takes the standard
+symmetric (absolute-maximum) rule: ``s = max(|lo|, |hi|) / ((qmax - qmin) / 2)``
+with the same zero-scale replacement, and ``z = 0``.  On the product's
+unsigned format a symmetric code ``q`` is stored as ``q + 2**(bits-1)`` with
+zero point ``2**(bits-1)`` (``to_unsigned``), which dequantises to the same
+``q * s``.
+
 Parity pins: ``tests/test_mse_oracle.py`` (a hand-worked example in
 ``tests/golden/mse_search.txt``, closed forms, invariants, special cases).
 """
@@ -50,10 +60,13 @@ F32 = np.float32
 EPS32 = np.finfo(np.float32).eps  # 2**-23
 
 
-def qrange(bits: int):
-    """Code range of unsigned (asymmetric) integers of ``bits`` bits."""
+def qrange(bits: int, symmetric: bool = False):
+    """Code range of ``bits``-bit integers: unsigned [0, 2^b - 1], or signed
+    [-2^(b-1), 2^(b-1) - 1] for the symmetric form."""
     if not 1 <= bits <= 8:
         raise ValueError(f"bits must be in 1..8, got {bits}")
+    if symmetric:
+        return -(1 << (bits - 1)), (1 << (bits - 1)) - 1
     return 0, (1 << bits) - 1
 
 
@@ -77,11 +90,28 @@ def qparams(lo, hi, bits: int):
     return s, z
 
 
-def fake_quant(w, s, z, bits: int):
+def qparams_symmetric(lo, hi, bits: int):
+    """fp32 (scale, zero point = 0) of the range [lo, hi] for signed codes:
+    s = max(|lo|, |hi|) / ((qmax - qmin) / 2), a zero scale replaced by 2^-23."""
+    qmin, qmax = qrange(bits, symmetric=True)
+    a = np.maximum(np.abs(np.asarray(lo, F32)), np.abs(np.asarray(hi, F32))).astype(F32)
+    s = (a / F32((qmax - qmin) / 2)).astype(F32)
+    s = np.where(s == F32(0), F32(EPS32), s).astype(F32)
+    return s, np.zeros_like(s, dtype=F32)
+
+
+def to_unsigned(codes, zero, bits: int):
+    """Signed symmetric codes and zero points as the product's unsigned format:
+    q + 2^(bits-1) and z + 2^(bits-1) (the same (q - z) * s)."""
+    off = 1 << (bits - 1)
+    return (np.asarray(codes) + off).astype(np.int32), (np.asarray(zero, F32) + F32(off)).astype(F32)
+
+
+def fake_quant(w, s, z, bits: int, symmetric: bool = False):
     """(codes, w_hat): q = clamp(round(w / s + z)), w_hat = (q - z) * s, fp32.
 
     ``s`` and ``z`` broadcast against ``w`` (one value per group: shape (..., 1))."""
-    qmin, qmax = qrange(bits)
+    qmin, qmax = qrange(bits, symmetric)
     w = np.asarray(w, F32)
     t = ((w / s).astype(F32) + z).astype(F32)
     q = np.clip(np.rint(t), F32(qmin), F32(qmax)).astype(F32)
@@ -100,12 +130,15 @@ def group_error(w, w_hat, norm: float) -> np.ndarray:
 
 
 def search(w, bits: int, group_size: int, maxshrink: float = 0.2, grid: int = 100,
-           norm: float = 2.4, patience: int | None = None) -> dict:
+           norm: float = 2.4, patience: int | None = None, symmetric: bool = False) -> dict:
     """The grid search for every group of W (rows x cols, fp32; cols % group_size == 0).
 
     Defaults are the page's benchmark CLI (maxshrink 0.20, grid 100, norm 2.4);
     its patience default, 5, is passed explicitly, since None means every
     candidate is evaluated.
+
+    ``symmetric``: signed codes and the symmetric parameter rule
+    (``qparams_symmetric``); the zero points returned are then 0 (signed).
 
     Returns a dict of arrays of shape (rows, cols // group_size):
     ``step`` (best candidate index), ``err`` (its error), ``scale``, ``zero``
@@ -125,6 +158,7 @@ def search(w, bits: int, group_size: int, maxshrink: float = 0.2, grid: int = 10
     mn = grp.min(axis=-1)
     mx = grp.max(axis=-1)
     ps = candidates(maxshrink, grid)
+    params = (lambda lo, hi: qparams_symmetric(lo, hi, bits)) if symmetric else (lambda lo, hi: qparams(lo, hi, bits))
     best_err = np.full(mn.shape, np.inf)
     best_step = np.zeros(mn.shape, dtype=np.int32)
     errors = []
@@ -132,8 +166,8 @@ def search(w, bits: int, group_size: int, maxshrink: float = 0.2, grid: int = 10
     for i, p in enumerate(ps):
         lo = (mn * p).astype(F32)
         hi = (mx * p).astype(F32)
-        s, z = qparams(lo, hi, bits)
-        _, w_hat = fake_quant(grp, s[..., None], z[..., None], bits)
+        s, z = params(lo, hi)
+        _, w_hat = fake_quant(grp, s[..., None], z[..., None], bits, symmetric)
         err = group_error(grp, w_hat, norm)
         errors.append(err)
         improved = err < best_err
@@ -146,6 +180,6 @@ def search(w, bits: int, group_size: int, maxshrink: float = 0.2, grid: int = 10
     p_best = ps[best_step]
     lo = (mn * p_best).astype(F32)
     hi = (mx * p_best).astype(F32)
-    s, z = qparams(lo, hi, bits)
+    s, z = params(lo, hi)
     return {"step": best_step, "err": best_err, "scale": s, "zero": z, "min": lo, "max": hi,
             "errors": np.stack(errors, axis=-1), "steps_evaluated": len(errors)}

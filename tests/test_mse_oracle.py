@@ -27,8 +27,9 @@ def pin_golden(impl):
         G = c["group"]
         w = np.array(c["values"], np.float32).reshape(1, -1)
         patience = int(c["patience"][0]) if "patience" in c else None
+        kw = {"symmetric": True} if "symmetric" in c and int(c["symmetric"][0]) else {}
         r = impl.search(w, c["bits"], G, maxshrink=c["maxshrink"][0], grid=int(c["grid"][0]),
-                        norm=c["norm"][0], patience=patience)
+                        norm=c["norm"][0], patience=patience, **kw)
         assert r["steps_evaluated"] == int(c["evaluated"][0]), name
         assert np.array_equal(r["step"][0], np.array(c["steps"], np.int32)), (name, r["step"])
         assert np.array_equal(r["scale"][0], np.array(c["scale"], np.float32)), (name, r["scale"])
@@ -100,8 +101,46 @@ def pin_zero_group(impl):
     assert np.all(r["zero"] == 0) and np.all(r["err"] == 0)
 
 
+def pin_symmetric_range_matches_asymmetric(impl):
+    """A group whose range is symmetric, mn = -mx with mx = (2^b - 1)/2 * 2^-e, and one
+    candidate (p = 1): the asymmetric rule gives the same scale 2^-e and zero point
+    2^(b-1), so the symmetric search must give the same scale, errors and, stored in
+    the product's unsigned format, zero point 2^(b-1)."""
+    rng = np.random.default_rng(10)
+    for bits in (2, 3, 4, 8):
+        half = ((1 << bits) - 1) / 2.0
+        G = 32
+        e = rng.integers(2, 8, size=(3, 4, 1))
+        mx = half * 2.0 ** -e
+        w = rng.uniform(-1.0, 1.0, size=(3, 4, G)) * mx
+        w[..., 0] = -mx[..., 0]
+        w[..., 1] = mx[..., 0]
+        w = w.astype(np.float32).reshape(3, 4 * G)
+        a = impl.search(w, bits, G, maxshrink=1.0, grid=1, norm=2.4)
+        b = impl.search(w, bits, G, maxshrink=1.0, grid=1, norm=2.4, symmetric=True)
+        assert np.array_equal(b["scale"], (2.0 ** -e[..., 0]).astype(np.float32)), bits
+        assert np.array_equal(a["scale"], b["scale"]), bits
+        assert np.array_equal(a["errors"], b["errors"]), bits
+        assert np.all(b["zero"] == 0), bits
+        _, zu = mo.to_unsigned(np.zeros_like(b["step"]), b["zero"], bits)
+        assert np.array_equal(zu, a["zero"]), bits
+
+
+def pin_symmetric_invariants(impl):
+    """Power-of-two scaling and the first-argmin rule hold for the symmetric form too."""
+    rng = np.random.default_rng(11)
+    w = rng.standard_normal((4, 256)).astype(np.float32)
+    base = impl.search(w, 4, 32, maxshrink=0.3, grid=50, norm=2.4, symmetric=True)
+    assert np.all(base["zero"] == 0)
+    assert np.array_equal(base["step"], np.argmin(base["errors"], axis=-1))
+    r = impl.search(w * np.float32(0.25), 4, 32, maxshrink=0.3, grid=50, norm=2.4, symmetric=True)
+    assert np.array_equal(r["step"], base["step"])
+    assert np.array_equal(r["scale"], base["scale"] * np.float32(0.25))
+
+
 PINS = [pin_golden, pin_on_grid_is_exact, pin_power_of_two_scaling, pin_exhaustive_is_first_argmin,
-        pin_long_patience_changes_nothing, pin_zero_group]
+        pin_long_patience_changes_nothing, pin_zero_group, pin_symmetric_range_matches_asymmetric,
+        pin_symmetric_invariants]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -149,8 +188,8 @@ def _qparams_zero_sign(lo, hi, bits):        # z = qmin + round(lo / s)
     return s, np.clip(np.float32(qmin) + np.rint(lo / s), qmin, qmax).astype(np.float32)
 
 
-def _fake_quant_floor(w, s, z, bits):        # floor instead of round to nearest
-    qmin, qmax = mo.qrange(bits)
+def _fake_quant_floor(w, s, z, bits, symmetric=False):   # floor instead of round to nearest
+    qmin, qmax = mo.qrange(bits, symmetric)
     q = np.clip(np.floor((np.asarray(w, np.float32) / s + z).astype(np.float32)), qmin, qmax).astype(np.float32)
     return q.astype(np.int32), ((q - z) * s).astype(np.float32)
 
@@ -172,23 +211,24 @@ def _candidates_wrong(maxshrink, grid):      # p_i = 1 - i * maxshrink / grid
     return np.array([1.0 - i * maxshrink / grid for i in range(n)]).astype(np.float32)
 
 
-def _search_ties_move(w, bits, group_size, maxshrink=0.2, grid=100, norm=2.4, patience=None):
-    r = mo.search(w, bits, group_size, maxshrink, grid, norm, patience)
+def _search_ties_move(w, bits, group_size, maxshrink=0.2, grid=100, norm=2.4, patience=None, symmetric=False):
+    r = mo.search(w, bits, group_size, maxshrink, grid, norm, patience, symmetric)
     e = r["errors"]
     last = e.shape[-1] - 1 - np.argmin(e[..., ::-1], axis=-1)   # the last smallest error wins
     r = dict(r)
     r["step"] = last.astype(np.int32)
     p = mo.candidates(maxshrink, grid)[last]
     grp = np.asarray(w, np.float32).reshape(w.shape[0], -1, group_size)
-    r["scale"], r["zero"] = mo.qparams((grp.min(-1) * p).astype(np.float32),
-                                       (grp.max(-1) * p).astype(np.float32), bits)
+    qp = mo.qparams_symmetric if symmetric else mo.qparams
+    r["scale"], r["zero"] = qp((grp.min(-1) * p).astype(np.float32), (grp.max(-1) * p).astype(np.float32), bits)
     return r
 
 
-def _search_patience_per_group(w, bits, group_size, maxshrink=0.2, grid=100, norm=2.4, patience=None):
+def _search_patience_per_group(w, bits, group_size, maxshrink=0.2, grid=100, norm=2.4, patience=None,
+                               symmetric=False):
     if patience is None:
-        return mo.search(w, bits, group_size, maxshrink, grid, norm)
-    r = dict(mo.search(w, bits, group_size, maxshrink, grid, norm))
+        return mo.search(w, bits, group_size, maxshrink, grid, norm, symmetric=symmetric)
+    r = dict(mo.search(w, bits, group_size, maxshrink, grid, norm, symmetric=symmetric))
     e = r["errors"]
     steps = np.zeros(e.shape[:-1], np.int32)
     for idx in np.ndindex(*e.shape[:-1]):
@@ -209,7 +249,20 @@ def _search_patience_per_group(w, bits, group_size, maxshrink=0.2, grid=100, nor
     return r
 
 
+def _qparams_sym_denominator(lo, hi, bits):   # symmetric scale over qmax = 2^(b-1) - 1
+    qmin, qmax = mo.qrange(bits, symmetric=True)
+    a = np.maximum(np.abs(np.asarray(lo, np.float32)), np.abs(np.asarray(hi, np.float32)))
+    s = (a / np.float32(qmax)).astype(np.float32)
+    return np.where(s == 0, np.float32(mo.EPS32), s).astype(np.float32), np.zeros_like(s)
+
+
+def _fake_quant_sym_unsigned(w, s, z, bits, symmetric=False):   # symmetric codes clipped to [0, 2^b - 1]
+    return mo.fake_quant(w, s, z, bits, False)
+
+
 MUTANTS = {
+    "symmetric_scale_over_qmax": _module_with(qparams_symmetric=_qparams_sym_denominator),
+    "symmetric_unsigned_clip": _module_with(fake_quant=_fake_quant_sym_unsigned),
     "range_without_zero": _module_with(qparams=_qparams_no_zero),
     "zero_point_sign": _module_with(qparams=_qparams_zero_sign),
     "floor_rounding": _module_with(fake_quant=_fake_quant_floor),
