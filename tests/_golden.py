@@ -23,7 +23,7 @@ def read_cases(name: str) -> dict:
             cur = None
         else:
             toks = rest.split()
-            if key in ("wq", "wlo"):
+            if key in ("wq", "wlo", "qz"):
                 cur[key] = [int(t, 16) for t in toks]
             elif key in ("bits", "K", "N", "M", "group"):
                 cur[key] = int(toks[0])
