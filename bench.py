@@ -43,6 +43,9 @@ HEADLINE = "decode_gemv_m1"
 GEMM_WL = "prefill_gemm"
 METRIC = "packed-int GEMV HBM GB/s and % of peak at M=1; wq_gemm TFLOPS at M=512"
 FALLBACK_HBM, FALLBACK_TF = 6650.0, 1590.0
+# Nominal B200 figures, reported beside the measured ones: HBM3e ~8 TB/s,
+# dense fp16 / bf16 tensor cores 2.25 PFLOP/s.
+NOMINAL_HBM, NOMINAL_TF = 8000.0, 2250.0
 
 
 def algo_bytes(wl) -> int:
@@ -289,7 +292,68 @@ def cpu_baseline(seconds: float = 10.0):
             oracle.set_threads(cores)
     return {"value": round(algo_bytes(wl) * reps / el / 1e9, 3), "unit": "GB/s", "cores": cores,
             "kind": "oracle", "cpu": cpu_model(), "single_thread": single,
+            "numpy": numpy_baseline(seconds / 4),
             "sample": f"{reps} full decode GEMVs (M=1, K=N=4096, 4-bit, g128) in {el:.1f} s, fp64 C, OpenMP"}
+
+
+def numpy_baseline(seconds: float):
+    """The NumPy twin of the oracle (unpack, dequantise, fp64 matmul through the
+    BLAS NumPy links) on full decode GEMVs, with the BLAS thread count."""
+    import oracle
+    wl = wq_inputs.WORKLOADS[HEADLINE]
+    case = wq_inputs.draw(wl, 0)
+    wq_, wlo = oracle.numpy_oracle.pack(case.codes, wl.bits)
+    try:
+        from threadpoolctl import threadpool_info
+        blas = [{"api": d.get("internal_api"), "threads": d.get("num_threads")} for d in threadpool_info()
+                if d.get("user_api") == "blas"]
+    except Exception:  # threadpoolctl missing: the count is unknown
+        blas = None
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.numpy_oracle.wq_matmul(case.x, wq_, wlo, case.scales, case.zeros, wl.bits, wl.group_size)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or reps >= 200:
+            break
+    return {"value": round(algo_bytes(wl) * reps / el / 1e9, 4), "unit": "GB/s", "blas": blas,
+            "sample": f"{reps} full decode GEMVs in {el:.1f} s, NumPy fp64 (dequantise, then x @ w)"}
+
+
+def mse_bench(wq, torch, dev, reps: int = 5):
+    """Times wq_mse_search on the page's workload shape with synthetic weights
+    drawn like an nn.Linear initialisation (uniform in +-1/sqrt(4096)), and the
+    NumPy oracle on a bounded sample of the same shape's rows."""
+    import numpy as np
+    R, C, G, bits = 14336, 4096, 16, 4
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(42)
+    w = (torch.rand((R, C), generator=gen, device=dev) * 2 - 1) / 64.0
+    out = {"workload": f"W {R}x{C} fp32, group {G}, {bits}-bit, 20 candidates (maxshrink 0.2, grid 100), norm 2.4"}
+    for name, pat in (("patience_5", 5), ("exhaustive", None)):
+        for _ in range(2):
+            wq.mse_search(w, bits, G, norm=2.4, patience=pat)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            r = wq.mse_search(w, bits, G, norm=2.4, patience=pat)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        out[name] = {"ms": round(ms, 4), "groups_per_s": round(R * C / G / (ms * 1e-3), 1),
+                     "weight_GBps": round(R * C * 4 / (ms * 1e-3) / 1e9, 1)}
+    # the oracle (NumPy, fp32 steps and fp64 errors) on 1024 rows of the same shape
+    import oracle.mse_observer as mo
+    sample = w[:1024].cpu().numpy()
+    t0 = time.perf_counter()
+    mo.search(sample, bits, G, maxshrink=0.2, grid=100, norm=2.4, patience=5)
+    el = time.perf_counter() - t0
+    out["cpu_baseline"] = {"groups_per_s": round(1024 * C / G / el, 1), "cores": 1, "kind": "oracle",
+                           "sample": f"1024 of the {R} rows ({1024 * C // G} groups) in {el:.2f} s, NumPy"}
+    del w, r
+    return out
 
 
 # ------------------------------------------------------------------ reference arm
@@ -515,6 +579,13 @@ def main(argv=None):
                "frac_of_sustained": round(b_tf / tf_sust, 4) if tf_sust else None}
         del bg, bsets, bx
 
+    # ---- the MSE-observer search (the step that chooses s and z) on the page's
+    # benchmark shape: a 14336 x 4096 fp32 weight, group 16, 4 bits, 20 shrink
+    # candidates (maxshrink 0.2, grid 100), patience 5, norm 2.4
+    mse = None
+    if not args.no_secondary:
+        mse = mse_bench(wq, torch, dev)
+
     # ---- every workload once (rank-local, for the table)
     table = []
     if not args.no_secondary:
@@ -558,12 +629,14 @@ def main(argv=None):
                              "WQ_FLAG_PDL_INPUTS_READY (each waits for the previous only before writing y)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                     "nominal_peak": NOMINAL_HBM, "frac_of_nominal": round(achieved / NOMINAL_HBM, 4),
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
                      "algorithmic_bytes_per_launch": algo_bytes(wl), "launch_us": round(per_launch_s * 1e6, 3)},
         "gemm": {"workload": "M=512 K=4096 N=2048 4-bit g128", "TFLOPS": round(g_tflops, 1),
                  "us": round(g_launch_s * 1e6, 3),
                  "roofline": {"bound": "tensor", "achieved": round(g_tflops, 1), "peak": tf_peak, "unit": "TFLOP/s",
                               "frac": round(g_tflops / tf_peak, 4), "traffic": g_traffic,
+                              "nominal_peak": NOMINAL_TF, "frac_of_nominal": round(g_tflops / NOMINAL_TF, 4),
                               "peak_source": "measured bf16 burst (fp16 nominal ratio 1:1)"},
                  "l2": f"{GL} rotating input sets ({algo_bytes(gwl) * GL / 1e6:.0f} MB) per graph"},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
@@ -578,6 +651,7 @@ def main(argv=None):
         "clocks": sampler.report(),
         "gpu_launches": args.steps * L * world,
         "workloads": table,
+        "mse_search": mse,
         "source": src_digest(),
     }
     if rank == 0 and world == 1:

@@ -17,6 +17,11 @@ Entry points (same names as the C ABI, without the ``wq_`` prefix):
 * ``matmul(...)``: same arguments as ``gemm``; ``wq_gemv`` or ``wq_gemm`` by M
 * ``gemm_noalloc(x, w_q, w_lo, scales, zeros, bits, group_size, out) -> out``
 * ``selftest_wait_timeout(limit_ns) -> status`` (the bounded-wait failure path)
+* ``from_gptqmodel(qweight, qzeros, bits, group_size, K, dtype) -> (w_q, w_lo, zeros)``
+  and ``gptqmodel_quantized_matmul(x, qweight, qzeros, scales, bits, group_size)``
+  (the GPTQModel packed format)
+* ``mse_search(w, bits, group_size, maxshrink=0.2, grid=100, norm=2.4,
+  patience=None, symmetric=False) -> dict`` (per-group s, z of the MSE observer)
 
 x, scales, zeros, bias and the output are all ``torch.float16`` or all
 ``torch.bfloat16`` (the type of x decides; bfloat16 sets ``WQ_FLAG_BF16``).
@@ -83,6 +88,10 @@ def lib() -> ctypes.CDLL:
         L.wq_gemm_noalloc.restype = i
         L.wq_device_status.argtypes = [i]
         L.wq_selftest_wait_timeout.argtypes = [ctypes.c_uint64, p]
+        L.wq_gptqmodel_convert.argtypes = [p, p, i, i, i, i, p, p, p, u, p]
+        L.wq_gptqmodel_convert.restype = i
+        L.wq_mse_search.argtypes = [p, i, i, i, i, i, i, i, ctypes.c_float, i, p, p, p, p, p, ctypes.c_size_t, p]
+        L.wq_mse_search.restype = i
         for f in ("wq_pack_kmajor", "wq_unpack_kmajor", "wq_gemv", "wq_gemm", "wq_device_status",
                   "wq_selftest_wait_timeout"):
             getattr(L, f).restype = i
@@ -141,11 +150,13 @@ def words_shape(K: int, N: int, bits: int):
 
 
 _BITS = (1, 2, 3, 4, 8)
+_EPS = {1: 32, 2: 16, 3: 16, 4: 8, 8: 4}  # codes per word of the main plane
 
 
 def _same_device(ref, **tensors):
+    d = ref.device
     for name, t in tensors.items():
-        if t is not None and t.device != ref.device:
+        if t is not None and t.device != d:
             raise ValueError(f"{name} is on {t.device}, x on {ref.device}: all tensors must share one device")
 
 
@@ -155,19 +166,19 @@ def _check_planes(w_q, w_lo, K: int, bits: int):
     The library sizes its copies from K, N and bits, so a plane of another shape
     would be read out of its bounds; a bit width it does not take is left to the
     C call, which rejects it."""
-    if bits not in _BITS:
+    eps = _EPS.get(bits)
+    if eps is None:
         return
     N = w_q.shape[1]
-    hs, ls = words_shape(K, N, bits)
-    if tuple(w_q.shape) != hs:
-        raise ValueError(f"w_q has shape {tuple(w_q.shape)}; K={K}, {bits}-bit words need {hs}")
-    if ls is None and w_lo is not None:
-        raise ValueError(f"w_lo must be None for {bits}-bit words")
-    if ls is not None:
+    if w_q.shape != (K // eps, N):
+        raise ValueError(f"w_q has shape {tuple(w_q.shape)}; K={K}, {bits}-bit words need {(K // eps, N)}")
+    if bits == 3:
         if w_lo is None:
             raise ValueError("3-bit words need the lo plane w_lo")
-        if tuple(w_lo.shape) != ls:
-            raise ValueError(f"w_lo has shape {tuple(w_lo.shape)}; K={K} 3-bit needs {ls}")
+        if w_lo.shape != (K // 32, N):
+            raise ValueError(f"w_lo has shape {tuple(w_lo.shape)}; K={K} 3-bit needs {(K // 32, N)}")
+    elif w_lo is not None:
+        raise ValueError(f"w_lo must be None for {bits}-bit words")
 
 
 def _check_product(x, w_q, w_lo, scales, zeros, bias, out, bits: int, group_size: int):
@@ -175,20 +186,27 @@ def _check_product(x, w_q, w_lo, scales, zeros, bias, out, bits: int, group_size
     imply, and sits on x's device.  Raises ValueError before any C call.
     Shapes the C rules reject anyway (a K that is not a multiple of the word
     width, a group size that does not divide K) are left to the C call, which
-    names the rule."""
+    names the rule.  (Runs on every call: kept to plain shape comparisons.)"""
     M, K = x.shape
     N = w_q.shape[1]
-    _same_device(x, w_q=w_q, w_lo=w_lo, scales=scales, zeros=zeros, bias=bias, out=out)
+    d = x.get_device()
+    if (d < 0 or w_q.get_device() != d or scales.get_device() != d or zeros.get_device() != d
+            or (w_lo is not None and w_lo.get_device() != d) or (bias is not None and bias.get_device() != d)
+            or (out is not None and out.get_device() != d)):
+        _same_device(x, w_q=w_q, w_lo=w_lo, scales=scales, zeros=zeros, bias=bias, out=out)
     _check_planes(w_q, w_lo, K, bits)
     G = K if group_size == -1 else group_size
     if G > 0 and K % G == 0:
-        for name, t in (("scales", scales), ("zeros", zeros)):
-            if tuple(t.shape) != (K // G, N):
-                raise ValueError(f"{name} has shape {tuple(t.shape)}; K={K}, group size {group_size} "
-                                 f"and N={N} need {(K // G, N)}")
-    if bias is not None and tuple(bias.shape) != (N,):
+        sz = (K // G, N)
+        if scales.shape != sz:
+            raise ValueError(f"scales has shape {tuple(scales.shape)}; K={K}, group size {group_size} "
+                             f"and N={N} need {sz}")
+        if zeros.shape != sz:
+            raise ValueError(f"zeros has shape {tuple(zeros.shape)}; K={K}, group size {group_size} "
+                             f"and N={N} need {sz}")
+    if bias is not None and bias.shape != (N,):
         raise ValueError(f"bias has shape {tuple(bias.shape)}; N={N} needs ({N},)")
-    if out is not None and tuple(out.shape) != (M, N):
+    if out is not None and out.shape != (M, N):
         raise ValueError(f"out has shape {tuple(out.shape)}; M={M}, N={N} need {(M, N)}")
 
 
@@ -368,3 +386,82 @@ def matmul(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pd
 
 def uses_gemv(M: int, K: int, N: int, bits: int, group_size: int) -> bool:
     return bool(lib().wq_matmul_uses_gemv(M, K, N, bits, group_size))
+
+
+def mse_search(w, bits: int, group_size: int, maxshrink: float = 0.2, grid: int = 100, norm: float = 2.4,
+               patience=None, symmetric: bool = False):
+    """``wq_mse_search``: the MSE-observer search of each group's scale and zero
+    point over ``int(maxshrink * grid)`` shrink candidates (as the page counts
+    them), on the current stream.
+
+    ``w``: (rows, cols) float32 CUDA tensor, groups of ``group_size`` values
+    along a row.  ``patience``: None evaluates every candidate.  Returns a dict
+    of (rows, cols // group_size) tensors ``step`` (int32), ``scale``,
+    ``zero`` and ``err`` (float32); with ``symmetric`` the zero points are 0
+    (signed codes)."""
+    torch = _torch()
+    _need(w, torch.float32, "w")
+    rows, cols = w.shape
+    steps = int(maxshrink * grid)
+    if group_size < 1 or cols % group_size != 0:
+        raise ValueError(f"cols={cols} is not a multiple of group_size={group_size}")
+    shape = (rows, cols // group_size)
+    out = {k: torch.empty(shape, dtype=torch.float32, device=w.device) for k in ("scale", "zero", "err")}
+    out["step"] = torch.empty(shape, dtype=torch.int32, device=w.device)
+    pat = 0 if patience is None else int(patience)
+    if patience is not None and pat < 1:
+        raise ValueError("patience must be at least 1 (None evaluates every candidate)")
+    ws = torch.empty(1, dtype=torch.int32, device=w.device) if pat else None
+    st = lib().wq_mse_search(_ptr(w), rows, cols, group_size, bits, 1 if symmetric else 0, steps, grid,
+                             float(norm), pat, _ptr(out["scale"]), _ptr(out["zero"]), _ptr(out["step"]),
+                             _ptr(out["err"]), _ptr(ws), 4 if ws is not None else 0, _stream())
+    _check("wq_mse_search", st)
+    return out
+
+
+_GQ_V = {2: 16, 3: 10, 4: 8, 8: 4}
+
+
+def from_gptqmodel(qweight, qzeros, bits: int, group_size: int, K: int, dtype=None):
+    """``wq_gptqmodel_convert``: GPTQModel (qweight, qzeros) -> this library's
+    (w_q, w_lo, zeros).  For 2, 4 and 8 bits w_q is ``qweight`` itself (the same
+    K-major words); 3-bit words (10 per int32) become the two planes.  ``zeros``
+    has the type ``dtype`` (float16 by default, or bfloat16)."""
+    torch = _torch()
+    dtype = torch.float16 if dtype is None else dtype
+    if dtype not in (torch.float16, torch.bfloat16):
+        raise TypeError("zeros are float16 or bfloat16")
+    if bits not in _GQ_V:
+        raise ValueError(f"the GPTQModel format takes 2, 3, 4 or 8 bits, not {bits}")
+    _need(qweight, torch.int32, "qweight")
+    _need(qzeros, torch.int32, "qzeros")
+    _same_device(qweight, qzeros=qzeros)
+    V = _GQ_V[bits]
+    N = qweight.shape[1]
+    G = K if group_size == -1 else group_size
+    if tuple(qweight.shape) != ((K + V - 1) // V, N):
+        raise ValueError(f"qweight has shape {tuple(qweight.shape)}; K={K}, {bits}-bit needs {((K + V - 1) // V, N)}")
+    if G < 1 or K % G != 0:
+        raise ValueError(f"group size {group_size} does not divide K={K}")
+    if tuple(qzeros.shape) != (K // G, (N + V - 1) // V):
+        raise ValueError(f"qzeros has shape {tuple(qzeros.shape)}; needs {(K // G, (N + V - 1) // V)}")
+    dev = qweight.device
+    zeros = torch.empty((K // G, N), dtype=dtype, device=dev)
+    if bits == 3:
+        hs, ls = words_shape(K, N, 3)
+        w_q = torch.empty(hs, dtype=torch.int32, device=dev)
+        w_lo = torch.empty(ls, dtype=torch.int32, device=dev)
+    else:
+        w_q, w_lo = qweight, None
+    flags = WQ_FLAG_BF16 if dtype is torch.bfloat16 else 0
+    st = lib().wq_gptqmodel_convert(_ptr(qweight), _ptr(qzeros), K, N, bits, group_size,
+                                    _ptr(w_q) if bits == 3 else None, _ptr(w_lo), _ptr(zeros), flags, _stream())
+    _check("wq_gptqmodel_convert", st)
+    return w_q, w_lo, zeros
+
+
+def gptqmodel_quantized_matmul(x, qweight, qzeros, scales, bits: int, group_size: int, out=None):
+    """The README's ``gptqmodel_quantized_matmul``: y = x @ dequantize(qweight)
+    with GPTQModel operands, through ``from_gptqmodel`` and ``matmul``."""
+    w_q, w_lo, zeros = from_gptqmodel(qweight, qzeros, bits, group_size, x.shape[1], dtype=_elem_type(x))
+    return matmul(x, w_q, w_lo, scales, zeros, bits, group_size, out=out)

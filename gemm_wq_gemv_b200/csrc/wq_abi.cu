@@ -172,6 +172,45 @@ wq_status wq_matmul(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo
                    workspace_bytes, stream);
 }
 
+wq_status wq_gptqmodel_convert(const uint32_t* qweight, const uint32_t* qzeros, int K, int N, int bits,
+                               int group_size, uint32_t* w_q, uint32_t* w_lo, uint16_t* zeros, unsigned flags,
+                               void* stream) {
+    if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return WQ_ERR_UNSUPPORTED;
+    wq_status st = check_plane_shape(K, N, bits, w_lo, true);
+    if (st != WQ_OK) return st;
+    if (flags & ~WQ_FLAG_BF16) return WQ_ERR_INVALID_ARG;
+    const int G = group_size == -1 ? K : group_size;
+    if (G < 1 || K % G != 0) return WQ_ERR_INVALID_ARG;
+    if (!qweight || !qzeros || !zeros || (bits == 3 && !w_q)) return WQ_ERR_INVALID_ARG;
+    if (!aligned(qweight, 4) || !aligned(qzeros, 4) || !aligned(zeros, 2) || (w_q && !aligned(w_q, 4)) ||
+        (w_lo && !aligned(w_lo, 4)))
+        return WQ_ERR_ALIGNMENT;
+    if ((st = check_device()) != WQ_OK) return st;
+    return wq::launch_gptqmodel_convert(qweight, qzeros, K, N, bits, G, w_q, w_lo, zeros,
+                                        (flags & WQ_FLAG_BF16) != 0, (cudaStream_t)stream);
+}
+
+wq_status wq_mse_search(const float* w, int rows, int cols, int group_size, int bits, int symmetric,
+                        int steps, int grid, float norm, int patience, float* scale, float* zero,
+                        int32_t* step, float* err, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+    if (bits < 1 || bits > 8) return WQ_ERR_UNSUPPORTED;
+    if (rows < 1 || cols < 1 || group_size < 1 || cols % group_size != 0) return WQ_ERR_INVALID_ARG;
+    if (symmetric != 0 && symmetric != 1) return WQ_ERR_INVALID_ARG;
+    if (steps < 1 || steps > 32 || grid < 1 || patience < 0) return WQ_ERR_INVALID_ARG;
+    if (!(norm > 0.0f) || !(norm < 3.0e38f)) return WQ_ERR_INVALID_ARG;  // rejects NaN and infinities
+    if (!w || !scale || !zero || !step || !err) return WQ_ERR_INVALID_ARG;
+    if (patience > 0 && (!workspace || workspace_bytes < 4)) return WQ_ERR_INVALID_ARG;
+    if (!aligned(w, 4) || !aligned(scale, 4) || !aligned(zero, 4) || !aligned(step, 4) ||
+        !aligned(err, 4) || (workspace && !aligned(workspace, 4)))
+        return WQ_ERR_ALIGNMENT;
+    wq_status st = check_device();
+    if (st != WQ_OK) return st;
+    return wq::launch_mse_search(w, rows, cols, group_size, bits, symmetric, steps, grid, norm, patience,
+                                 scale, zero, step, err, static_cast<uint32_t*>(workspace),
+                                 (cudaStream_t)stream);
+}
+
 wq_status wq_device_status(int reset) {
     const wq_status a = wq::gemm_device_status(reset);
     const wq_status b = wq::gemv_device_status(reset);

@@ -48,6 +48,12 @@ namespace {
 constexpr int LCOLS = 32;  // output columns per CTA
 constexpr int LWK = 8;     // warps per CTA (split along K)
 constexpr int LMAXS = 4;   // ring slots per warp (at most)
+// Independent MMA accumulator chains per column pair.  A warp's MMAs into one
+// accumulator form a dependency chain, and on B200 the warp-level MMA takes
+// long enough from issue to result that a single chain per pair, 2 MMAs per
+// quad for 16 quads, leaves the warp mostly waiting; the quads' MMAs rotate
+// over LACC accumulators instead, summed when a group ends.
+constexpr int LACC = 1;
 constexpr uint64_t LWAIT_NS = 2000000000ull;
 
 struct LeanParams {
@@ -276,15 +282,17 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const LeanParams p) {
     __syncthreads();
 
     // ---- (4) main loop
-    float acc[4][NE], dsum[2][4], xsum[NE];
+    float acc[4][NE], dsum[LACC][2][4], xsum[NE];
 #pragma unroll
     for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int e = 0; e < NE; ++e) acc[c][e] = 0.0f;
 #pragma unroll
-    for (int T = 0; T < 2; ++T)
+    for (int c = 0; c < LACC; ++c)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dsum[T][e] = 0.0f;
+        for (int T = 0; T < 2; ++T)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dsum[c][T][e] = 0.0f;
 #pragma unroll
     for (int e = 0; e < NE; ++e) xsum[e] = 0.0f;
     // B fragment address: token g (duplicates beyond M are harmless), word row t of quad 0
@@ -320,15 +328,19 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const LeanParams p) {
             const int T = c >> 1, half = c & 1;
 #pragma unroll
             for (int e = 0; e < NE; ++e) {
-                float d = dsum[T][2 * half + e];
+                float d = dsum[0][T][2 * half + e];
+#pragma unroll
+                for (int ch = 1; ch < LACC; ++ch) d += dsum[ch][T][2 * half + e];
                 if (k.frac) d = fmaf(-k.zr[c], xsum[e], d);
                 acc[c][e] = fmaf(k.sc[c], d, acc[c][e]);
             }
         }
 #pragma unroll
-        for (int T = 0; T < 2; ++T)
+        for (int ch = 0; ch < LACC; ++ch)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) dsum[T][e] = 0.0f;
+            for (int T = 0; T < 2; ++T)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dsum[ch][T][e] = 0.0f;
 #pragma unroll
         for (int e = 0; e < NE; ++e) xsum[e] = 0.0f;
     };
@@ -339,9 +351,11 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const LeanParams p) {
     const uint32_t off_even = (uint32_t)t * 128 + (((uint32_t)cg ^ (uint32_t)t) << 4);
     const uint32_t off_odd = (uint32_t)t * 128 + (((uint32_t)cg ^ (uint32_t)(t + 4)) << 4);
 
-    // one quad: iq is the quad within the slot (compile-time), i the quad within the warp
-    auto quad = [&](uint32_t slot_addr, int iq, int i) {
-        const uint4 hv = lds128_u32(slot_addr + 512 * iq + ((iq & 1) ? off_odd : off_even));
+    // one quad: iq = i4 + j is the quad within the slot (j < 4 compile-time, i4 a
+    // multiple of 4), i the quad within the warp
+    auto quad = [&](uint32_t slot_addr, int i4, int j, int i) {
+        const int iq = i4 + j;
+        const uint4 hv = lds128_u32(slot_addr + 512 * iq + ((j & 1) ? off_odd : off_even));
         uint32_t bx[EPS / 2];
         if constexpr (EPS >= 8) {
 #pragma unroll
@@ -371,7 +385,7 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const LeanParams p) {
                 a[1] = WB.pair(k.cc[2 * T + 1], 2 * h);
                 a[2] = WA.pair(k.cc[2 * T], 2 * h + 1);
                 a[3] = WB.pair(k.cc[2 * T + 1], 2 * h + 1);
-                mma_16816<BF>(dsum[T], a, bx[2 * h], bx[2 * h + 1]);
+                mma_16816<BF>(dsum[(j * MMAS + h) % LACC][T], a, bx[2 * h], bx[2 * h + 1]);
             }
         }
         if (--left == 0) {  // end of a group: fold, then the next group's constants
@@ -393,12 +407,16 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const LeanParams p) {
         const uint32_t slot_addr = ring0 + (uint32_t)slot * BOX_BYTES;
         const int i0 = b * BQ;
         if (i0 + BQ <= nq) {
+#pragma unroll 1
+            for (int i4 = 0; i4 < BQ; i4 += 4)
 #pragma unroll
-            for (int iq = 0; iq < BQ; ++iq) quad(slot_addr, iq, i0 + iq);
+                for (int j = 0; j < 4; ++j) quad(slot_addr, i4, j, i0 + i4 + j);
         } else {
+#pragma unroll 1
+            for (int i4 = 0; i4 < BQ; i4 += 4)
 #pragma unroll
-            for (int iq = 0; iq < BQ; ++iq)
-                if (i0 + iq < nq) quad(slot_addr, iq, i0 + iq);
+                for (int j = 0; j < 4; ++j)
+                    if (i0 + i4 + j < nq) quad(slot_addr, i4, j, i0 + i4 + j);
         }
         xaddr += QK * 2 * BQ;
         // every lane has read this slot: refill it with box b + S

@@ -30,6 +30,9 @@ wq_status launch_pack(const uint8_t* codes, int K, int N, int bits, uint32_t* w_
                       uint32_t* bad_count, cudaStream_t s);
 wq_status launch_unpack(const uint32_t* w_q, const uint32_t* w_lo, int K, int N, int bits,
                         uint8_t* codes, cudaStream_t s);
+wq_status launch_gptqmodel_convert(const uint32_t* qweight, const uint32_t* qzeros, int K, int N, int bits,
+                                   int G, uint32_t* w_q, uint32_t* w_lo, uint16_t* zeros, bool bf,
+                                   cudaStream_t s);
 wq_status launch_gemv(const Problem& p, cudaStream_t s);
 // GEMV with a small shared-memory footprint for 4- and 8-bit words and M <= 8
 // (wq_gemv_lean.cu); launch_gemv routes the shapes it takes there.
@@ -37,6 +40,9 @@ bool gemv_lean_takes(const Problem& p);
 wq_status launch_gemv_lean(const Problem& p, cudaStream_t s);
 wq_status launch_gemm(const Problem& p, cudaStream_t s);
 size_t gemm_workspace_bytes(int M, int K, int N, int bits, int G);
+wq_status launch_mse_search(const float* w, int rows, int cols, int group_size, int bits, int symmetric,
+                            int steps, int grid, float norm, int patience, float* scale, float* zero,
+                            int32_t* step, float* err, uint32_t* any_mask, cudaStream_t stream);
 
 // Device status words (one per kernel file): nonzero once a bounded wait ran out.
 // Reading synchronises the device; reset clears the word.

@@ -229,6 +229,68 @@ wq_status wq_gemm_noalloc(const uint16_t* x, const uint32_t* w_q, const uint32_t
                           unsigned flags, void* stream);
 
 /*
+ * The GPTQModel packed format ("GPTQModel-Compatible Triton Kernel" README,
+ * "API Reference": `gptqmodel_quantized_matmul(x, qweight, qzeros, scales,
+ * bits, group_size)`; "Quantization Format": 2-bit 16, 3-bit 10 (with
+ * padding), 4-bit 8, 8-bit 4 values per int32; "Dequantization Formula":
+ * scales * (quantized_weight - quantized_zero)) converted to this library's
+ * operands, so that wq_gemv / wq_gemm / wq_matmul compute that product.
+ * Readings of what the README leaves open: code k of a column sits in word
+ * k / V at bit bits * (k % V), lowest first (for 2, 4, 8 bits the K-major words
+ * of this library unchanged); 3-bit words use bits 0-29; qzeros hold the zero
+ * points of each group packed along N the same way, with no offset.
+ *   qweight  (ceil(K / V), N) int32 device array.
+ *   qzeros   (K / G, ceil(N / V)) int32 device array (G = K for group_size -1).
+ *   w_q      3-bit: (K / 16, N) output hi plane; 2, 4, 8 bits: NULL (pass qweight
+ *            itself to the products) or an output that receives a copy.
+ *   w_lo     3-bit: (K / 32, N) output lo plane; NULL otherwise.
+ *   zeros    (K / G, N) output, the zero points as binary16 (bfloat16 with
+ *            WQ_FLAG_BF16, the only flag taken).
+ * bits 2, 3, 4 or 8 (else WQ_ERR_UNSUPPORTED); K % 32 == 0 for 3 bits (the
+ * two-plane format), K % (32 / bits) otherwise; the group size divides K.
+ * Asynchronous on `stream`.
+ */
+wq_status wq_gptqmodel_convert(const uint32_t* qweight, const uint32_t* qzeros, int K, int N, int bits,
+                               int group_size, uint32_t* w_q, uint32_t* w_lo, uint16_t* zeros,
+                               unsigned flags, void* stream);
+
+/*
+ * MSE-observer search of per-group scales and zero points ("Benchmark for MSE
+ * observer grid search" page: `grid_search_eager`,
+ * `grid_search_eager_no_patience`, and the fake quantisation of
+ * `_fused_grid_search_kernel`), the step upstream of this library's product
+ * that chooses the s and z it consumes.
+ *   w          (rows, cols) fp32 device array, row-major, 4-byte aligned;
+ *              groups are group_size consecutive values of a row.
+ *   bits       1..8.  symmetric = 0: unsigned codes [0, 2^bits - 1] with the
+ *              affine rule -- the range widened to contain 0,
+ *              s = (hi - lo) / (2^bits - 1), z = clamp(-rint(lo / s)).
+ *              symmetric = 1: signed codes [-2^(bits-1), 2^(bits-1) - 1],
+ *              s = max(|lo|, |hi|) / ((2^bits - 1) / 2), z = 0 (stored in
+ *              this library's unsigned format as q + 2^(bits-1) with zero
+ *              point 2^(bits-1)).  A zero scale becomes 2^-23.
+ *   steps      candidates, 1..32: candidate i shrinks the group's [min, max]
+ *              by p_i = 1 - i / grid (the page evaluates int(maxshrink * grid)).
+ *   grid       >= 1.   norm: the error exponent, finite and > 0.
+ *   patience   0: every candidate is evaluated; else the search stops after
+ *              `patience` candidates in a row in which no group of the whole
+ *              tensor improved, as the page's eager search does.
+ *   scale, zero, err  (rows, cols / group_size) fp32 outputs: the winning
+ *              candidate's parameters and its error sum |w_hat - w|^norm.
+ *   step       (rows, cols / group_size) int32 output: the winning candidate.
+ *   workspace  4 bytes of device memory (any contents) when patience > 0, else
+ *              may be NULL; calls that may run at the same time must not share it.
+ * Every step up to w_hat is done in IEEE fp32 (correctly rounded division,
+ * round to nearest even), so a candidate's parameters are bit-exact; the error
+ * is summed in fp32.  Requires rows, cols >= 1, cols % group_size == 0, and
+ * 4-byte aligned arrays.  Asynchronous on `stream`.
+ */
+wq_status wq_mse_search(const float* w, int rows, int cols, int group_size, int bits, int symmetric,
+                        int steps, int grid, float norm, int patience, float* scale, float* zero,
+                        int32_t* step, float* err, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/*
  * Device-side status of the current device: WQ_OK, or WQ_ERR_TIMEOUT when a
  * kernel on this device gave up a bounded wait since the last reset (its
  * output is then incomplete).  Synchronises the device.  reset != 0 clears it.

@@ -168,3 +168,29 @@ def test_selftest_argument_checks(libwq):
     import torch
     if not torch.cuda.is_available():
         assert L.wq_selftest_wait_timeout(1_000_000, None) == 6   # reaches CUDA: no device here
+
+
+def test_mse_search_argument_checks(libwq):
+    """wq_mse_search rejects bad shapes, bit widths, candidate counts, norms and
+    pointers on the host, before any launch."""
+    L = libwq.lib()
+    f = ctypes.c_float
+
+    def call(w=P, rows=4, cols=64, G=16, bits=4, sym=0, steps=20, grid=100, norm=2.4, pat=0,
+             out=P, ws=None, ws_bytes=0):
+        return L.wq_mse_search(w, rows, cols, G, bits, sym, steps, grid, f(norm), pat, out, out, out, out, ws,
+                               ctypes.c_size_t(ws_bytes), None)
+    assert call(bits=0) == 2 and call(bits=9) == 2
+    assert call(rows=0) == 1 and call(cols=0) == 1 and call(G=0) == 1
+    assert call(cols=60, G=16) == 1                     # cols % group_size
+    assert call(sym=2) == 1
+    assert call(steps=0) == 1 and call(steps=33) == 1   # 1..32 candidates
+    assert call(grid=0) == 1 and call(pat=-1) == 1
+    assert call(norm=0.0) == 1 and call(norm=float("nan")) == 1 and call(norm=float("inf")) == 1
+    assert call(w=None) == 1 and call(out=None) == 1
+    assert call(pat=5) == 1                             # patience needs a 4-byte workspace
+    assert call(w=P + 2) == 3
+    import torch
+    if not torch.cuda.is_available():
+        assert call() == 6                              # valid: reaches CUDA, which has no device here
+        assert call(pat=5, ws=P, ws_bytes=4) == 6
