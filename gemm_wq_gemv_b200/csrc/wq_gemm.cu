@@ -69,15 +69,15 @@ struct GemmParams {
     uint32_t bar_off;    // offset of the barrier block from the aligned base
     uint4* ws;           // split-K slices: [tile][rank][32-token chunk][16-byte piece][128 columns]
     int late_wait;       // wait for the previous kernel only before writing the workspace / y
-    int xbulk;           // split-K exchange through bulk copies staged in the (then idle) stage ring
-    uint32_t recv_off;   // byte offset in the ring of the received slices (xbulk)
 };
 
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
 }
 
-template <int BITS, bool BF>
+// GW: every group covers whole 64-deep k blocks (G a multiple of 64, or G = K),
+// the common case, compiled without the per-row group logic of the others.
+template <int BITS, bool BF, bool GW>
 __global__ void __launch_bounds__(NWARPS * 32, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
             const __grid_constant__ CUtensorMap tm_lo, const __grid_constant__ CUtensorMap tm_s,
@@ -96,8 +96,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     uint64_t* full_a = full_tma + p.stages;
     uint64_t* empty = full_a + p.stages;
     uint64_t* accum = empty + p.stages;
-    uint64_t* recv_bar = accum + 1;  // the peers' slices have landed (bulk exchange)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_bar + 1);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5;
@@ -114,7 +113,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
             mbar_init(&empty[s], 1);
         }
         mbar_init(accum, 1);
-        mbar_init(recv_bar, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -158,7 +156,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
                 tma_load_2d(st + p.off_s, &tm_s, &full_tma[s], n0, grow);
                 tma_load_2d(st + p.off_z, &tm_z, &full_tma[s], n0, grow);
                 kg += BK;
-                if (p.gmode == 0) {         // a group spans whole k blocks: next row once kg reaches it
+                if (GW) {                   // a group spans whole k blocks: next row once kg reaches it
                     if (kg >= gnext) { ++grow; gnext += p.G; }
                 } else if (p.gmode == 1) {  // 64 / G rows per k block
                     grow += p.GPB;
@@ -239,7 +237,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
                 const uint8_t* st = base + (size_t)s * p.stage_bytes;
                 uint32_t c[NC], s2, zs2;
                 uint32_t a32[32];  // this thread's 64 k values (32 pairs) of the stage's A row
-                if (p.gmode == 0) {  // one group covers the whole k block
+                if constexpr (GW) {  // one group covers the whole k block
                     consts(st, 0, c, s2, zs2);
 #pragma unroll
                     for (int rw = 0; rw < RW; ++rw) word(st, rw, c, s2, zs2, a32 + rw * (EPS / 2));
@@ -307,90 +305,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     // threads of a warp write (and later read) 512 contiguous bytes per piece.
     constexpr size_t CHUNK_U4 = CHUNK_BYTES / 16;
     const size_t tile_slot = (size_t)(blockIdx.y * gridDim.x + blockIdx.x) * (size_t)p.CS;
-    if (split && p.xbulk) {
-        // The same exchange through the copy engines.  The stage ring is idle now
-        // (every MMA has completed): each CTA stages its non-owned chunks there in
-        // the workspace's slice layout, one thread writes them to the workspace
-        // with bulk copies, and after the cluster barrier the owners bring their
-        // peers' slices back into the ring with bulk copies and add them from
-        // shared memory.  A few copy operations keep many bytes in flight, where
-        // per-thread 16-byte stores and loads are limited by the requests each SM
-        // can have outstanding.
-        const uint32_t ring = smem_u32(base);
-        const int nown = (nchunks - rank + p.CS - 1) / p.CS;  // chunks j = rank (mod CS)
-        if (warp >= 2 && !*abort_flag) {
-            for (int j = 0, sidx = 0; j < nchunks; ++j) {
-                if (j % p.CS == rank) continue;
-                const int t = sidx++;  // staging slot of this chunk
-                if ((t & 1) != hf) continue;
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tm_row + 32 * j, v);
-                tmem_ld_wait();
-                const uint32_t dst = ring + (uint32_t)t * (uint32_t)CHUNK_BYTES + 16u * (uint32_t)nl;
-#pragma unroll
-                for (int pc = 0; pc < 8; ++pc)
-                    sts128_u32(dst + 2048u * pc, make_uint4(v[4 * pc], v[4 * pc + 1], v[4 * pc + 2], v[4 * pc + 3]));
-            }
-            fence_proxy_async_smem();  // the staged slices are visible to the copy engine
-        }
-        if (warp >= 2) named_barrier(1, 8 * 32);
-        if (warp == 2 && lane == 0 && !*abort_flag) {
-            uint4* mine = p.ws + (tile_slot + rank) * nchunks * CHUNK_U4;
-            for (int j = 0, t = 0; j < nchunks; ++j) {
-                if (j % p.CS == rank) continue;
-                bulk_store_s2g(mine + (size_t)j * CHUNK_U4, ring + (uint32_t)(t++) * (uint32_t)CHUNK_BYTES,
-                               (uint32_t)CHUNK_BYTES);
-            }
-            bulk_commit();
-            bulk_wait_all();      // the slices are written
-            fence_proxy_async();  // ... and ordered before the barrier's release
-        }
-        cluster_sync();  // release / acquire: every CTA's slices are in the workspace
-        if (warp == 2 && lane == 0 && !*abort_flag) {
-            fence_proxy_async();  // the bulk reads below follow the acquire
-            mbar_arrive_expect_tx(recv_bar, (uint32_t)((p.CS - 1) * nown) * (uint32_t)CHUNK_BYTES);
-            for (int src = 0, pi = 0; src < p.CS; ++src) {
-                if (src == rank) continue;
-                for (int o = 0; o < nown; ++o)
-                    bulk_load_g2s(ring + p.recv_off + (uint32_t)(pi * nown + o) * (uint32_t)CHUNK_BYTES,
-                                  p.ws + ((tile_slot + src) * nchunks + rank + o * p.CS) * CHUNK_U4,
-                                  (uint32_t)CHUNK_BYTES, recv_bar);
-                ++pi;
-            }
-        }
-        if (warp >= 2 && !*abort_flag) {
-            if (!mbar_wait_bounded(recv_bar, 0, WAIT_NS)) fail();
-            for (int j = rank + hf * p.CS; j < nchunks && !*abort_flag; j += 2 * p.CS) {
-                const int o = (j - rank) / p.CS;
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tm_row + 32 * j, v);
-                tmem_ld_wait();
-                float acc[32];
-#pragma unroll
-                for (int cc = 0; cc < 32; ++cc) acc[cc] = __uint_as_float(v[cc]);
-                for (int pi = 0; pi < p.CS - 1; ++pi) {
-                    const uint32_t src = ring + p.recv_off + (uint32_t)(pi * nown + o) * (uint32_t)CHUNK_BYTES +
-                                         16u * (uint32_t)nl;
-#pragma unroll
-                    for (int pc = 0; pc < 8; ++pc) {
-                        const uint4 u = lds128_u32(src + 2048u * pc);
-                        acc[4 * pc] += __uint_as_float(u.x);
-                        acc[4 * pc + 1] += __uint_as_float(u.y);
-                        acc[4 * pc + 2] += __uint_as_float(u.z);
-                        acc[4 * pc + 3] += __uint_as_float(u.w);
-                    }
-                }
-                if (ncol < p.N) {
-                    const float bv = p.bias ? T16::load(p.bias[ncol]) : 0.0f;
-#pragma unroll
-                    for (int cc = 0; cc < 32; ++cc) {
-                        const int m = m0 + 32 * j + cc;
-                        if (m < p.M) p.y[(size_t)m * p.N + ncol] = T16::store(acc[cc] + bv);
-                    }
-                }
-            }
-        }
-    } else {
     if (split && warp >= 2 && !*abort_flag) {
         uint4* mine = p.ws + (tile_slot + rank) * nchunks * CHUNK_U4;
         // this CTA's non-owned chunks, alternately to the two warps of the quadrant
@@ -442,7 +356,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
             }
         }
     }
-    }  // per-thread exchange
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -490,7 +403,6 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     constexpr int EPS = Fmt<BITS>::EPS;
     constexpr int RW = BK / EPS;
     constexpr int RL = (BITS == 3) ? BK / 32 : 0;
-    auto kern = gemm_kernel<BITS, BF>;
 
     GemmParams p{};
     p.y = pb.y;
@@ -509,6 +421,7 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     }
     p.g_shift = 0;
     while ((1 << (p.g_shift + 1)) <= pb.G && p.g_shift < 6) ++p.g_shift;
+    auto kern = p.gmode == 0 ? gemm_kernel<BITS, BF, true> : gemm_kernel<BITS, BF, false>;
 
     // token tiles of at most 256 (balanced), K split over a cluster where it pays
     const Tiling t = plan(pb.M, pb.K, pb.N, pb.ws ? pb.ws_bytes : 0);
@@ -542,17 +455,6 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     p.stages = stages;
     const size_t ring = (size_t)stages * p.stage_bytes;
     p.bar_off = (uint32_t)ring;
-    // Bulk split-K exchange when the staged and received slices fit in the ring:
-    // at most ceil(TN/32) - floor(TN/32 / CS) chunks sent, ceil(TN/32 / CS) x (CS - 1) received.
-    if (CS > 1) {
-        const int nch = TN / 32;
-        const size_t send = (size_t)(nch - nch / CS) * CHUNK_BYTES;
-        const size_t recv = (size_t)((nch + CS - 1) / CS) * (CS - 1) * CHUNK_BYTES;
-        if (send + recv <= ring) {
-            p.xbulk = 1;
-            p.recv_off = (uint32_t)send;
-        }
-    }
     // Enough shared memory that the CTAs resident on one SM never ask for more
     // than the SM's 512 tensor-memory columns together, so tcgen05.alloc never
     // waits on a CTA of another cluster: over 116 KB (one CTA per SM) when a CTA
@@ -578,7 +480,9 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
                         CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return WQ_ERR_CUDA;
 
-    static std::atomic<uint64_t> attr_ctx[MAX_DEVICES];  // context the smem limit was raised in
+    // context the smem limit was raised in, per kernel instantiation
+    static std::atomic<uint64_t> attr_ctx_gw[MAX_DEVICES], attr_ctx_any[MAX_DEVICES];
+    std::atomic<uint64_t>* attr_ctx = p.gmode == 0 ? attr_ctx_gw : attr_ctx_any;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return WQ_ERR_CUDA;
     if (const wq_status st = ensure_smem_attr((const void*)kern, (int)limit, attr_ctx, dev); st != WQ_OK) return st;

@@ -31,10 +31,6 @@ __device__ __forceinline__ uint4 lds128_u32(uint32_t a) {
     return r;
 }
 
-__device__ __forceinline__ void sts128_u32(uint32_t a, uint4 v) {
-    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
-}
-
 __device__ __forceinline__ uint2 lds64_u32(uint32_t a) {
     uint2 r;
     asm("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(a) : "memory");
@@ -255,34 +251,6 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const void* tmap, ui
         "[%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
         "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "l"(pol)
         : "memory");
-}
-
-// Untiled bulk copies (no tensor map): shared -> global, tracked by bulk groups,
-// and global -> shared, completing on an mbarrier.  Addresses and sizes are
-// 16-byte multiples.
-__device__ __forceinline__ void bulk_store_s2g(void* gdst, uint32_t ssrc, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-
-// Wait until every committed bulk group of this thread has completed (its writes performed).
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-__device__ __forceinline__ void bulk_load_g2s(uint32_t sdst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(sdst),
-        "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// Order this thread's async-proxy (bulk copy) accesses with its generic-proxy ones.
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async;" ::: "memory"); }
-
-// Barrier among `count` threads (a multiple of 32) on hardware barrier `id` (1..15).
-__device__ __forceinline__ void named_barrier(int id, int count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
