@@ -66,6 +66,7 @@ struct LeanParams {
     int QW;         // quads per warp (a multiple of the quads per box)
     int KS;         // CTAs per cluster along K (1: no cluster)
     int qpg;        // quads per group (a large number when one group spans K)
+    int qpg_shift;  // log2(qpg) when qpg is a power of two, else -1
     int BQ;         // quads per TMA box (R = 4 BQ word rows)
     int S;          // ring slots per warp (a power of two)
     int sz_rows;    // s (and z) rows loaded per CTA: sz_box x (number of boxes)
@@ -94,29 +95,24 @@ __device__ __forceinline__ uint4 ldg_x(const uint16_t* xr, int k0, int K) {
 }
 
 // Conversion constants of a lane's 4 columns for one group, from the group's z
-// values (uint2: columns 0-1 and 2-3 as 16-bit pairs), and whether any zero
-// point of the group is fractional (warp-wide).  fp16: two columns per fp16x2
-// instruction -- z is clamped to [-256, 256] and rounded to an integer by adding
-// 1536 (fp16 spacing 1 on [1024, 2048), ties to even as rint), and the
-// constants -(1024 + zi) and -(64 + zi) are differences of exact integers below
-// 2048.  bf16: per column.  The scales and fractional parts are read again when
-// the group ends (group_scales), so no register holds them meanwhile.
+// values (uint2: columns 0-1 and 2-3 as 16-bit pairs).  fp16: two columns per
+// fp16x2 instruction -- z is clamped to [-256, 256] and rounded to an integer by
+// adding 1536 (fp16 spacing 1 on [1024, 2048), ties to even as rint, the same
+// integer as zero_int), and the constants -(1024 + zi) and -(64 + zi) are
+// differences of exact integers below 2048.  bf16: per column.
 template <int BITS, bool BF>
 struct GroupConsts {
     static constexpr int NC = ncons<BITS, BF>();
     uint32_t cc[4][NC];
-    bool frac;
 
     __device__ __forceinline__ void make(uint2 zv) {
         using T16 = Dt<BF>;
-        bool f = false;
         if constexpr (!BF) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const uint32_t z2 = h ? zv.y : zv.x;
                 const uint32_t zc = hmin2_u32(hmax2_u32(z2, h2c(0xDC00u)), h2c(0x5C00u));  // [-256, 256]
                 const uint32_t r = hadd2_u32(zc, h2c(0x6600u));                            // 1536 + zi
-                f |= hsub2_u32(r, h2c(0x6600u)) != z2;
                 const uint32_t c0 = hsub2_u32(h2c(0x6000u), r);  // 512 - 1536 - zi = -(1024 + zi)
                 cc[2 * h][0] = prmt(c0, c0, 0x1010u);
                 cc[2 * h + 1][0] = prmt(c0, c0, 0x3232u);
@@ -132,34 +128,17 @@ struct GroupConsts {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const float zi = zero_int<BITS, BF>(zz[c]);
-                f |= zz[c] != zi;
 #pragma unroll
                 for (int ci = 0; ci < NC; ++ci) cc[c][ci] = pair_const<BITS, BF>(ci, zi);
             }
         }
-        frac = __any_sync(0xffffffffu, f);
     }
 };
 
-// Scales of a lane's 4 columns and, when the group has fractional zero points,
-// their fractional parts z - zi (zi as the conversion constants round it).
-template <int BITS, bool BF>
-__device__ __forceinline__ void group_scales(uint2 sv, uint2 zv, bool frac, float (&sc)[4], float (&zr)[4]) {
-    using T16 = Dt<BF>;
-    const float2 s01 = T16::pair(sv.x), s23 = T16::pair(sv.y);
-    sc[0] = s01.x; sc[1] = s01.y; sc[2] = s23.x; sc[3] = s23.y;
-    if (frac) {
-        const float2 z01 = T16::pair(zv.x), z23 = T16::pair(zv.y);
-        const float zz[4] = {z01.x, z01.y, z23.x, z23.y};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) zr[c] = zz[c] - zero_int<BITS, BF>(zz[c]);
-    } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) zr[c] = 0.0f;
-    }
-}
-
-template <int BITS, bool BF, int BQ, bool M1>
+// ALIGNED: one box holds each warp's whole range (QW == BQ quads, all inside K)
+// and groups start on the range's 4-quad blocks, so the main loop runs group by
+// group without per-quad bookkeeping.
+template <int BITS, bool BF, int BQ, bool M1, bool ALIGNED>
 __global__ void __launch_bounds__(LWK * 32, 3)
 gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
                  const __grid_constant__ CUtensorMap tm_z, const LeanParams p) {
@@ -185,7 +164,9 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
     const int cta_q0 = rank * LWK * p.QW;
     const int q_begin = cta_q0 + warp * p.QW;
     const int nq = max(0, min(p.Q, q_begin + p.QW) - q_begin);
-    const int g_cta0 = min(cta_q0, p.Q - 1) / p.qpg;  // first group of the CTA's K range
+    // group of quad q (a shift for the usual power-of-two quads per group)
+    auto gdiv = [&](int q) { return p.qpg_shift >= 0 ? (q >> p.qpg_shift) : q / p.qpg; };
+    const int g_cta0 = gdiv(min(cta_q0, p.Q - 1));  // first group of the CTA's K range
 
     // ---- (1) every load of the CTA, issued first: the warp's words (boxes of BQ
     // quads into a ring of S slots) and, by warp 0, the s and z rows
@@ -231,172 +212,205 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
     // quads of this warp whose 4 word rows all lie inside K (the rest: the ragged end)
     const int nq_full = max(0, min(p.Kw / 4, q_begin + p.QW) - q_begin);
 
-    // ---- (3) s and z: the group constants of the lane's 4 columns
+    // ---- (3) s and z.  Whether any zero point of the CTA's groups is
+    // fractional is settled once, from the z rows in shared memory, and the
+    // main loop is compiled for each case.
     bool ok_all = mbar_wait_bounded(bar_sz, 0, LWAIT_NS);
     if (!ok_all) atomicExch(&g_gemv_lean_status, 1u);
+    bool frac = false;
+    if (ok_all) {
+        const uint16_t* zt = reinterpret_cast<const uint16_t*>(smem + p.off_sz + z_off);
+        for (int e = threadIdx.x; e < p.sz_rows * LCOLS; e += LWK * 32) {
+            const float z = T16::load(zt[e]);
+            frac |= z != zero_int<BITS, BF>(z);
+        }
+    }
+    frac = __syncthreads_or(frac) != 0;
     ok_all = __all_sync(0xffffffffu, ok_all);
     const uint32_t sz_lane = sz_base + 2u * (uint32_t)(4 * cg);
-    GroupConsts<BITS, BF> k;
     auto sz_addr = [&](int gi) { return sz_lane + (LCOLS * 2u) * (uint32_t)(gi - g_cta0); };
+    GroupConsts<BITS, BF> k;
     auto consts = [&](int gi) { k.make(lds64_u32(sz_addr(gi) + z_off)); };
-    int gcur = q_begin / p.qpg;
+    int gcur = gdiv(q_begin);
     int left = p.qpg - (q_begin - gcur * p.qpg);  // quads left in the current group
     if (ok_all && nq > 0) consts(gcur);
-
-    // ---- (4) main loop
-    float acc[4][NE], dsum[2][4], xsum = 0.0f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int e = 0; e < NE; ++e) acc[c][e] = 0.0f;
-#pragma unroll
-    for (int T = 0; T < 2; ++T)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dsum[T][e] = 0.0f;
-    // fold the group's dot products into acc (scaled by s, fractional zero points applied)
-    auto fold = [&]() {
-        float X[NE];
-#pragma unroll
-        for (int e = 0; e < NE; ++e) X[e] = 0.0f;
-        float sc[4], zr[4];
-        const uint32_t a = sz_addr(gcur);
-        group_scales<BITS, BF>(lds64_u32(a), k.frac ? lds64_u32(a + z_off) : make_uint2(0u, 0u), k.frac, sc, zr);
-        if (k.frac) {  // warp-uniform: the x sum of token 2 t + e over the group's quads of this warp
-            float tot = xsum + __shfl_xor_sync(0xffffffffu, xsum, 1);
-            tot += __shfl_xor_sync(0xffffffffu, tot, 2);
-#pragma unroll
-            for (int e = 0; e < NE; ++e) X[e] = __shfl_sync(0xffffffffu, tot, M1 ? 0 : 4 * (2 * t + e));
-        }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int T = c >> 1, half = c & 1;
-#pragma unroll
-            for (int e = 0; e < NE; ++e) {
-                float d = dsum[T][2 * half + e];
-                if (k.frac) d = fmaf(-zr[c], X[e], d);
-                acc[c][e] = fmaf(sc[c], d, acc[c][e]);
-            }
-        }
-#pragma unroll
-        for (int T = 0; T < 2; ++T)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dsum[T][e] = 0.0f;
-        xsum = 0.0f;
-    };
 
     // Per-lane offsets of this lane's 16-byte vector inside a slot: quad iq,
     // word row R = 4 iq + t, 16-byte chunk cg swizzled with (R & 7), whose
     // value only depends on the parity of iq.
     const uint32_t off_even = (uint32_t)t * 128 + (((uint32_t)cg ^ (uint32_t)t) << 4);
     const uint32_t off_odd = (uint32_t)t * 128 + (((uint32_t)cg ^ (uint32_t)(t + 4)) << 4);
+    // this lane's x values of quad i of the warp's range (all of its rows inside K)
+    auto ldx = [&](int i) {
+        if constexpr (EPS == 8) {  // 4 word rows = 32 values on per quad
+            return __ldg(reinterpret_cast<const uint4*>(xr + kx0) + 4 * i);
+        } else {                   // 16 values on per quad
+            const uint2 v = __ldg(reinterpret_cast<const uint2*>(xr + kx0) + 4 * i);
+            return make_uint4(v.x, v.y, 0u, 0u);
+        }
+    };
 
-    // One quad: iq is the quad within the slot (its parity is j's), i the quad
-    // within the warp.  Its x values are read here, from global memory; FRAC
-    // (warp-uniform) adds this lane's row sum of x to xsum.
-    // The words hv (this lane's 16 bytes of the quad) and x values xa of one quad.
-    auto quad = [&](const uint4& hv, const uint4& xa, auto frac_tag) {
+    // ---- (4) main loop, FRAC: the CTA has fractional zero points
+    float acc[4][NE];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < NE; ++e) acc[c][e] = 0.0f;
+    auto main_loop = [&](auto frac_tag) {
         constexpr bool FRAC = decltype(frac_tag)::value;
-        uint32_t bx[EPS / 2];
-        if constexpr (EPS == 8) {  // pairs (0, 4), (1, 5), (2, 6), (3, 7) of the row's 8 values
-            bx[0] = prmt(xa.x, xa.z, 0x5410u);
-            bx[1] = prmt(xa.x, xa.z, 0x7632u);
-            bx[2] = prmt(xa.y, xa.w, 0x5410u);
-            bx[3] = prmt(xa.y, xa.w, 0x7632u);
-        } else {                   // pairs (0, 2), (1, 3) of the row's 4 values
-            bx[0] = prmt(xa.x, xa.y, 0x5410u);
-            bx[1] = prmt(xa.x, xa.y, 0x7632u);
-        }
-        if constexpr (FRAC) {
-            const uint32_t xv[4] = {xa.x, xa.y, xa.z, xa.w};
+        float dsum[2][4], xsum = 0.0f;
 #pragma unroll
-            for (int u = 0; u < EPS / 2; ++u) {
-                const float2 f = T16::pair(xv[u]);
-                xsum += f.x + f.y;
+        for (int T = 0; T < 2; ++T)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dsum[T][e] = 0.0f;
+        // fold the group's dot products into acc (scaled by s, fractional zero points applied)
+        auto fold = [&]() {
+            const uint32_t a = sz_addr(gcur);
+            const uint2 sv = lds64_u32(a);
+            const float2 s01 = T16::pair(sv.x), s23 = T16::pair(sv.y);
+            const float sc[4] = {s01.x, s01.y, s23.x, s23.y};
+            float zr[4] = {0.0f, 0.0f, 0.0f, 0.0f}, X[NE];
+#pragma unroll
+            for (int e = 0; e < NE; ++e) X[e] = 0.0f;
+            if constexpr (FRAC) {
+                const uint2 zv = lds64_u32(a + z_off);
+                const float2 z01 = T16::pair(zv.x), z23 = T16::pair(zv.y);
+                const float zz[4] = {z01.x, z01.y, z23.x, z23.y};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) zr[c] = zz[c] - zero_int<BITS, BF>(zz[c]);
+                // the x sum of token 2 t + e over the group's quads of this warp
+                float tot = xsum + __shfl_xor_sync(0xffffffffu, xsum, 1);
+                tot += __shfl_xor_sync(0xffffffffu, tot, 2);
+#pragma unroll
+                for (int e = 0; e < NE; ++e) X[e] = __shfl_sync(0xffffffffu, tot, M1 ? 0 : 4 * (2 * t + e));
             }
-        }
-        const uint32_t wv[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
-        for (int T = 0; T < 2; ++T) {
-            Word<BITS, BF> WA, WB;
-            WA.prep(wv[2 * T], 0u, 0u);
-            WB.prep(wv[2 * T + 1], 0u, 0u);
+            for (int c = 0; c < 4; ++c) {
+                const int T = c >> 1, half = c & 1;
 #pragma unroll
-            for (int h = 0; h < MMAS; ++h) {
-                uint32_t a[4];
-                a[0] = WA.pair(k.cc[2 * T], 2 * h);
-                a[1] = WB.pair(k.cc[2 * T + 1], 2 * h);
-                a[2] = WA.pair(k.cc[2 * T], 2 * h + 1);
-                a[3] = WB.pair(k.cc[2 * T + 1], 2 * h + 1);
-                mma_16816<BF>(dsum[T], a, bx[2 * h], bx[2 * h + 1]);
+                for (int e = 0; e < NE; ++e) {
+                    float d = dsum[T][2 * half + e];
+                    if constexpr (FRAC) d = fmaf(-zr[c], X[e], d);
+                    acc[c][e] = fmaf(sc[c], d, acc[c][e]);
+                }
             }
-        }
-    };
-    // end of a group: fold, then the next group's constants
-    auto group_end = [&](int i) {
-        fold();
-        left = p.qpg;
-        ++gcur;
-        if (i + 1 < nq) consts(gcur);
-    };
-
-    for (int b = 0; b < nbox && ok_all; ++b) {
-        const int slot = b & (S - 1);
-        const bool good = mbar_wait_bounded(&bar[slot], (uint32_t)((b / S) & 1), LWAIT_NS);
-        if (!good) atomicExch(&g_gemv_lean_status, 1u);
-        if (!__all_sync(0xffffffffu, good)) {  // give up this warp's range
-            ok_all = false;
-            break;
-        }
-        const uint32_t slot_addr = ring0 + (uint32_t)slot * BOX_BYTES;
-        const int i0 = b * BQ;
-#pragma unroll 1
-        for (int i4 = 0; i4 < BQ && i0 + i4 < nq; i4 += 4) {
-            const int i = i0 + i4;
-            // this lane's 16-byte vectors of quads i4 .. i4 + 3 of the slot: word rows
-            // 4 iq + t, the swizzled chunk alternating with the parity of iq
+#pragma unroll
+            for (int T = 0; T < 2; ++T)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dsum[T][e] = 0.0f;
+            xsum = 0.0f;
+        };
+        // one quad: the words hv (this lane's 16 bytes) and its x values xa
+        auto quad = [&](const uint4& hv, const uint4& xa) {
+            uint32_t bx[EPS / 2];
+            if constexpr (EPS == 8) {  // pairs (0, 4), (1, 5), (2, 6), (3, 7) of the row's 8 values
+                bx[0] = prmt(xa.x, xa.z, 0x5410u);
+                bx[1] = prmt(xa.x, xa.z, 0x7632u);
+                bx[2] = prmt(xa.y, xa.w, 0x5410u);
+                bx[3] = prmt(xa.y, xa.w, 0x7632u);
+            } else {                   // pairs (0, 2), (1, 3) of the row's 4 values
+                bx[0] = prmt(xa.x, xa.y, 0x5410u);
+                bx[1] = prmt(xa.x, xa.y, 0x7632u);
+            }
+            if constexpr (FRAC) {  // this lane's row sum of x (fp32)
+                const uint32_t xv[4] = {xa.x, xa.y, xa.z, xa.w};
+#pragma unroll
+                for (int u = 0; u < EPS / 2; ++u) {
+                    const float2 f = T16::pair(xv[u]);
+                    xsum += f.x + f.y;
+                }
+            }
+            const uint32_t wv[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+            for (int T = 0; T < 2; ++T) {
+                Word<BITS, BF> WA, WB;
+                WA.prep(wv[2 * T], 0u, 0u);
+                WB.prep(wv[2 * T + 1], 0u, 0u);
+#pragma unroll
+                for (int h = 0; h < MMAS; ++h) {
+                    uint32_t a[4];
+                    a[0] = WA.pair(k.cc[2 * T], 2 * h);
+                    a[1] = WB.pair(k.cc[2 * T + 1], 2 * h);
+                    a[2] = WA.pair(k.cc[2 * T], 2 * h + 1);
+                    a[3] = WB.pair(k.cc[2 * T + 1], 2 * h + 1);
+                    mma_16816<BF>(dsum[T], a, bx[2 * h], bx[2 * h + 1]);
+                }
+            }
+        };
+        // the four quads i4 .. i4 + 3 of a slot, quads i .. i + 3 of the warp
+        auto block = [&](uint32_t slot_addr, int i4, int i) {
             const uint32_t wblk = slot_addr + 512u * (uint32_t)i4;
-            if (i + 4 <= nq_full && left >= 4) {  // four whole quads inside one group: straight-line code
-                auto ldw = [&](int j) { return lds128_u32(wblk + 512u * j + ((j & 1) ? off_odd : off_even)); };
-                auto ldx = [&](int j) {
-                    if constexpr (EPS == 8) {  // 4 word rows = 32 values on per quad
-                        return __ldg(reinterpret_cast<const uint4*>(xr + kx0) + 4 * (i + j));
-                    } else {                   // 16 values on per quad
-                        const uint2 v = __ldg(reinterpret_cast<const uint2*>(xr + kx0) + 4 * (i + j));
-                        return make_uint4(v.x, v.y, 0u, 0u);
-                    }
-                };
-                if (k.frac) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) quad(ldw(j), ldx(j), std::true_type{});
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) quad(ldw(j), ldx(j), std::false_type{});
+            for (int j = 0; j < 4; ++j) quad(lds128_u32(wblk + 512u * j + ((j & 1) ? off_odd : off_even)), ldx(i + j));
+        };
+
+        if constexpr (ALIGNED) {
+            if (ok_all && nq > 0) {
+                const bool good = mbar_wait_bounded(&bar[0], 0u, LWAIT_NS);
+                if (!good) atomicExch(&g_gemv_lean_status, 1u);
+                ok_all = __all_sync(0xffffffffu, good);
+            }
+            if (!ok_all || nq == 0) return;
+            const int seg = min(p.qpg, BQ);  // quads per group, or the whole range inside one group
+#pragma unroll 1
+            for (int q0 = 0; q0 < BQ; q0 += seg) {
+                if (q0 > 0) consts(gcur);
+#pragma unroll 1
+                for (int i = q0; i < q0 + seg; i += 4) block(ring0, i, i);
+                fold();
+                ++gcur;
+            }
+        } else {
+            // end of a group: fold, then the next group's constants
+            auto group_end = [&](int i) {
+                fold();
+                left = p.qpg;
+                ++gcur;
+                if (i + 1 < nq) consts(gcur);
+            };
+            for (int b = 0; b < nbox && ok_all; ++b) {
+                const int slot = b & (S - 1);
+                const bool good = mbar_wait_bounded(&bar[slot], (uint32_t)((b / S) & 1), LWAIT_NS);
+                if (!good) atomicExch(&g_gemv_lean_status, 1u);
+                if (!__all_sync(0xffffffffu, good)) {  // give up this warp's range
+                    ok_all = false;
+                    break;
                 }
-                left -= 4;
-                if (left == 0) group_end(i + 3);
-            } else {  // ragged end of the range, or groups shorter than four quads
+                const uint32_t slot_addr = ring0 + (uint32_t)slot * BOX_BYTES;
+                const int i0 = b * BQ;
+#pragma unroll 1
+                for (int i4 = 0; i4 < BQ && i0 + i4 < nq; i4 += 4) {
+                    const int i = i0 + i4;
+                    if (i + 4 <= nq_full && left >= 4) {  // four whole quads inside one group
+                        block(slot_addr, i4, i);
+                        left -= 4;
+                        if (left == 0) group_end(i + 3);
+                    } else {  // ragged end of the range, or groups shorter than four quads
+                        const uint32_t wblk = slot_addr + 512u * (uint32_t)i4;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    if (i + j < nq) {
-                        const uint4 hv = lds128_u32(wblk + 512u * j + ((j & 1) ? off_odd : off_even));
-                        const uint4 xa = ldg_x<EPS>(xr, kx0 + 4 * EPS * (i + j), p.K);
-                        if (k.frac)
-                            quad(hv, xa, std::true_type{});
-                        else
-                            quad(hv, xa, std::false_type{});
-                        if (--left == 0) group_end(i + j);
+                        for (int j = 0; j < 4; ++j) {
+                            if (i + j < nq) {
+                                quad(lds128_u32(wblk + 512u * j + ((j & 1) ? off_odd : off_even)),
+                                     ldg_x<EPS>(xr, kx0 + 4 * EPS * (i + j), p.K));
+                                if (--left == 0) group_end(i + j);
+                            }
+                        }
                     }
+                }
+                // every lane has read this slot: refill it with box b + S
+                __syncwarp();
+                if (lane == 0 && b + S < nbox) {
+                    fence_proxy_async_smem();
+                    issue(b + S);
                 }
             }
+            if (ok_all && nq > 0 && left != p.qpg) fold();  // the warp's range ended inside a group
         }
-        // every lane has read this slot: refill it with box b + S
-        __syncwarp();
-        if (lane == 0 && b + S < nbox) {
-            fence_proxy_async_smem();
-            issue(b + S);
-        }
-    }
-    if (ok_all && nq > 0 && left != p.qpg) fold();  // the warp's range ended inside a group
+    };
+    if (frac)
+        main_loop(std::true_type{});
+    else
+        main_loop(std::false_type{});
 
     // ---- (5) reduce over the warps of the CTA (and the CTAs of the cluster), write y.
     // Each warp's partials go to the first slot of its own ring, which it has consumed.
@@ -464,10 +478,10 @@ size_t lean_layout(LeanParams& p) {
     return off + 1024;  // slack for aligning the base to 1024 bytes
 }
 
-template <int BITS, bool BF, int BQ, bool M1>
+template <int BITS, bool BF, int BQ, bool M1, bool ALIGNED>
 wq_status launch_lean(const CUtensorMap& mw, const CUtensorMap& ms, const CUtensorMap& mz, const LeanParams& p,
                       size_t smem, const Problem& pb, cudaStream_t stream) {
-    auto kern = gemv_lean_kernel<BITS, BF, BQ, M1>;
+    auto kern = gemv_lean_kernel<BITS, BF, BQ, M1, ALIGNED>;
     static std::atomic<uint64_t> attr_ctx[MAX_DEVICES];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return WQ_ERR_CUDA;
@@ -507,6 +521,9 @@ wq_status run_lean(const Problem& pb, cudaStream_t stream) {
     p.Kw = pb.K / EPS;
     p.Q = (p.Kw + 3) / 4;
     p.qpg = (pb.G == pb.K) ? (1 << 29) : pb.G / QK;
+    p.qpg_shift = -1;
+    for (int sh = 0; sh < 30; ++sh)
+        if (p.qpg == (1 << sh)) p.qpg_shift = sh;
     const int n_groups = (pb.K + pb.G - 1) / pb.G;
     const int colblocks = (pb.N + LCOLS - 1) / LCOLS;
     const int sms = sm_count();
@@ -554,12 +571,22 @@ wq_status run_lean(const Problem& pb, cudaStream_t stream) {
     ok = ok && make_map(&mz, CU_TENSOR_MAP_DATA_TYPE_UINT16, pb.zeros, pb.N, n_groups, (uint64_t)pb.N * 2, LCOLS,
                         p.sz_box, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return WQ_ERR_CUDA;
+    // ALIGNED: one box per warp covering its QW quads, every warp of every rank
+    // full and inside K, and groups starting on 4-quad blocks of the ranges
+    const bool aligned = p.S == 1 && p.QW == BQ && p.Q == KS * LWK * p.QW && p.Kw == 4 * p.Q &&
+                         ((p.qpg <= p.QW && p.QW % p.qpg == 0 && p.qpg % 4 == 0) ||
+                          (p.qpg > p.QW && (p.qpg % p.QW == 0 || p.qpg >= p.Q)));
     const bool m1 = pb.M == 1;
-    if (BQ == 16)
-        return m1 ? launch_lean<BITS, BF, 16, true>(mw, ms, mz, p, smem, pb, stream)
-                  : launch_lean<BITS, BF, 16, false>(mw, ms, mz, p, smem, pb, stream);
-    return m1 ? launch_lean<BITS, BF, 8, true>(mw, ms, mz, p, smem, pb, stream)
-              : launch_lean<BITS, BF, 8, false>(mw, ms, mz, p, smem, pb, stream);
+    auto go = [&](auto bq, auto a) {
+        constexpr int B = decltype(bq)::value;
+        constexpr bool A = decltype(a)::value;
+        return m1 ? launch_lean<BITS, BF, B, true, A>(mw, ms, mz, p, smem, pb, stream)
+                  : launch_lean<BITS, BF, B, false, A>(mw, ms, mz, p, smem, pb, stream);
+    };
+    using I16 = std::integral_constant<int, 16>;
+    using I8 = std::integral_constant<int, 8>;
+    if (BQ == 16) return aligned ? go(I16{}, std::true_type{}) : go(I16{}, std::false_type{});
+    return aligned ? go(I8{}, std::true_type{}) : go(I8{}, std::false_type{});
 }
 
 }  // namespace

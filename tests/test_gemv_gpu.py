@@ -239,3 +239,56 @@ def test_rejected_calls(cuda, libwq):
     with pytest.raises(ValueError, match="out"):
         libwq.gemv(d["x"], w_q, None, d["scales"], d["zeros"], 4, 128,
                    out=torch.empty((1, 128), dtype=torch.float16, device=cuda))
+
+
+# Shapes whose plan gives every warp one box covering its whole range, with all
+# groups starting on 4-quad blocks (the group-by-group main loop of the 4/8-bit
+# kernel): 4-bit K = 16384 and 8-bit K = 8192 over N = 64 split K over a cluster
+# of 8 CTAs, 8 quads per warp; 4096 x 4096 takes one CTA per column block, 16
+# quads per warp (G = 256: two 4-quad blocks per group).  G = -1 is one group
+# across the range.
+ALIGNED = [(3, 16384, 64, 4, 128), (1, 16384, 64, 4, -1), (2, 8192, 64, 8, 128), (1, 4096, 4096, 4, 256)]
+
+
+@pytest.mark.parametrize("M,K,N,bits,G", ALIGNED)
+def test_aligned_plan_fractional_zero_points(cuda, libwq, orc, M, K, N, bits, G):
+    import torch
+    case = wq_inputs.custom(M, K, N, bits, G, seed=K + N + bits)
+    rng = np.random.default_rng(K + bits)
+    case.zeros = rng.uniform(-0.5, (1 << bits) - 0.5, size=case.zeros.shape).astype(np.float16)
+    d = to_dev(case, cuda)
+    d["zeros"] = torch.from_numpy(case.zeros).to(cuda)
+    y = run_gemv(libwq, d, bits, G)
+    y_ref, b = oracle_product(orc, case)
+    check_product(y, y_ref, b, f"aligned plan, fractional z, {(M, K, N, bits, G)}")
+
+
+@pytest.mark.parametrize("M,K,N,bits,G", ALIGNED)
+def test_aligned_plan_q_equals_z_gives_zero(cuda, libwq, M, K, N, bits, G):
+    import torch
+    case = wq_inputs.custom(M, K, N, bits, G, seed=11)
+    Gr = K if G == -1 else G
+    zq = np.random.default_rng(13).integers(0, 1 << bits, size=(K // Gr, N))
+    d = to_dev(case, cuda)
+    d["codes"] = torch.from_numpy(np.repeat(zq, Gr, axis=0).astype(np.uint8)).to(cuda)
+    d["zeros"] = torch.from_numpy(zq.astype(np.float16)).to(cuda)
+    y = run_gemv(libwq, d, bits, G)
+    assert np.all(y.astype(np.float64) == 0.0)
+
+
+@pytest.mark.parametrize("M,K,N,bits,G", ALIGNED)
+def test_aligned_plan_one_hot_rows_are_exact(cuda, libwq, M, K, N, bits, G):
+    import torch
+    Mh = 8
+    case = wq_inputs.custom(Mh, K, N, bits, G, seed=17)
+    ks = np.random.default_rng(K).choice(K, Mh, replace=False)
+    x = np.zeros((Mh, K), np.float16)
+    x[np.arange(Mh), ks] = 1.0
+    d = to_dev(case, cuda)
+    d["x"] = torch.from_numpy(x).to(cuda)
+    y = run_gemv(libwq, d, bits, G)
+    Gr = K if G == -1 else G
+    q = case.codes.astype(np.float64)
+    g = ks // Gr
+    w = (q[ks] - case.zeros[g].astype(np.float64)) * case.scales[g].astype(np.float64)
+    assert np.array_equal(y, w.astype(np.float16))
