@@ -41,6 +41,9 @@ import wq_inputs  # noqa: E402
 
 HEADLINE = "decode_gemv_m1"
 GEMM_WL = "prefill_gemm"
+# the kernels those two launch, as ncu names them (spaces as underscores)
+HEADLINE_KERNEL = "gemv_lean_kernel<4,_0,_16,_1,_1>"
+GEMM_KERNEL = "gemm_kernel<4,_0,_1>"
 METRIC = "packed-int GEMV HBM GB/s and % of peak at M=1; wq_gemm TFLOPS at M=512"
 FALLBACK_HBM, FALLBACK_TF = 6650.0, 1590.0
 # Nominal B200 figures, reported beside the measured ones: HBM3e ~8 TB/s,
@@ -476,7 +479,7 @@ def main(argv=None):
     value = job_rate(bytes_step, args.steps, world, el) / 1e9
     per_launch_s = el / (args.steps * L)
     achieved = algo_bytes(wl) / per_launch_s / 1e9
-    traffic = ncu_traffic("gemv_kernel<4,_1,_0>", HEADLINE)
+    traffic = ncu_traffic(HEADLINE_KERNEL, HEADLINE)
 
     # ---- the same stack as a dependency chain (x of each product = y of the previous)
     cg, cs = capture(torch, lambda: stack.run_chain(wq))
@@ -546,7 +549,7 @@ def main(argv=None):
     gel = max_over_ranks(time_graph(torch, gg, gs, gsteps, args.warmup, barrier))
     g_launch_s = gel / (gsteps * GL)
     g_tflops = algo_flops(gwl) / g_launch_s / 1e12
-    g_traffic = ncu_traffic("gemm_kernel<4,_0>", GEMM_WL)
+    g_traffic = ncu_traffic(GEMM_KERNEL, GEMM_WL)
     del gstack, gg
 
     # ---- context: the same kernel on a large product (no split-K, many k blocks),

@@ -74,6 +74,8 @@ struct LeanParams {
     uint32_t off_sz;   // s rows (from the 1024-aligned base), then z rows at + sz_stride
     uint32_t sz_stride;  // sz_rows * 64 bytes rounded up to 128 (a TMA destination)
     uint32_t off_part, off_bar;
+    uint32_t off_x;    // XS: the CTA's x slice, one row of xs_stride bytes per token
+    uint32_t xs_stride;
     int late_wait;  // wait for the previous kernel only before writing y
 };
 
@@ -138,7 +140,11 @@ struct GroupConsts {
 // ALIGNED: one box holds each warp's whole range (QW == BQ quads, all inside K)
 // and groups start on the range's 4-quad blocks, so the main loop runs group by
 // group without per-quad bookkeeping.
-template <int BITS, bool BF, int BQ, bool M1, bool ALIGNED>
+// XS: x is written by the previous kernel on the stream.  Every load that does
+// not depend on it is issued and waited for first; after the grid dependency
+// wait the CTA copies its slice of x into shared memory in one round trip, and
+// the quads read it from there.
+template <int BITS, bool BF, int BQ, bool M1, bool ALIGNED, bool XS>
 __global__ void __launch_bounds__(LWK * 32, 3)
 gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
                  const __grid_constant__ CUtensorMap tm_z, const LeanParams p) {
@@ -203,7 +209,7 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
     // the next kernel on the stream may start now (it waits for this grid
     // before it touches anything this one writes)
     grid_launch_dependents();
-    if (!p.late_wait) grid_dependency_wait();  // x may be the previous kernel's output
+    if (!XS && !p.late_wait) grid_dependency_wait();  // x may be the previous kernel's output
 
     // ---- (2) this lane's x: token g (duplicates beyond M are harmless), word
     // row 4 i + t of the warp's quad i
@@ -217,21 +223,28 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
     // main loop is compiled for each case.
     bool ok_all = mbar_wait_bounded(bar_sz, 0, LWAIT_NS);
     if (!ok_all) atomicExch(&g_gemv_lean_status, 1u);
+    ok_all = __all_sync(0xffffffffu, ok_all);
+    const uint32_t sz_lane = sz_base + 2u * (uint32_t)(4 * cg);
+    auto sz_addr = [&](int gi) { return sz_lane + (LCOLS * 2u) * (uint32_t)(gi - g_cta0); };
+    int gcur = gdiv(q_begin);
+    // whether any zero point of the warp's groups is fractional (a warp vote)
     bool frac = false;
-    if (ok_all) {
+    if (ok_all && nq > 0) {
+        const int g_last = gdiv(q_begin + nq - 1);
         const uint16_t* zt = reinterpret_cast<const uint16_t*>(smem + p.off_sz + z_off);
-        for (int e = threadIdx.x; e < p.sz_rows * LCOLS; e += LWK * 32) {
+        for (int e = (gcur - g_cta0) * LCOLS + lane; e < (g_last - g_cta0 + 1) * LCOLS; e += 32) {
             const float z = T16::load(zt[e]);
             frac |= z != zero_int<BITS, BF>(z);
         }
     }
-    frac = __syncthreads_or(frac) != 0;
-    ok_all = __all_sync(0xffffffffu, ok_all);
-    const uint32_t sz_lane = sz_base + 2u * (uint32_t)(4 * cg);
-    auto sz_addr = [&](int gi) { return sz_lane + (LCOLS * 2u) * (uint32_t)(gi - g_cta0); };
+    frac = __any_sync(0xffffffffu, frac);
     GroupConsts<BITS, BF> k;
-    auto consts = [&](int gi) { k.make(lds64_u32(sz_addr(gi) + z_off)); };
-    int gcur = gdiv(q_begin);
+    uint2 sv = make_uint2(0u, 0u);  // the current group's s values of the lane's 4 columns
+    auto consts = [&](int gi) {
+        const uint32_t a = sz_addr(gi);
+        sv = lds64_u32(a);
+        k.make(lds64_u32(a + z_off));
+    };
     int left = p.qpg - (q_begin - gcur * p.qpg);  // quads left in the current group
     if (ok_all && nq > 0) consts(gcur);
 
@@ -240,11 +253,32 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
     // value only depends on the parity of iq.
     const uint32_t off_even = (uint32_t)t * 128 + (((uint32_t)cg ^ (uint32_t)t) << 4);
     const uint32_t off_odd = (uint32_t)t * 128 + (((uint32_t)cg ^ (uint32_t)(t + 4)) << 4);
+    // XS: the weights, s and z are in flight or landed; now wait for the previous
+    // kernel and copy the CTA's x slice (zeros past K) into shared memory
+    const int kc0 = cta_q0 * 4 * EPS;  // first k of the CTA's range
+    if constexpr (XS) {
+        grid_dependency_wait();
+        const int per_tok = LWK * p.QW * 4 * EPS / 8;  // 16-byte chunks of one token's slice
+        for (int c = threadIdx.x; c < p.M * per_tok; c += LWK * 32) {
+            const int m = c / per_tok, o = c - m * per_tok;
+            const int kk = kc0 + 8 * o;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (kk < p.K) v = *reinterpret_cast<const uint4*>(p.x + (size_t)m * p.K + kk);  // K % 8 == 0
+            *reinterpret_cast<uint4*>(smem + p.off_x + (size_t)m * p.xs_stride + 16 * o) = v;
+        }
+        __syncthreads();
+    }
+    const uint32_t xs_lane = smem_u32(smem + p.off_x) + (uint32_t)(M1 ? 0 : min(g, p.M - 1)) * p.xs_stride +
+                             2u * (uint32_t)(kx0 - kc0);
     // this lane's x values of quad i of the warp's range (all of its rows inside K)
     auto ldx = [&](int i) {
-        if constexpr (EPS == 8) {  // 4 word rows = 32 values on per quad
+        if constexpr (XS) {
+            if constexpr (EPS == 8) return lds128_u32(xs_lane + 64u * i);
+            const uint2 v = lds64_u32(xs_lane + 32u * i);
+            return make_uint4(v.x, v.y, 0u, 0u);
+        } else if constexpr (EPS == 8) {  // 4 word rows = 32 values on per quad
             return __ldg(reinterpret_cast<const uint4*>(xr + kx0) + 4 * i);
-        } else {                   // 16 values on per quad
+        } else {                          // 16 values on per quad
             const uint2 v = __ldg(reinterpret_cast<const uint2*>(xr + kx0) + 4 * i);
             return make_uint4(v.x, v.y, 0u, 0u);
         }
@@ -265,15 +299,13 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
             for (int e = 0; e < 4; ++e) dsum[T][e] = 0.0f;
         // fold the group's dot products into acc (scaled by s, fractional zero points applied)
         auto fold = [&]() {
-            const uint32_t a = sz_addr(gcur);
-            const uint2 sv = lds64_u32(a);
             const float2 s01 = T16::pair(sv.x), s23 = T16::pair(sv.y);
             const float sc[4] = {s01.x, s01.y, s23.x, s23.y};
             float zr[4] = {0.0f, 0.0f, 0.0f, 0.0f}, X[NE];
 #pragma unroll
             for (int e = 0; e < NE; ++e) X[e] = 0.0f;
             if constexpr (FRAC) {
-                const uint2 zv = lds64_u32(a + z_off);
+                const uint2 zv = lds64_u32(sz_addr(gcur) + z_off);
                 const float2 z01 = T16::pair(zv.x), z23 = T16::pair(zv.y);
                 const float zz[4] = {z01.x, z01.y, z23.x, z23.y};
 #pragma unroll
@@ -391,7 +423,7 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
                         for (int j = 0; j < 4; ++j) {
                             if (i + j < nq) {
                                 quad(lds128_u32(wblk + 512u * j + ((j & 1) ? off_odd : off_even)),
-                                     ldg_x<EPS>(xr, kx0 + 4 * EPS * (i + j), p.K));
+                                     XS ? ldx(i + j) : ldg_x<EPS>(xr, kx0 + 4 * EPS * (i + j), p.K));
                                 if (--left == 0) group_end(i + j);
                             }
                         }
@@ -457,14 +489,17 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
         }
         cluster_sync();  // peers keep their shared memory until every read is done
     } else {
-        if (p.late_wait) grid_dependency_wait();
-        for (int i = threadIdx.x; i < nout; i += LWK * 32) store(i, warp_sum(i));
+        for (int i = threadIdx.x; i < nout; i += LWK * 32) {
+            const float v = warp_sum(i);
+            if (p.late_wait) grid_dependency_wait();  // a no-op after the first time
+            store(i, v);
+        }
     }
 }
 
 // Shared-memory plan of one launch: the rings, the s / z rows, the cluster
 // partials and the mbarriers.
-size_t lean_layout(LeanParams& p) {
+size_t lean_layout(LeanParams& p, bool xs) {
     size_t off = (size_t)LWK * p.S * p.BQ * 4 * LCOLS * 4;  // the rings (1024-byte multiples)
     p.off_sz = (uint32_t)off;
     p.sz_stride = ((uint32_t)p.sz_rows * LCOLS * 2u + 127u) & ~127u;
@@ -475,13 +510,16 @@ size_t lean_layout(LeanParams& p) {
     off = (off + 7) & ~(size_t)7;
     p.off_bar = (uint32_t)off;
     off += (size_t)(LWK * LMAXS + 1) * 8;
+    off = (off + 15) & ~(size_t)15;
+    p.off_x = (uint32_t)off;
+    off += xs ? (size_t)p.M * p.xs_stride : 0;
     return off + 1024;  // slack for aligning the base to 1024 bytes
 }
 
-template <int BITS, bool BF, int BQ, bool M1, bool ALIGNED>
+template <int BITS, bool BF, int BQ, bool M1, bool ALIGNED, bool XS>
 wq_status launch_lean(const CUtensorMap& mw, const CUtensorMap& ms, const CUtensorMap& mz, const LeanParams& p,
                       size_t smem, const Problem& pb, cudaStream_t stream) {
-    auto kern = gemv_lean_kernel<BITS, BF, BQ, M1, ALIGNED>;
+    auto kern = gemv_lean_kernel<BITS, BF, BQ, M1, ALIGNED, XS>;
     static std::atomic<uint64_t> attr_ctx[MAX_DEVICES];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return WQ_ERR_CUDA;
@@ -560,7 +598,10 @@ wq_status run_lean(const Problem& pb, cudaStream_t stream) {
     rows = std::min(rows, n_groups);
     p.sz_box = std::min(rows, 256);
     p.sz_rows = (rows + p.sz_box - 1) / p.sz_box * p.sz_box;
-    const size_t smem = lean_layout(p);
+    // x written by the previous kernel (WQ_FLAG_PDL): stage it once per CTA
+    const bool xs = (pb.flags & WQ_FLAG_PDL) && !(pb.flags & WQ_FLAG_PDL_INPUTS_READY);
+    p.xs_stride = (uint32_t)(LWK * p.QW * 4 * EPS * 2) + (pb.M > 1 ? 16u : 0u);  // pad: tokens on other banks
+    const size_t smem = lean_layout(p, xs);
     if (smem > 227 * 1024) return WQ_ERR_UNSUPPORTED;
 
     CUtensorMap mw, ms, mz;
@@ -580,8 +621,11 @@ wq_status run_lean(const Problem& pb, cudaStream_t stream) {
     auto go = [&](auto bq, auto a) {
         constexpr int B = decltype(bq)::value;
         constexpr bool A = decltype(a)::value;
-        return m1 ? launch_lean<BITS, BF, B, true, A>(mw, ms, mz, p, smem, pb, stream)
-                  : launch_lean<BITS, BF, B, false, A>(mw, ms, mz, p, smem, pb, stream);
+        if (xs)
+            return m1 ? launch_lean<BITS, BF, B, true, A, true>(mw, ms, mz, p, smem, pb, stream)
+                      : launch_lean<BITS, BF, B, false, A, true>(mw, ms, mz, p, smem, pb, stream);
+        return m1 ? launch_lean<BITS, BF, B, true, A, false>(mw, ms, mz, p, smem, pb, stream)
+                  : launch_lean<BITS, BF, B, false, A, false>(mw, ms, mz, p, smem, pb, stream);
     };
     using I16 = std::integral_constant<int, 16>;
     using I8 = std::integral_constant<int, 8>;
@@ -605,6 +649,9 @@ wq_status gemv_lean_device_status(int reset) {
 bool gemv_lean_takes(const Problem& p) {
     if (p.bits != 4 && p.bits != 8) return false;
     if (p.M > 8) return false;
+    // x written by the previous kernel on the stream: the staged copy of x is
+    // read in 16-byte rows
+    if ((p.flags & WQ_FLAG_PDL) && !(p.flags & WQ_FLAG_PDL_INPUTS_READY) && p.K % 8 != 0) return false;
     const int qk = 4 * (32 / p.bits);
     return p.G == p.K || p.G % qk == 0;
 }

