@@ -144,15 +144,18 @@ struct GroupConsts {
 // not depend on it is issued and waited for first; after the grid dependency
 // wait the CTA copies its slice of x into shared memory in one round trip, and
 // the quads read it from there.
-template <int BITS, bool BF, int BQ, bool M1, bool ALIGNED, bool XS>
-__global__ void __launch_bounds__(LWK * 32, 3)
+// TOK: 1 (one token), 8 (M <= 8) or 16 (M <= 16: two 8-token MMA tiles).
+template <int BITS, bool BF, int BQ, int TOK, bool ALIGNED, bool XS>
+__global__ void __launch_bounds__(LWK * 32, TOK > 8 ? 2 : 3)
 gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
                  const __grid_constant__ CUtensorMap tm_z, const LeanParams p) {
     using F = Fmt<BITS>;
     using T16 = Dt<BF>;
     constexpr int EPS = F::EPS;
     constexpr int MMAS = EPS / 4;  // MMAs per column pair per quad
-    constexpr int NE = M1 ? 1 : 2; // tokens per lane that can exist (2 t, 2 t + 1)
+    constexpr bool M1 = TOK == 1;
+    constexpr int NT = TOK > 8 ? 2 : 1;  // 8-token MMA tiles
+    constexpr int NE = M1 ? 1 : 2;       // tokens per lane and tile that can exist (2 t, 2 t + 1)
     constexpr uint32_t BOX_BYTES = (uint32_t)BQ * 4u * LCOLS * 4u;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base: the 128-byte swizzle of the TMA boxes repeats every 1024 bytes
@@ -211,9 +214,11 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
     grid_launch_dependents();
     if (!XS && !p.late_wait) grid_dependency_wait();  // x may be the previous kernel's output
 
-    // ---- (2) this lane's x: token g (duplicates beyond M are harmless), word
-    // row 4 i + t of the warp's quad i
-    const uint16_t* xr = p.x + (M1 ? (size_t)0 : (size_t)min(g, p.M - 1) * (size_t)p.K);
+    // ---- (2) this lane's x: tokens g + 8 n (duplicates beyond M are harmless),
+    // word row 4 i + t of the warp's quad i
+    const uint16_t* xr[NT];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) xr[n] = p.x + (M1 ? (size_t)0 : (size_t)min(g + 8 * n, p.M - 1) * (size_t)p.K);
     const int kx0 = (4 * q_begin + t) * EPS;
     // quads of this warp whose 4 word rows all lie inside K (the rest: the ragged end)
     const int nq_full = max(0, min(p.Kw / 4, q_begin + p.QW) - q_begin);
@@ -268,88 +273,115 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
         }
         __syncthreads();
     }
-    const uint32_t xs_lane = smem_u32(smem + p.off_x) + (uint32_t)(M1 ? 0 : min(g, p.M - 1)) * p.xs_stride +
-                             2u * (uint32_t)(kx0 - kc0);
-    // this lane's x values of quad i of the warp's range (all of its rows inside K)
-    auto ldx = [&](int i) {
+    uint32_t xs_lane[NT];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+        xs_lane[n] = smem_u32(smem + p.off_x) + (uint32_t)(M1 ? 0 : min(g + 8 * n, p.M - 1)) * p.xs_stride +
+                     2u * (uint32_t)(kx0 - kc0);
+    // this lane's x values (token tile n) of quad i of the warp's range (all of its rows inside K)
+    auto ldx = [&](int i, int n) {
         if constexpr (XS) {
-            if constexpr (EPS == 8) return lds128_u32(xs_lane + 64u * i);
-            const uint2 v = lds64_u32(xs_lane + 32u * i);
+            if constexpr (EPS == 8) return lds128_u32(xs_lane[n] + 64u * i);
+            const uint2 v = lds64_u32(xs_lane[n] + 32u * i);
             return make_uint4(v.x, v.y, 0u, 0u);
         } else if constexpr (EPS == 8) {  // 4 word rows = 32 values on per quad
-            return __ldg(reinterpret_cast<const uint4*>(xr + kx0) + 4 * i);
+            return __ldg(reinterpret_cast<const uint4*>(xr[n] + kx0) + 4 * i);
         } else {                          // 16 values on per quad
-            const uint2 v = __ldg(reinterpret_cast<const uint2*>(xr + kx0) + 4 * i);
+            const uint2 v = __ldg(reinterpret_cast<const uint2*>(xr[n] + kx0) + 4 * i);
             return make_uint4(v.x, v.y, 0u, 0u);
         }
     };
+    // the same with a guard for rows past K (the ragged end of the range)
+    auto ldx_guarded = [&](int i, int n) {
+        if constexpr (XS) return ldx(i, n);  // the staged slice is zero past K
+        return ldg_x<EPS>(xr[n], kx0 + 4 * EPS * i, p.K);
+    };
 
     // ---- (4) main loop, FRAC: the CTA has fractional zero points
-    float acc[4][NE];
+    float acc[4][NT][NE];
 #pragma unroll
     for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int e = 0; e < NE; ++e) acc[c][e] = 0.0f;
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+            for (int e = 0; e < NE; ++e) acc[c][n][e] = 0.0f;
     auto main_loop = [&](auto frac_tag) {
         constexpr bool FRAC = decltype(frac_tag)::value;
-        float dsum[2][4], xsum = 0.0f;
+        float dsum[2][NT][4], xsum[NT];
 #pragma unroll
-        for (int T = 0; T < 2; ++T)
+        for (int n = 0; n < NT; ++n) {
+            xsum[n] = 0.0f;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) dsum[T][e] = 0.0f;
+            for (int T = 0; T < 2; ++T)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dsum[T][n][e] = 0.0f;
+        }
         // fold the group's dot products into acc (scaled by s, fractional zero points applied)
         auto fold = [&]() {
             const float2 s01 = T16::pair(sv.x), s23 = T16::pair(sv.y);
             const float sc[4] = {s01.x, s01.y, s23.x, s23.y};
-            float zr[4] = {0.0f, 0.0f, 0.0f, 0.0f}, X[NE];
+            float zr[4] = {0.0f, 0.0f, 0.0f, 0.0f}, X[NT][NE];
 #pragma unroll
-            for (int e = 0; e < NE; ++e) X[e] = 0.0f;
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int e = 0; e < NE; ++e) X[n][e] = 0.0f;
             if constexpr (FRAC) {
                 const uint2 zv = lds64_u32(sz_addr(gcur) + z_off);
                 const float2 z01 = T16::pair(zv.x), z23 = T16::pair(zv.y);
                 const float zz[4] = {z01.x, z01.y, z23.x, z23.y};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) zr[c] = zz[c] - zero_int<BITS, BF>(zz[c]);
-                // the x sum of token 2 t + e over the group's quads of this warp
-                float tot = xsum + __shfl_xor_sync(0xffffffffu, xsum, 1);
-                tot += __shfl_xor_sync(0xffffffffu, tot, 2);
+                // the x sum of token 8 n + 2 t + e over the group's quads of this warp
 #pragma unroll
-                for (int e = 0; e < NE; ++e) X[e] = __shfl_sync(0xffffffffu, tot, M1 ? 0 : 4 * (2 * t + e));
+                for (int n = 0; n < NT; ++n) {
+                    float tot = xsum[n] + __shfl_xor_sync(0xffffffffu, xsum[n], 1);
+                    tot += __shfl_xor_sync(0xffffffffu, tot, 2);
+#pragma unroll
+                    for (int e = 0; e < NE; ++e) X[n][e] = __shfl_sync(0xffffffffu, tot, M1 ? 0 : 4 * (2 * t + e));
+                }
             }
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int T = c >> 1, half = c & 1;
 #pragma unroll
-                for (int e = 0; e < NE; ++e) {
-                    float d = dsum[T][2 * half + e];
-                    if constexpr (FRAC) d = fmaf(-zr[c], X[e], d);
-                    acc[c][e] = fmaf(sc[c], d, acc[c][e]);
-                }
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int e = 0; e < NE; ++e) {
+                        float d = dsum[T][n][2 * half + e];
+                        if constexpr (FRAC) d = fmaf(-zr[c], X[n][e], d);
+                        acc[c][n][e] = fmaf(sc[c], d, acc[c][n][e]);
+                    }
             }
 #pragma unroll
-            for (int T = 0; T < 2; ++T)
+            for (int n = 0; n < NT; ++n) {
+                xsum[n] = 0.0f;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) dsum[T][e] = 0.0f;
-            xsum = 0.0f;
+                for (int T = 0; T < 2; ++T)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dsum[T][n][e] = 0.0f;
+            }
         };
-        // one quad: the words hv (this lane's 16 bytes) and its x values xa
-        auto quad = [&](const uint4& hv, const uint4& xa) {
-            uint32_t bx[EPS / 2];
-            if constexpr (EPS == 8) {  // pairs (0, 4), (1, 5), (2, 6), (3, 7) of the row's 8 values
-                bx[0] = prmt(xa.x, xa.z, 0x5410u);
-                bx[1] = prmt(xa.x, xa.z, 0x7632u);
-                bx[2] = prmt(xa.y, xa.w, 0x5410u);
-                bx[3] = prmt(xa.y, xa.w, 0x7632u);
-            } else {                   // pairs (0, 2), (1, 3) of the row's 4 values
-                bx[0] = prmt(xa.x, xa.y, 0x5410u);
-                bx[1] = prmt(xa.x, xa.y, 0x7632u);
-            }
-            if constexpr (FRAC) {  // this lane's row sum of x (fp32)
-                const uint32_t xv[4] = {xa.x, xa.y, xa.z, xa.w};
+        // one quad: the words hv (this lane's 16 bytes) and its x values xa[n]
+        auto quad = [&](const uint4& hv, const uint4 (&xa)[NT]) {
+            uint32_t bx[NT][EPS / 2];
 #pragma unroll
-                for (int u = 0; u < EPS / 2; ++u) {
-                    const float2 f = T16::pair(xv[u]);
-                    xsum += f.x + f.y;
+            for (int n = 0; n < NT; ++n) {
+                if constexpr (EPS == 8) {  // pairs (0, 4), (1, 5), (2, 6), (3, 7) of the row's 8 values
+                    bx[n][0] = prmt(xa[n].x, xa[n].z, 0x5410u);
+                    bx[n][1] = prmt(xa[n].x, xa[n].z, 0x7632u);
+                    bx[n][2] = prmt(xa[n].y, xa[n].w, 0x5410u);
+                    bx[n][3] = prmt(xa[n].y, xa[n].w, 0x7632u);
+                } else {                   // pairs (0, 2), (1, 3) of the row's 4 values
+                    bx[n][0] = prmt(xa[n].x, xa[n].y, 0x5410u);
+                    bx[n][1] = prmt(xa[n].x, xa[n].y, 0x7632u);
+                }
+                if constexpr (FRAC) {  // this lane's row sum of x (fp32)
+                    const uint32_t xv[4] = {xa[n].x, xa[n].y, xa[n].z, xa[n].w};
+#pragma unroll
+                    for (int u = 0; u < EPS / 2; ++u) {
+                        const float2 f = T16::pair(xv[u]);
+                        xsum[n] += f.x + f.y;
+                    }
                 }
             }
             const uint32_t wv[4] = {hv.x, hv.y, hv.z, hv.w};
@@ -365,7 +397,8 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
                     a[1] = WB.pair(k.cc[2 * T + 1], 2 * h);
                     a[2] = WA.pair(k.cc[2 * T], 2 * h + 1);
                     a[3] = WB.pair(k.cc[2 * T + 1], 2 * h + 1);
-                    mma_16816<BF>(dsum[T], a, bx[2 * h], bx[2 * h + 1]);
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) mma_16816<BF>(dsum[T][n], a, bx[n][2 * h], bx[n][2 * h + 1]);
                 }
             }
         };
@@ -373,7 +406,12 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
         auto block = [&](uint32_t slot_addr, int i4, int i) {
             const uint32_t wblk = slot_addr + 512u * (uint32_t)i4;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) quad(lds128_u32(wblk + 512u * j + ((j & 1) ? off_odd : off_even)), ldx(i + j));
+            for (int j = 0; j < 4; ++j) {
+                uint4 xa[NT];
+#pragma unroll
+                for (int n = 0; n < NT; ++n) xa[n] = ldx(i + j, n);
+                quad(lds128_u32(wblk + 512u * j + ((j & 1) ? off_odd : off_even)), xa);
+            }
         };
 
         if constexpr (ALIGNED) {
@@ -422,8 +460,10 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             if (i + j < nq) {
-                                quad(lds128_u32(wblk + 512u * j + ((j & 1) ? off_odd : off_even)),
-                                     XS ? ldx(i + j) : ldg_x<EPS>(xr, kx0 + 4 * EPS * (i + j), p.K));
+                                uint4 xa[NT];
+#pragma unroll
+                                for (int n = 0; n < NT; ++n) xa[n] = ldx_guarded(i + j, n);
+                                quad(lds128_u32(wblk + 512u * j + ((j & 1) ? off_odd : off_even)), xa);
                                 if (--left == 0) group_end(i + j);
                             }
                         }
@@ -453,10 +493,12 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-            for (int e = 0; e < NE; ++e) {
-                const int m = 2 * t + e;
-                if (m < p.M) red[m * LCOLS + 4 * cg + c] = acc[c][e];
-            }
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int e = 0; e < NE; ++e) {
+                    const int m = 8 * n + 2 * t + e;
+                    if (m < p.M) red[m * LCOLS + 4 * cg + c] = acc[c][n][e];
+                }
     }
     __syncthreads();
     auto warp_sum = [&](int i) {
@@ -516,10 +558,10 @@ size_t lean_layout(LeanParams& p, bool xs) {
     return off + 1024;  // slack for aligning the base to 1024 bytes
 }
 
-template <int BITS, bool BF, int BQ, bool M1, bool ALIGNED, bool XS>
+template <int BITS, bool BF, int BQ, int TOK, bool ALIGNED, bool XS>
 wq_status launch_lean(const CUtensorMap& mw, const CUtensorMap& ms, const CUtensorMap& mz, const LeanParams& p,
                       size_t smem, const Problem& pb, cudaStream_t stream) {
-    auto kern = gemv_lean_kernel<BITS, BF, BQ, M1, ALIGNED, XS>;
+    auto kern = gemv_lean_kernel<BITS, BF, BQ, TOK, ALIGNED, XS>;
     static std::atomic<uint64_t> attr_ctx[MAX_DEVICES];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return WQ_ERR_CUDA;
@@ -617,15 +659,16 @@ wq_status run_lean(const Problem& pb, cudaStream_t stream) {
     const bool aligned = p.S == 1 && p.QW == BQ && p.Q == KS * LWK * p.QW && p.Kw == 4 * p.Q &&
                          ((p.qpg <= p.QW && p.QW % p.qpg == 0 && p.qpg % 4 == 0) ||
                           (p.qpg > p.QW && (p.qpg % p.QW == 0 || p.qpg >= p.Q)));
-    const bool m1 = pb.M == 1;
     auto go = [&](auto bq, auto a) {
         constexpr int B = decltype(bq)::value;
         constexpr bool A = decltype(a)::value;
-        if (xs)
-            return m1 ? launch_lean<BITS, BF, B, true, A, true>(mw, ms, mz, p, smem, pb, stream)
-                      : launch_lean<BITS, BF, B, false, A, true>(mw, ms, mz, p, smem, pb, stream);
-        return m1 ? launch_lean<BITS, BF, B, true, A, false>(mw, ms, mz, p, smem, pb, stream)
-                  : launch_lean<BITS, BF, B, false, A, false>(mw, ms, mz, p, smem, pb, stream);
+        auto tok = [&](auto xs_tag) {
+            constexpr bool X = decltype(xs_tag)::value;
+            if (pb.M == 1) return launch_lean<BITS, BF, B, 1, A, X>(mw, ms, mz, p, smem, pb, stream);
+            if (pb.M <= 8) return launch_lean<BITS, BF, B, 8, A, X>(mw, ms, mz, p, smem, pb, stream);
+            return launch_lean<BITS, BF, B, 16, A, X>(mw, ms, mz, p, smem, pb, stream);
+        };
+        return xs ? tok(std::true_type{}) : tok(std::false_type{});
     };
     using I16 = std::integral_constant<int, 16>;
     using I8 = std::integral_constant<int, 8>;
@@ -648,7 +691,7 @@ wq_status gemv_lean_device_status(int reset) {
 
 bool gemv_lean_takes(const Problem& p) {
     if (p.bits != 4 && p.bits != 8) return false;
-    if (p.M > 8) return false;
+    if (p.M > 16) return false;
     // x written by the previous kernel on the stream: the staged copy of x is
     // read in 16-byte rows
     if ((p.flags & WQ_FLAG_PDL) && !(p.flags & WQ_FLAG_PDL_INPUTS_READY) && p.K % 8 != 0) return false;
