@@ -153,7 +153,11 @@ int wq_matmul_uses_gemv(int M, int K, int N, int bits, int group_size) {
     if (!supported_bits(bits) || M < 1 || K < 1 || N < 1) return 0;
     const int G = group_size == -1 ? K : group_size;
     const bool gemv_group = G == K || (G > 0 && G % (4 * main_eps(bits)) == 0);
-    const bool small_m = M <= 8 || (M <= 16 && (long long)M * K < 65536);
+    // 4- and 8-bit words: the lean GEMV takes up to 16 tokens (M = 16 of 4096 x 4096
+    // in 3.4 us, below the GEMM's fixed cost per launch); other widths stage x on
+    // chip, so M = 9..16 goes there only while M * K < 65536
+    const bool lean = bits == 4 || bits == 8;
+    const bool small_m = M <= 8 || (M <= 16 && (lean || (long long)M * K < 65536));
     return (gemv_group && small_m) ? 1 : 0;
 }
 

@@ -173,8 +173,9 @@ wq_status wq_gemm(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
 /*
  * The product for any M, routed to wq_gemv or wq_gemm by a measured crossover
  * (the M-crossover of the "next" list; not in the pages): wq_gemv when
- * M <= 8, or M <= 16 with M * K < 65536 (x then fits its on-chip staging),
- * and the group size is one wq_gemv takes; wq_gemm otherwise.  Same arguments
+ * M <= 8, or M <= 16 with 4- or 8-bit words or with M * K < 65536 (x then
+ * fits its on-chip staging), and the group size is one wq_gemv takes;
+ * wq_gemm otherwise.  Same arguments
  * and rules as wq_gemm; the workspace is used only on the wq_gemm route
  * (wq_matmul_workspace_size() reports 0 on the other).
  */

@@ -139,15 +139,19 @@ def test_pack_argument_checks(libwq):
 
 
 def test_matmul_route(libwq):
-    """wq_matmul's crossover: wq_gemv for M <= 8, or M <= 16 with M * K < 65536,
-    when the group size is one wq_gemv takes; wq_gemm otherwise."""
+    """wq_matmul's crossover: wq_gemv for M <= 8, or M <= 16 with 4- or 8-bit
+    words or M * K < 65536, when the group size is one wq_gemv takes; wq_gemm
+    otherwise."""
     L = libwq.lib()
     route = lambda *a: int(L.wq_matmul_uses_gemv(*a))
     assert route(1, 4096, 4096, 4, 128) == 1
     assert route(8, 8192, 8192, 4, 128) == 1
     assert route(12, 4096, 4096, 4, 128) == 1
-    assert route(12, 8192, 4096, 4, 128) == 0      # 12 x 8192 >= 65536
-    assert route(16, 4096, 4096, 4, 128) == 0      # 16 x 4096 = 65536
+    assert route(12, 8192, 4096, 4, 128) == 1      # 4-bit: up to 16 tokens
+    assert route(16, 4096, 4096, 8, 128) == 1
+    assert route(12, 8192, 4096, 2, 128) == 0      # 2-bit: 12 x 8192 >= 65536
+    assert route(16, 4096, 4096, 3, 128) == 0      # 3-bit: 16 x 4096 = 65536
+    assert route(16, 2048, 4096, 1, 128) == 1      # 1-bit: 16 x 2048 < 65536
     assert route(17, 512, 256, 4, 128) == 0
     assert route(1, 4096, 4096, 4, 16) == 0        # group 16 is wq_gemm's only
     assert route(1, 4096, 4096, 4, -1) == 1

@@ -219,6 +219,6 @@ def test_matmul_either_route_matches_oracle(cuda, libwq, orc, M):
     d = to_dev(case, cuda)
     w_q, w_lo = libwq.pack_kmajor(d["codes"], 4)
     y = libwq.matmul(d["x"], w_q, w_lo, d["scales"], d["zeros"], 4, 128).cpu().numpy()
-    assert libwq.uses_gemv(M, K, N, 4, 128) == (M <= 12)
+    assert libwq.uses_gemv(M, K, N, 4, 128) == (M <= 16)
     y_ref, b = oracle_product(orc, case)
     check_product(y, y_ref, b, f"matmul M={M}")
