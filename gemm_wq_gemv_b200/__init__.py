@@ -92,6 +92,12 @@ def lib() -> ctypes.CDLL:
         L.wq_gptqmodel_convert.restype = i
         L.wq_mse_search.argtypes = [p, i, i, i, i, i, i, i, ctypes.c_float, i, p, p, p, p, p, ctypes.c_size_t, p]
         L.wq_mse_search.restype = i
+        L.wq_gemv_plan_create.argtypes = [p, p, p, p, p, i, i, i, i, i, u, ctypes.POINTER(p)]
+        L.wq_gemv_plan_create.restype = i
+        L.wq_gemv_plan_run.argtypes = [p, p, p, p]
+        L.wq_gemv_plan_run.restype = i
+        L.wq_gemv_plan_destroy.argtypes = [p]
+        L.wq_gemv_plan_destroy.restype = None
         for f in ("wq_pack_kmajor", "wq_unpack_kmajor", "wq_gemv", "wq_gemm", "wq_device_status",
                   "wq_selftest_wait_timeout"):
             getattr(L, f).restype = i
@@ -302,6 +308,71 @@ def gemv(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl:
     tensor of x's type added to every row of the output."""
     return _product("wq_gemv", x, w_q, w_lo, scales, zeros, bits, group_size, out, pdl,
                     inputs_ready=inputs_ready, bias=bias)
+
+
+class GemvPlan:
+    """A decode product with its weights bound once (``wq_gemv_plan``): the
+    dashq_kernel.py page's TritonQuantLinear, as a prepared launch.
+
+    ``plan = GemvPlan(w_q, w_lo, scales, zeros, bits, group_size, M, bias=None,
+    pdl=False, inputs_ready=False)`` checks the weights as ``gemv`` would for an
+    ``(M, K)`` x of the scales' type and records the kernel, its launch shape
+    and the weight descriptors; ``plan(x, out=None)`` is then ``gemv(x, ...)``
+    with the same bits, for a CUDA tensor x of shape (M, K) on the same device,
+    at the cost of one launch.  The plan holds references to the weight
+    tensors, which must not be resized or moved (their contents may change)."""
+
+    def __init__(self, w_q, w_lo, scales, zeros, bits: int, group_size: int, M: int, bias=None,
+                 pdl: bool = False, inputs_ready: bool = False):
+        torch = _torch()
+        dt = _elem_type(scales)
+        if bits not in _BITS:
+            raise ValueError(f"bits must be one of {_BITS}, got {bits}")
+        K = w_q.shape[0] * _EPS[bits]  # word rows x codes per word
+        x_meta = torch.empty((M, K), dtype=dt, device=w_q.device)
+        for t, name in ((w_q, "w_q"), (scales, "scales"), (zeros, "zeros")):
+            _need(t, torch.int32 if name == "w_q" else dt, name)
+        if w_lo is not None:
+            _need(w_lo, torch.int32, "w_lo")
+        if bias is not None:
+            _need(bias, dt, "bias", ndim=1)
+        _check_product(x_meta, w_q, w_lo, scales, zeros, bias, None, bits, group_size)
+        N = w_q.shape[1]
+        flags = ((WQ_FLAG_PDL if pdl else 0) | (WQ_FLAG_PDL_INPUTS_READY if inputs_ready else 0)
+                 | (WQ_FLAG_BF16 if dt is torch.bfloat16 else 0))
+        self._lib = lib()
+        h = ctypes.c_void_p()
+        with torch.cuda.device(w_q.device):
+            st = self._lib.wq_gemv_plan_create(_ptr(w_q), _ptr(w_lo), _ptr(scales), _ptr(zeros), _ptr(bias),
+                                               M, K, N, bits, group_size, flags, ctypes.byref(h))
+        _check("wq_gemv_plan_create", st)
+        self._h = h.value
+        self._keep = (w_q, w_lo, scales, zeros, bias)
+        self.dtype, self.device, self.M, self.K, self.N = dt, w_q.device, M, K, N
+        self._dev = w_q.get_device()
+        self._xshape, self._yshape = (M, K), (M, N)
+        self._run = self._lib.wq_gemv_plan_run
+
+    def __call__(self, x, out=None):
+        if not (getattr(x, "is_cuda", False) and x.dtype is self.dtype and x.shape == self._xshape
+                and x.is_contiguous() and x.get_device() == self._dev):
+            raise ValueError(f"x must be a contiguous {self.dtype} CUDA tensor of shape {self._xshape} "
+                             f"on {self.device}")
+        if out is None:
+            out = _torch().empty(self._yshape, dtype=self.dtype, device=x.device)
+        elif not (getattr(out, "is_cuda", False) and out.dtype is self.dtype and out.shape == self._yshape
+                  and out.is_contiguous() and out.get_device() == self._dev):
+            raise ValueError(f"out must be a contiguous {self.dtype} CUDA tensor of shape {self._yshape} "
+                             f"on {self.device}")
+        st = self._run(self._h, x.data_ptr(), out.data_ptr(), _stream())
+        if st != 0:
+            raise WQError("wq_gemv_plan_run", st)
+        return out
+
+    def __del__(self):
+        h, self._h = getattr(self, "_h", None), None
+        if h:
+            self._lib.wq_gemv_plan_destroy(h)
 
 
 def gemm_workspace_size(M: int, K: int, N: int, bits: int, group_size: int) -> int:

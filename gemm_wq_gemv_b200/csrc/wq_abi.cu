@@ -4,6 +4,8 @@
 // Nothing is launched unless every check passes.
 #include <cuda_runtime.h>
 
+#include <new>
+
 #include "wq_internal.h"
 
 namespace {
@@ -124,6 +126,49 @@ wq_status wq_gemv(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
     wq::Problem p{x, w_q, w_lo, scales, zeros, bias, y, M, K, N, bits, G, flags, nullptr, 0};
     return wq::launch_gemv(p, (cudaStream_t)stream);
 }
+
+struct wq_gemv_plan {
+    wq::Prepared pr;
+    int dev;
+};
+
+wq_status wq_gemv_plan_create(const uint32_t* w_q, const uint32_t* w_lo, const uint16_t* scales,
+                              const uint16_t* zeros, const uint16_t* bias, int M, int K, int N, int bits,
+                              int group_size, unsigned flags, wq_gemv_plan** plan) {
+    if (!plan) return WQ_ERR_INVALID_ARG;
+    *plan = nullptr;
+    // x and y are bound at each run: w_q stands in for them in the shared checks
+    const uint16_t* stand_in = reinterpret_cast<const uint16_t*>(w_q);
+    int G = 0;
+    wq_status st = check_product(stand_in, w_q, w_lo, scales, zeros, stand_in, M, K, N, bits, group_size, flags, G);
+    if (st != WQ_OK) return st;
+    if (bias && !aligned(bias, 2)) return WQ_ERR_ALIGNMENT;
+    if (M > 16) return WQ_ERR_INVALID_ARG;
+    if (G != K && G % (4 * main_eps(bits)) != 0) return WQ_ERR_UNSUPPORTED;
+    if ((st = check_device()) != WQ_OK) return st;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return WQ_ERR_CUDA;
+    wq_gemv_plan* h = new (std::nothrow) wq_gemv_plan();
+    if (!h) return WQ_ERR_CUDA;
+    h->dev = dev;
+    const wq::Problem p{nullptr, w_q, w_lo, scales, zeros, bias, nullptr, M, K, N, bits, G, flags, nullptr, 0};
+    if ((st = wq::prepare_gemv(p, h->pr)) != WQ_OK) {
+        delete h;
+        return st;
+    }
+    *plan = h;
+    return WQ_OK;
+}
+
+wq_status wq_gemv_plan_run(const wq_gemv_plan* plan, const uint16_t* x, uint16_t* y, void* stream) {
+    if (!plan || !x || !y) return WQ_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(y, 16)) return WQ_ERR_ALIGNMENT;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != plan->dev) return WQ_ERR_INVALID_ARG;
+    return wq::launch_prepared(plan->pr, x, y, (cudaStream_t)stream);
+}
+
+void wq_gemv_plan_destroy(wq_gemv_plan* plan) { delete plan; }
 
 wq_status wq_gemm(const uint16_t* x, const uint32_t* w_q, const uint32_t* w_lo,
                   const uint16_t* scales, const uint16_t* zeros, const uint16_t* bias, uint16_t* y,

@@ -34,6 +34,8 @@
 //    to the fp32 sum before the final rounding.
 #include <algorithm>
 #include <array>
+#include <cstddef>
+#include <cstring>
 #include <map>
 #include <mutex>
 #include <type_traits>
@@ -590,8 +592,10 @@ int ilog2(int v) {
     return r;
 }
 
+static_assert(4 * sizeof(CUtensorMap) + sizeof(Params) <= sizeof(Prepared::args), "prepared launch arguments");
+
 template <int BITS, int NT, bool BF>
-wq_status run(const Problem& pb, cudaStream_t stream) {
+wq_status run(const Problem& pb, cudaStream_t stream, Prepared* prep) {
     using F = Fmt<BITS>;
     constexpr int EPS = F::EPS;
     constexpr int QK = 4 * EPS;
@@ -742,6 +746,28 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
         ml = mw;
     if (!ok) return WQ_ERR_CUDA;
 
+    if (prep) {  // record the launch instead of making it
+        Prepared& r = *prep;
+        r.kern = (const void*)kern;
+        r.grid = dim3(colblocks, best.CS, 1);
+        r.block = dim3(best.WK * 32, 1, 1);
+        r.smem = best_smem;
+        r.cluster_y = best.CS > 1 ? (unsigned)best.CS : 1u;
+        r.pdl = (pb.flags & (WQ_FLAG_PDL | WQ_FLAG_PDL_INPUTS_READY)) != 0;
+        r.nargs = 5;
+        const size_t mo = sizeof(CUtensorMap);
+        const CUtensorMap* maps[4] = {&mw, &ml, &ms, &mz};
+        for (int i = 0; i < 4; ++i) {
+            std::memcpy(r.args + i * mo, maps[i], mo);
+            r.arg_off[i] = i * mo;
+        }
+        std::memcpy(r.args + 4 * mo, &best, sizeof(best));
+        r.arg_off[4] = 4 * mo;
+        r.x_off = 4 * mo + offsetof(Params, x);
+        r.y_off = 4 * mo + offsetof(Params, y);
+        return WQ_OK;
+    }
+
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(colblocks, best.CS, 1);
     cfg.blockDim = dim3(best.WK * 32, 1, 1);
@@ -782,26 +808,32 @@ wq_status gemv_device_status(int reset) {
 namespace {
 
 template <bool BF>
-wq_status launch_typed(const Problem& p, cudaStream_t s) {
+wq_status launch_typed(const Problem& p, cudaStream_t s, Prepared* prep) {
     const bool two = p.M > 8;
     switch (p.bits) {
-        case 1: return two ? run<1, 2, BF>(p, s) : run<1, 1, BF>(p, s);
-        case 2: return two ? run<2, 2, BF>(p, s) : run<2, 1, BF>(p, s);
-        case 3: return two ? run<3, 2, BF>(p, s) : run<3, 1, BF>(p, s);
-        case 4: return two ? run<4, 2, BF>(p, s) : run<4, 1, BF>(p, s);
-        case 8: return two ? run<8, 2, BF>(p, s) : run<8, 1, BF>(p, s);
+        case 1: return two ? run<1, 2, BF>(p, s, prep) : run<1, 1, BF>(p, s, prep);
+        case 2: return two ? run<2, 2, BF>(p, s, prep) : run<2, 1, BF>(p, s, prep);
+        case 3: return two ? run<3, 2, BF>(p, s, prep) : run<3, 1, BF>(p, s, prep);
+        case 4: return two ? run<4, 2, BF>(p, s, prep) : run<4, 1, BF>(p, s, prep);
+        case 8: return two ? run<8, 2, BF>(p, s, prep) : run<8, 1, BF>(p, s, prep);
         default: return WQ_ERR_UNSUPPORTED;
     }
 }
 
 }  // namespace
 
-wq_status launch_gemv(const Problem& p, cudaStream_t s) {
+namespace {
+wq_status gemv_route(const Problem& p, cudaStream_t s, Prepared* prep) {
     if (gemv_lean_takes(p)) {
-        const wq_status st = launch_gemv_lean(p, s);
+        const wq_status st = launch_gemv_lean(p, s, prep);
         if (st != WQ_ERR_UNSUPPORTED) return st;  // else: its x stage does not fit; the kernel below takes it
     }
-    return (p.flags & WQ_FLAG_BF16) ? launch_typed<true>(p, s) : launch_typed<false>(p, s);
+    return (p.flags & WQ_FLAG_BF16) ? launch_typed<true>(p, s, prep) : launch_typed<false>(p, s, prep);
 }
+}  // namespace
+
+wq_status launch_gemv(const Problem& p, cudaStream_t s) { return gemv_route(p, s, nullptr); }
+
+wq_status prepare_gemv(const Problem& p, Prepared& pr) { return gemv_route(p, nullptr, &pr); }
 
 }  // namespace wq

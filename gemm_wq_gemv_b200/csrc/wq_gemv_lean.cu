@@ -38,6 +38,8 @@
 // Every mbarrier wait is bounded; on time-out the kernel records it in the
 // GEMV's device status word and skips the rest of the warp's range.
 #include <algorithm>
+#include <cstddef>
+#include <cstring>
 #include <type_traits>
 
 #include "wq_dequant.cuh"
@@ -539,6 +541,8 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
     }
 }
 
+static_assert(3 * sizeof(CUtensorMap) + sizeof(LeanParams) <= sizeof(Prepared::args), "prepared launch arguments");
+
 // Shared-memory plan of one launch: the rings, the s / z rows, the cluster
 // partials and the mbarriers.
 size_t lean_layout(LeanParams& p, bool xs) {
@@ -560,12 +564,31 @@ size_t lean_layout(LeanParams& p, bool xs) {
 
 template <int BITS, bool BF, int BQ, int TOK, bool ALIGNED, bool XS>
 wq_status launch_lean(const CUtensorMap& mw, const CUtensorMap& ms, const CUtensorMap& mz, const LeanParams& p,
-                      size_t smem, const Problem& pb, cudaStream_t stream) {
+                      size_t smem, const Problem& pb, cudaStream_t stream, Prepared* prep) {
     auto kern = gemv_lean_kernel<BITS, BF, BQ, TOK, ALIGNED, XS>;
     static std::atomic<uint64_t> attr_ctx[MAX_DEVICES];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return WQ_ERR_CUDA;
     if (const wq_status st = ensure_smem_attr((const void*)kern, 227 * 1024, attr_ctx, dev); st != WQ_OK) return st;
+    if (prep) {  // record the launch instead of making it
+        Prepared& r = *prep;
+        r.kern = (const void*)kern;
+        r.grid = dim3((pb.N + LCOLS - 1) / LCOLS, p.KS, 1);
+        r.block = dim3(LWK * 32, 1, 1);
+        r.smem = smem;
+        r.cluster_y = p.KS > 1 ? (unsigned)p.KS : 1u;
+        r.pdl = (pb.flags & (WQ_FLAG_PDL | WQ_FLAG_PDL_INPUTS_READY)) != 0;
+        r.nargs = 4;
+        const size_t mo = sizeof(CUtensorMap);
+        std::memcpy(r.args, &mw, mo);
+        std::memcpy(r.args + mo, &ms, mo);
+        std::memcpy(r.args + 2 * mo, &mz, mo);
+        std::memcpy(r.args + 3 * mo, &p, sizeof(p));
+        r.arg_off[0] = 0; r.arg_off[1] = mo; r.arg_off[2] = 2 * mo; r.arg_off[3] = 3 * mo;
+        r.x_off = 3 * mo + offsetof(LeanParams, x);
+        r.y_off = 3 * mo + offsetof(LeanParams, y);
+        return WQ_OK;
+    }
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((pb.N + LCOLS - 1) / LCOLS, p.KS, 1);
     cfg.blockDim = dim3(LWK * 32, 1, 1);
@@ -591,7 +614,7 @@ wq_status launch_lean(const CUtensorMap& mw, const CUtensorMap& ms, const CUtens
 }
 
 template <int BITS, bool BF>
-wq_status run_lean(const Problem& pb, cudaStream_t stream) {
+wq_status run_lean(const Problem& pb, cudaStream_t stream, Prepared* prep) {
     constexpr int EPS = Fmt<BITS>::EPS;
     constexpr int QK = 4 * EPS;
     LeanParams p{};
@@ -664,9 +687,9 @@ wq_status run_lean(const Problem& pb, cudaStream_t stream) {
         constexpr bool A = decltype(a)::value;
         auto tok = [&](auto xs_tag) {
             constexpr bool X = decltype(xs_tag)::value;
-            if (pb.M == 1) return launch_lean<BITS, BF, B, 1, A, X>(mw, ms, mz, p, smem, pb, stream);
-            if (pb.M <= 8) return launch_lean<BITS, BF, B, 8, A, X>(mw, ms, mz, p, smem, pb, stream);
-            return launch_lean<BITS, BF, B, 16, A, X>(mw, ms, mz, p, smem, pb, stream);
+            if (pb.M == 1) return launch_lean<BITS, BF, B, 1, A, X>(mw, ms, mz, p, smem, pb, stream, prep);
+            if (pb.M <= 8) return launch_lean<BITS, BF, B, 8, A, X>(mw, ms, mz, p, smem, pb, stream, prep);
+            return launch_lean<BITS, BF, B, 16, A, X>(mw, ms, mz, p, smem, pb, stream, prep);
         };
         return xs ? tok(std::true_type{}) : tok(std::false_type{});
     };
@@ -699,11 +722,11 @@ bool gemv_lean_takes(const Problem& p) {
     return p.G == p.K || p.G % qk == 0;
 }
 
-wq_status launch_gemv_lean(const Problem& p, cudaStream_t s) {
+wq_status launch_gemv_lean(const Problem& p, cudaStream_t s, Prepared* prep) {
     const bool bf = (p.flags & WQ_FLAG_BF16) != 0;
     switch (p.bits) {
-        case 4: return bf ? run_lean<4, true>(p, s) : run_lean<4, false>(p, s);
-        case 8: return bf ? run_lean<8, true>(p, s) : run_lean<8, false>(p, s);
+        case 4: return bf ? run_lean<4, true>(p, s, prep) : run_lean<4, false>(p, s, prep);
+        case 8: return bf ? run_lean<8, true>(p, s, prep) : run_lean<8, false>(p, s, prep);
         default: return WQ_ERR_UNSUPPORTED;
     }
 }

@@ -2,6 +2,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cstring>
 
 #include "wq_internal.h"
 
@@ -129,6 +130,41 @@ int sm_count() {
     if (n <= 0) n = 148;
     if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
     return n;
+}
+
+}  // namespace wq
+
+namespace wq {
+
+wq_status launch_prepared(const Prepared& pr, const void* x, void* y, cudaStream_t s) {
+    alignas(64) unsigned char args[sizeof(pr.args)];
+    std::memcpy(args, pr.args, sizeof(args));
+    std::memcpy(args + pr.x_off, &x, sizeof(x));
+    std::memcpy(args + pr.y_off, &y, sizeof(y));
+    void* argv[6];
+    for (int i = 0; i < pr.nargs; ++i) argv[i] = args + pr.arg_off[i];
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = pr.grid;
+    cfg.blockDim = pr.block;
+    cfg.dynamicSmemBytes = pr.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attrs[2];
+    int na = 0;
+    if (pr.cluster_y > 1) {
+        attrs[na].id = cudaLaunchAttributeClusterDimension;
+        attrs[na].val.clusterDim.x = 1;
+        attrs[na].val.clusterDim.y = pr.cluster_y;
+        attrs[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (pr.pdl) {
+        attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attrs[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = attrs;
+    cfg.numAttrs = na;
+    return from_cuda(cudaLaunchKernelExC(&cfg, pr.kern, argv));
 }
 
 }  // namespace wq

@@ -34,10 +34,29 @@ wq_status launch_gptqmodel_convert(const uint32_t* qweight, const uint32_t* qzer
                                    int G, uint32_t* w_q, uint32_t* w_lo, uint16_t* zeros, bool bf,
                                    cudaStream_t s);
 wq_status launch_gemv(const Problem& p, cudaStream_t s);
-// GEMV with a small shared-memory footprint for 4- and 8-bit words and M <= 8
+
+// A GEMV launch prepared once for fixed weights, s, z, bias, shape and flags:
+// the kernel, its launch shape and its arguments (tensor maps, then the
+// parameter block), with the byte offsets of the x and y pointers inside the
+// argument bytes.  launch_prepared patches x and y into a copy and launches.
+struct Prepared {
+    const void* kern = nullptr;
+    dim3 grid{1, 1, 1}, block{1, 1, 1};
+    size_t smem = 0;
+    unsigned cluster_y = 1;   // CTAs per cluster along the grid's y extent (1: no cluster)
+    bool pdl = false;         // programmatic stream serialisation attribute
+    int nargs = 0;
+    size_t arg_off[6] = {};   // byte offset of each kernel argument in `args`
+    size_t x_off = 0, y_off = 0;
+    alignas(64) unsigned char args[5 * sizeof(CUtensorMap) + 512] = {};
+};
+// Fill `pr` for problem p (x and y may be null) instead of launching.
+wq_status prepare_gemv(const Problem& p, Prepared& pr);
+wq_status launch_prepared(const Prepared& pr, const void* x, void* y, cudaStream_t s);
+// GEMV with a small shared-memory footprint for 4- and 8-bit words and M <= 16
 // (wq_gemv_lean.cu); launch_gemv routes the shapes it takes there.
 bool gemv_lean_takes(const Problem& p);
-wq_status launch_gemv_lean(const Problem& p, cudaStream_t s);
+wq_status launch_gemv_lean(const Problem& p, cudaStream_t s, Prepared* prep = nullptr);
 wq_status launch_gemm(const Problem& p, cudaStream_t s);
 size_t gemm_workspace_bytes(int M, int K, int N, int bits, int G);
 wq_status launch_mse_search(const float* w, int rows, int cols, int group_size, int bits, int symmetric,

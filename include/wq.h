@@ -292,6 +292,34 @@ wq_status wq_mse_search(const float* w, int rows, int cols, int group_size, int 
                         void* stream);
 
 /*
+ * A decode product prepared once (the weights bound, x and y per call).  The
+ * dashq_kernel.py page's TritonQuantLinear holds the packed weights, scales
+ * and zero points as a layer and applies them to each new x; this is that
+ * layer at the C level: the plan keeps the kernel choice, its launch shape and
+ * the TMA descriptors of w_q, w_lo, scales and zeros, so a run is one launch.
+ *
+ * wq_gemv_plan_create: the arguments of wq_gemv without x, y and the stream,
+ *   checked by the same rules (x and y are checked at each run), on the current
+ *   device.  *plan receives a handle (null on error).  The plan refers to the
+ *   weight, s, z and bias arrays by address: they must stay allocated and may
+ *   not move while the plan is used (their contents may change).  Host-only
+ *   work plus device attribute queries; nothing is launched.
+ * wq_gemv_plan_run: y (M x N) = x (M x K) @ dequant(W_q) on `stream`, the same
+ *   result, bits and launch flags as wq_gemv with the plan's arguments.  x, y:
+ *   device pointers, 16-byte aligned (else WQ_ERR_ALIGNMENT).  The current
+ *   device must be the plan's (else WQ_ERR_INVALID_ARG, nothing launched).
+ *   Safe to call from several host threads on one plan (the plan is read only).
+ * wq_gemv_plan_destroy: frees the handle (null is allowed).  The plan is valid
+ *   in the CUDA context it was created in.
+ */
+typedef struct wq_gemv_plan wq_gemv_plan;
+wq_status wq_gemv_plan_create(const uint32_t* w_q, const uint32_t* w_lo, const uint16_t* scales,
+                              const uint16_t* zeros, const uint16_t* bias, int M, int K, int N, int bits,
+                              int group_size, unsigned flags, wq_gemv_plan** plan);
+wq_status wq_gemv_plan_run(const wq_gemv_plan* plan, const uint16_t* x, uint16_t* y, void* stream);
+void wq_gemv_plan_destroy(wq_gemv_plan* plan);
+
+/*
  * Device-side status of the current device: WQ_OK, or WQ_ERR_TIMEOUT when a
  * kernel on this device gave up a bounded wait since the last reset (its
  * output is then incomplete).  Synchronises the device.  reset != 0 clears it.

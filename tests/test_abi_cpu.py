@@ -198,3 +198,19 @@ def test_mse_search_argument_checks(libwq):
     if not torch.cuda.is_available():
         assert call() == 6                              # valid: reaches CUDA, which has no device here
         assert call(pat=5, ws=P, ws_bytes=4) == 6
+
+
+def test_gemv_plan_argument_checks(libwq):
+    """wq_gemv_plan_*: null handles and bad shapes are refused before any CUDA call."""
+    L = libwq.lib()
+    P = ctypes.c_void_p(64)  # any non-null, aligned address: never dereferenced here
+    h = ctypes.c_void_p()
+    assert L.wq_gemv_plan_create(P, None, P, P, None, 1, 512, 256, 4, 128, 0, None) == 1     # no handle slot
+    assert L.wq_gemv_plan_create(None, None, P, P, None, 1, 512, 256, 4, 128, 0, ctypes.byref(h)) == 1
+    assert h.value is None                                                                  # cleared on error
+    assert L.wq_gemv_plan_create(P, None, P, P, None, 17, 512, 256, 4, 128, 0, ctypes.byref(h)) == 1  # M > 16
+    assert L.wq_gemv_plan_create(P, None, P, P, None, 1, 512, 260, 4, 128, 0, ctypes.byref(h)) == 3   # N % 8
+    assert L.wq_gemv_plan_create(P, None, P, P, None, 1, 512, 256, 5, 128, 0, ctypes.byref(h)) == 2   # bits
+    assert L.wq_gemv_plan_create(P, None, P, P, None, 1, 512, 256, 4, 16, 0, ctypes.byref(h)) == 2    # G = 16
+    assert L.wq_gemv_plan_run(None, P, P, None) == 1
+    L.wq_gemv_plan_destroy(None)  # allowed
