@@ -29,10 +29,12 @@ x, scales, zeros, bias and the output are all ``torch.float16`` or all
 from __future__ import annotations
 
 import ctypes
+import os
 from pathlib import Path
 
 _PKG = Path(__file__).resolve().parent
-LIB_PATH = _PKG / "libwq.so"
+# WQ_LIB=checked loads the checked build (libwq_checked.so, see build.py) instead
+LIB_PATH = _PKG / ("libwq_checked.so" if os.environ.get("WQ_LIB") == "checked" else "libwq.so")
 
 STATUS = {
     0: "WQ_OK",
@@ -43,6 +45,7 @@ STATUS = {
     5: "WQ_ERR_TIMEOUT",
     6: "WQ_ERR_CUDA",
     7: "WQ_ERR_SCRATCH_LIMIT",
+    8: "WQ_ERR_CHECK",
 }
 WQ_FLAG_PDL = 1
 WQ_FLAG_PDL_INPUTS_READY = 2
@@ -98,6 +101,7 @@ def lib() -> ctypes.CDLL:
         L.wq_gemv_plan_run.restype = i
         L.wq_gemv_plan_destroy.argtypes = [p]
         L.wq_gemv_plan_destroy.restype = None
+        L.wq_checked_build.restype = i
         for f in ("wq_pack_kmajor", "wq_unpack_kmajor", "wq_gemv", "wq_gemm", "wq_device_status",
                   "wq_selftest_wait_timeout"):
             getattr(L, f).restype = i
@@ -422,8 +426,14 @@ def gemm(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out=None, pdl:
 
 
 def device_status(reset: bool = False) -> int:
-    """``wq_device_status``: 0, or 5 (WQ_ERR_TIMEOUT) if a kernel gave up a bounded wait."""
+    """``wq_device_status``: 0, 5 (WQ_ERR_TIMEOUT) if a kernel gave up a bounded
+    wait, or 8 (WQ_ERR_CHECK) if a bounds check of the checked build fired."""
     return int(lib().wq_device_status(1 if reset else 0))
+
+
+def checked_build() -> bool:
+    """Whether the loaded library is the checked build (``WQ_LIB=checked``)."""
+    return bool(lib().wq_checked_build())
 
 
 def gemm_noalloc(x, w_q, w_lo, scales, zeros, bits: int, group_size: int, out, pdl: bool = False,

@@ -88,6 +88,7 @@ const char* wq_status_string(wq_status s) {
         case WQ_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
         case WQ_ERR_CUDA: return "CUDA runtime error";
         case WQ_ERR_SCRATCH_LIMIT: return "shape needs more split-K scratch than the static array holds";
+        case WQ_ERR_CHECK: return "a bounds check of the checked build caught an access outside its array";
     }
     return "unknown status";
 }
@@ -258,6 +259,14 @@ wq_status wq_mse_search(const float* w, int rows, int cols, int group_size, int 
     return wq::launch_mse_search(w, rows, cols, group_size, bits, symmetric, steps, grid, norm, patience,
                                  scale, zero, step, err, static_cast<uint32_t*>(workspace),
                                  (cudaStream_t)stream);
+}
+
+int wq_checked_build(void) {
+#ifdef WQ_CHECKS
+    return 1;
+#else
+    return 0;
+#endif
 }
 
 wq_status wq_device_status(int reset) {

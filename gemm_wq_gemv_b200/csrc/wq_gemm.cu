@@ -68,6 +68,7 @@ struct GemmParams {
     uint32_t tmem_cols;
     uint32_t bar_off;    // offset of the barrier block from the aligned base
     uint4* ws;           // split-K slices: [tile][rank][32-token chunk][16-byte piece][128 columns]
+    size_t ws_u4;        // 16-byte units of the caller's workspace (checked build)
     int late_wait;       // wait for the previous kernel only before writing the workspace / y
 };
 
@@ -127,7 +128,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
 
     auto fail = [&]() {
         *abort_flag = 1;
-        atomicExch(&g_gemm_status, 1u);
+        atomicOr(&g_gemm_status, 1u);
     };
 
     if (warp == 0) {
@@ -315,6 +316,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
             tmem_ld_32x32b_x32(tm_row + 32 * j, v);
             tmem_ld_wait();
             uint4* dst = mine + (size_t)j * CHUNK_U4 + nl;
+            if (!check((size_t)(dst + 7 * 128 - p.ws) < p.ws_u4, &g_gemm_status)) continue;
 #pragma unroll
             for (int pc = 0; pc < 8; ++pc)
                 __stcg(dst + pc * 128, make_uint4(v[4 * pc], v[4 * pc + 1], v[4 * pc + 2], v[4 * pc + 3]));
@@ -334,6 +336,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
                 for (int src = 0; src < p.CS; ++src) {
                     if (src == rank) continue;
                     const uint4* sp = p.ws + ((tile_slot + src) * nchunks + j) * CHUNK_U4 + nl;
+                    if (!check((size_t)(sp + 7 * 128 - p.ws) < p.ws_u4, &g_gemm_status)) continue;
                     uint4 u[8];
 #pragma unroll
                     for (int pc = 0; pc < 8; ++pc) u[pc] = __ldcg(sp + pc * 128);
@@ -430,6 +433,7 @@ wq_status run(const Problem& pb, cudaStream_t stream) {
     p.CS = CS;
     p.kb_cta = (pb.K + BK - 1) / BK / CS;
     p.ws = static_cast<uint4*>(pb.ws);
+    p.ws_u4 = pb.ws_bytes / 16;
     p.late_wait = (pb.flags & WQ_FLAG_PDL_INPUTS_READY) ? 1 : 0;
 
     // stage layout: x tile | A tile | words | lo words | s rows | z rows (1024-aligned stage)
@@ -544,7 +548,7 @@ wq_status gemm_device_status(int reset) {
         const unsigned int zero = 0;
         if (cudaMemcpyToSymbol(g_gemm_status, &zero, sizeof(zero)) != cudaSuccess) return WQ_ERR_CUDA;
     }
-    return v ? WQ_ERR_TIMEOUT : WQ_OK;
+    return (v & 1u) ? WQ_ERR_TIMEOUT : (v & 2u) ? WQ_ERR_CHECK : WQ_OK;
 }
 
 }  // namespace wq

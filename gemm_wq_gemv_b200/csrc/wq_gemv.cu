@@ -222,7 +222,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
             const uint16_t* src = p.x + (size_t)m * p.K + k0;
 #pragma unroll
             for (int w = 0; w < UPC; ++w) v[u][w] = make_uint4(0, 0, 0, 0);
-            if (c < nchunk) {
+            if (c < nchunk && check(m < p.M, &g_gemv_status)) {
                 if constexpr (EPS >= 8) {
                     if (k0 < p.K) {
 #pragma unroll
@@ -278,7 +278,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     };
     auto table = [&]() {
         const bool good = mbar_wait_bounded(bar_sz, 0, WAIT_NS);
-        if (!good) atomicExch(&g_gemv_status, 1u);
+        if (!good) atomicOr(&g_gemv_status, 1u);
         if (good) tab_build();
     };
     // ---- (3) the records, and x.  x may come from the previous kernel on the
@@ -507,7 +507,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
 
         for (int kst = 0; kst < nst_w; ++kst) {
             const bool good = mbar_wait_bounded(&bar[kst & (nst - 1)], (kst / nst) & 1, WAIT_NS);
-            if (!good) atomicExch(&g_gemv_status, 1u);
+            if (!good) atomicOr(&g_gemv_status, 1u);
             if (!__all_sync(0xffffffffu, good)) break;  // give up this warp's range
             const uint32_t stage = st0 + (kst & (nst - 1)) * SB;
             const int i0 = kst * SQ;
@@ -566,7 +566,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
             float sacc = 0.0f;
             for (int r = 0; r < p.CS; ++r) sacc += ld_shared_cluster_f32(map_shared_rank(part_addr + 4u * i, r));
             const int m = i / COLS, col = col0 + i % COLS;
-            if (col < p.N) {
+            if (col < p.N && check(m < p.M, &g_gemv_status)) {
                 const float b = p.bias ? T16::load(p.bias[col]) : 0.0f;
                 p.y[(size_t)m * p.N + col] = T16::store(sacc + b);
             }
@@ -577,7 +577,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
         for (int i = threadIdx.x; i < p.M * COLS; i += blockDim.x) {
             const float sacc = sum_warps(red, p.WK, p.M * COLS, i);
             const int m = i / COLS, col = col0 + i % COLS;
-            if (col < p.N) {
+            if (col < p.N && check(m < p.M, &g_gemv_status)) {
                 const float b = p.bias ? T16::load(p.bias[col]) : 0.0f;
                 p.y[(size_t)m * p.N + col] = T16::store(sacc + b);
             }
@@ -802,7 +802,7 @@ wq_status gemv_device_status(int reset) {
         const unsigned int zero = 0;
         if (cudaMemcpyToSymbol(g_gemv_status, &zero, sizeof(zero)) != cudaSuccess) return WQ_ERR_CUDA;
     }
-    return v ? WQ_ERR_TIMEOUT : WQ_OK;
+    return (v & 1u) ? WQ_ERR_TIMEOUT : (v & 2u) ? WQ_ERR_CHECK : WQ_OK;
 }
 
 namespace {

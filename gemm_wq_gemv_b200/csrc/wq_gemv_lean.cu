@@ -229,10 +229,14 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
     // fractional is settled once, from the z rows in shared memory, and the
     // main loop is compiled for each case.
     bool ok_all = mbar_wait_bounded(bar_sz, 0, LWAIT_NS);
-    if (!ok_all) atomicExch(&g_gemv_lean_status, 1u);
+    if (!ok_all) atomicOr(&g_gemv_lean_status, 1u);
     ok_all = __all_sync(0xffffffffu, ok_all);
     const uint32_t sz_lane = sz_base + 2u * (uint32_t)(4 * cg);
-    auto sz_addr = [&](int gi) { return sz_lane + (LCOLS * 2u) * (uint32_t)(gi - g_cta0); };
+    auto sz_addr = [&](int gi) {
+        // the group's s / z row is one of the rows the CTA loaded
+        if (!check(gi >= g_cta0 && gi - g_cta0 < p.sz_rows, &g_gemv_lean_status)) gi = g_cta0;
+        return sz_lane + (LCOLS * 2u) * (uint32_t)(gi - g_cta0);
+    };
     int gcur = gdiv(q_begin);
     // whether any zero point of the warp's groups is fractional (a warp vote)
     bool frac = false;
@@ -271,7 +275,8 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
             const int kk = kc0 + 8 * o;
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
             if (kk < p.K) v = *reinterpret_cast<const uint4*>(p.x + (size_t)m * p.K + kk);  // K % 8 == 0
-            *reinterpret_cast<uint4*>(smem + p.off_x + (size_t)m * p.xs_stride + 16 * o) = v;
+            if (check(m < p.M && 16u * (uint32_t)o + 16u <= p.xs_stride, &g_gemv_lean_status))
+                *reinterpret_cast<uint4*>(smem + p.off_x + (size_t)m * p.xs_stride + 16 * o) = v;
         }
         __syncthreads();
     }
@@ -282,6 +287,12 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
                      2u * (uint32_t)(kx0 - kc0);
     // this lane's x values (token tile n) of quad i of the warp's range (all of its rows inside K)
     auto ldx = [&](int i, int n) {
+        if constexpr (CHECKED) {  // the row lies inside K (and, staged, inside the CTA's slice)
+            const int kl = kx0 + 4 * EPS * i;
+            const bool ok = XS ? (kl - kc0 + EPS <= LWK * p.QW * 4 * EPS && (uint32_t)(kl - kc0 + EPS) * 2u <= p.xs_stride)
+                               : (kl + EPS <= p.K);
+            if (!check(ok, &g_gemv_lean_status)) return make_uint4(0u, 0u, 0u, 0u);
+        }
         if constexpr (XS) {
             if constexpr (EPS == 8) return lds128_u32(xs_lane[n] + 64u * i);
             const uint2 v = lds64_u32(xs_lane[n] + 32u * i);
@@ -419,7 +430,7 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
         if constexpr (ALIGNED) {
             if (ok_all && nq > 0) {
                 const bool good = mbar_wait_bounded(&bar[0], 0u, LWAIT_NS);
-                if (!good) atomicExch(&g_gemv_lean_status, 1u);
+                if (!good) atomicOr(&g_gemv_lean_status, 1u);
                 ok_all = __all_sync(0xffffffffu, good);
             }
             if (!ok_all || nq == 0) return;
@@ -443,7 +454,7 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
             for (int b = 0; b < nbox && ok_all; ++b) {
                 const int slot = b & (S - 1);
                 const bool good = mbar_wait_bounded(&bar[slot], (uint32_t)((b / S) & 1), LWAIT_NS);
-                if (!good) atomicExch(&g_gemv_lean_status, 1u);
+                if (!good) atomicOr(&g_gemv_lean_status, 1u);
                 if (!__all_sync(0xffffffffu, good)) {  // give up this warp's range
                     ok_all = false;
                     break;
@@ -499,7 +510,8 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
 #pragma unroll
                 for (int e = 0; e < NE; ++e) {
                     const int m = 8 * n + 2 * t + e;
-                    if (m < p.M) red[m * LCOLS + 4 * cg + c] = acc[c][n][e];
+                    if (m < p.M && check((uint32_t)(m * LCOLS + LCOLS) * 4u <= S * BOX_BYTES, &g_gemv_lean_status))
+                        red[m * LCOLS + 4 * cg + c] = acc[c][n][e];
                 }
     }
     __syncthreads();
@@ -515,7 +527,7 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
     };
     auto store = [&](int i, float v) {
         const int m = i / LCOLS, col = col0 + i % LCOLS;
-        if (col < p.N) {
+        if (col < p.N && check(m < p.M, &g_gemv_lean_status)) {
             const float bv = p.bias ? T16::load(p.bias[col]) : 0.0f;
             p.y[(size_t)m * p.N + col] = T16::store(v + bv);
         }
@@ -709,7 +721,7 @@ wq_status gemv_lean_device_status(int reset) {
         const unsigned int zero = 0;
         if (cudaMemcpyToSymbol(g_gemv_lean_status, &zero, sizeof(zero)) != cudaSuccess) return WQ_ERR_CUDA;
     }
-    return v ? WQ_ERR_TIMEOUT : WQ_OK;
+    return (v & 1u) ? WQ_ERR_TIMEOUT : (v & 2u) ? WQ_ERR_CHECK : WQ_OK;
 }
 
 bool gemv_lean_takes(const Problem& p) {

@@ -16,6 +16,22 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 // ---------------------------------------------------------------- global loads
 
 // 64-bit L2 cache policy that marks lines for early eviction (streamed data).
+// Checked build (WQ_CHECKS): check(ok, word) records a failed bounds check as
+// bit 1 of a kernel file's status word and returns false, so that the caller
+// skips the access; in the normal build it is true and costs nothing.
+#ifdef WQ_CHECKS
+constexpr bool CHECKED = true;
+#else
+constexpr bool CHECKED = false;
+#endif
+__device__ __forceinline__ bool check(bool ok, unsigned int* word) {
+    if constexpr (CHECKED) {
+        if (!ok) atomicOr(word, 2u);
+        return ok;
+    }
+    return true;
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

@@ -60,7 +60,9 @@ typedef enum {
     WQ_ERR_CODE_RANGE = 4,    /* a code >= 2^bits was found (reported by the bindings) */
     WQ_ERR_TIMEOUT = 5,       /* a kernel gave up a bounded wait (see wq_device_status) */
     WQ_ERR_CUDA = 6,          /* the CUDA runtime refused a launch or query */
-    WQ_ERR_SCRATCH_LIMIT = 7  /* the shape needs more split-K scratch than wq_gemm_noalloc holds */
+    WQ_ERR_SCRATCH_LIMIT = 7, /* the shape needs more split-K scratch than wq_gemm_noalloc holds */
+    WQ_ERR_CHECK = 8          /* checked build only: a kernel's bounds check caught an access outside
+                                 its array and skipped it (see wq_device_status) */
 } wq_status;
 
 /*
@@ -322,9 +324,22 @@ void wq_gemv_plan_destroy(wq_gemv_plan* plan);
 /*
  * Device-side status of the current device: WQ_OK, or WQ_ERR_TIMEOUT when a
  * kernel on this device gave up a bounded wait since the last reset (its
- * output is then incomplete).  Synchronises the device.  reset != 0 clears it.
+ * output is then incomplete), or WQ_ERR_CHECK when a bounds check of the
+ * checked build fired.  Synchronises the device.  reset != 0 clears it.
  */
 wq_status wq_device_status(int reset);
+
+/*
+ * 1 if this library is the checked build (compiled with WQ_CHECKS, as
+ * libwq_checked.so), else 0.  Host-only.  In the checked build every kernel
+ * checks the index of each global and shared-memory access it computes itself
+ * (x, y, the split-K workspace, the s/z rows and the staging buffers; the TMA
+ * copies are bounded by their descriptors) against the array it belongs to;
+ * an access that fails is skipped and recorded, and wq_device_status then
+ * returns WQ_ERR_CHECK (after WQ_ERR_TIMEOUT, which it reports first).  It is
+ * the stand-in for a memory checker: slower, for tests.
+ */
+int wq_checked_build(void);
 
 /*
  * Failure-detection self-test (the pages have no counterpart).  Every mbarrier

@@ -17,11 +17,24 @@ def orc():
 
 @pytest.fixture(scope="session")
 def libwq():
-    """libwq.so, built in-tree if it is missing or older than its sources."""
+    """libwq.so, built in-tree if it is missing or older than its sources
+    (with WQ_LIB=checked: the checked build, libwq_checked.so)."""
+    import os
     from gemm_wq_gemv_b200 import build
-    build.build()
+    build.build(checks=os.environ.get("WQ_LIB") == "checked")
     import gemm_wq_gemv_b200 as wq
     return wq
+
+
+@pytest.fixture(autouse=True)
+def no_bounds_check_fired(request):
+    """Under the checked build, every GPU test ends with no bounds check fired."""
+    import os
+    yield
+    if os.environ.get("WQ_LIB") == "checked" and request.node.get_closest_marker("gpu"):
+        import gemm_wq_gemv_b200 as wq
+        st = wq.device_status(reset=True)
+        assert st in (0, 5), f"a bounds check of the checked build fired (status {st})"
 
 
 @pytest.fixture(scope="session")

@@ -31,8 +31,9 @@ def test_every_declared_symbol_is_exported(libwq):
 def test_version_and_strings(libwq):
     L = libwq.lib()
     assert L.wq_abi_version() == 3
-    for s in range(7):
-        assert L.wq_status_string(s)
+    for s in range(9):
+        assert L.wq_status_string(s) and L.wq_status_string(s) != b"unknown status"
+    assert L.wq_checked_build() in (0, 1)
     assert L.wq_status_string(99) == b"unknown status"
 
 
