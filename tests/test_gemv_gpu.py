@@ -50,6 +50,10 @@ SHAPES = [
     (16, 3072, 48, 3, -1),
     (4, 8192, 16, 4, 128),    # long K per column block: many quads per warp
     (16, 256, 4096, 4, 128),  # wide N, short K
+    (16, 8192, 64, 4, 128),   # two token tiles, K split over a cluster
+    (13, 4096, 128, 8, 256),  # 8-bit, two token tiles, ragged token count
+    (16, 2048, 96, 8, -1),    # 8-bit per channel, two token tiles
+    (9, 1056, 40, 4, 32),     # 33 quads over 8 warps, G = 32: one group per quad
 ]
 
 
