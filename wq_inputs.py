@@ -121,3 +121,22 @@ def bias_vector(N: int, seed: int, dtype: str = "fp16") -> np.ndarray:
     """A fused-bias vector ``(N,)`` ~ U[-1, 1]."""
     rng = np.random.default_rng(seed)
     return _as(rng.uniform(-1.0, 1.0, size=N), dtype)
+
+
+def gptq_problem(rows: int, cols: int, seed: int = 42):
+    """The GPTQ benchmark's synthetic problem ("benchmark GPTQ implementations"
+    page, ``make_inputs``): W (rows x cols) fp32 drawn as a linear layer's
+    default initialisation, U[-1/sqrt(cols), 1/sqrt(cols)], and the positive
+    definite Hessian H = A A^T + I (cols x cols, fp32) with A ~ N(0, 1).
+
+    One ``default_rng(seed)`` stream: W first, then A.  H is formed in fp64
+    and rounded to fp32 once (the page forms it in fp32 on the device; the
+    rounding of the input does not matter to parity, both sides get these
+    bytes)."""
+    rng = np.random.default_rng(seed)
+    bound = 1.0 / np.sqrt(cols)
+    W = rng.uniform(-bound, bound, size=(rows, cols)).astype(np.float32)
+    A = rng.standard_normal((cols, cols)).astype(np.float32).astype(np.float64)
+    H = A @ A.T
+    H[np.arange(cols), np.arange(cols)] += 1.0
+    return W, H.astype(np.float32)
