@@ -54,6 +54,8 @@ SHAPES = [
     (13, 4096, 128, 8, 256),  # 8-bit, two token tiles, ragged token count
     (16, 2048, 96, 8, -1),    # 8-bit per channel, two token tiles
     (9, 1056, 40, 4, 32),     # 33 quads over 8 warps, G = 32: one group per quad
+    (1, 4096, 4104, 4, 128),  # the one-token decode kernel, ragged last column block
+    (1, 2048, 4096, 4, 128),  # the one-token decode kernel, 8 quads per warp
 ]
 
 
@@ -256,7 +258,8 @@ def test_rejected_calls(cuda, libwq):
 # of 8 CTAs, 8 quads per warp; 4096 x 4096 takes one CTA per column block, 16
 # quads per warp (G = 256: two 4-quad blocks per group).  G = -1 is one group
 # across the range.
-ALIGNED = [(3, 16384, 64, 4, 128), (1, 16384, 64, 4, -1), (2, 8192, 64, 8, 128), (1, 4096, 4096, 4, 256)]
+ALIGNED = [(3, 16384, 64, 4, 128), (1, 16384, 64, 4, -1), (2, 8192, 64, 8, 128), (1, 4096, 4096, 4, 256),
+           (1, 4096, 4096, 4, 128), (1, 2048, 2560, 4, 128)]  # the last two: the one-token decode kernel
 
 
 @pytest.mark.parametrize("M,K,N,bits,G", ALIGNED)
