@@ -42,7 +42,7 @@ import wq_inputs  # noqa: E402
 HEADLINE = "decode_gemv_m1"
 GEMM_WL = "prefill_gemm"
 # the kernels those two launch, as ncu names them (spaces as underscores)
-HEADLINE_KERNEL = "gemv_lean_kernel<4,_0,_16,_1,_1,_0>"
+HEADLINE_KERNEL = "gemv_decode_kernel<16>"
 GEMM_KERNEL = "gemm_kernel<4,_0,_1>"
 METRIC = "packed-int GEMV HBM GB/s and % of peak at M=1; wq_gemm TFLOPS at M=512"
 FALLBACK_HBM, FALLBACK_TF = 6650.0, 1590.0
@@ -143,17 +143,16 @@ def job_rate(units_per_step: float, steps: int, world: int, elapsed_s: float) ->
 
 # ------------------------------------------------------------------ helpers
 # Sources that no timed kernel is built from (the failure-path self-test).
-DIGEST_EXCLUDE = {"wq_selftest.cu"}
+# the device code of the timed kernels (the decode GEMV and the prefill GEMM)
+DIGEST_SOURCES = ("wq_gemv_lean.cu", "wq_gemm.cu", "wq_ptx.cuh", "wq_dequant.cuh")
 
 
 def src_digest() -> str:
-    """Digest of the sources the timed kernels are built from: an ncu figure
-    taken on other sources does not count for this build."""
+    """Digest of the files the timed kernels' device code is built from: an ncu
+    figure taken on other kernel sources does not count for this build."""
     h = hashlib.sha1()
-    for f in sorted((ROOT / "gemm_wq_gemv_b200" / "csrc").glob("*")):
-        if f.name in DIGEST_EXCLUDE:
-            continue
-        h.update(f.read_bytes())
+    for name in DIGEST_SOURCES:
+        h.update((ROOT / "gemm_wq_gemv_b200" / "csrc" / name).read_bytes())
     return h.hexdigest()[:12]
 
 
@@ -359,6 +358,70 @@ def mse_bench(wq, torch, dev, reps: int = 5):
     return out
 
 
+def gptq_bench(wq, torch, dev, reps: int = 3):
+    """Times wq_gptq_quantize on the GPTQ page's benchmark problem: W 8192 x 8192
+    fp32 drawn like an nn.Linear initialisation, H = A A^T + I (A ~ N(0, 1)),
+    symmetric 8-bit arguments with groups of 128 (absolute-maximum scales),
+    blocks of 128, percdamp 0.01; and the oracle (NumPy fp32) on a 2048 x 2048
+    problem of the same recipe, beside the CUDA path on that problem."""
+    import numpy as np
+
+    def problem(n, seed):
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(seed)
+        w = (torch.rand((n, n), generator=gen, device=dev) * 2 - 1) / float(np.sqrt(n))
+        a = torch.randn((n, n), generator=gen, device=dev)
+        prev = torch.backends.cuda.matmul.allow_tf32
+        torch.backends.cuda.matmul.allow_tf32 = False  # the page's fp32 Hessian, not TF32
+        h = a @ a.T
+        torch.backends.cuda.matmul.allow_tf32 = prev
+        h += torch.eye(n, device=dev)
+        s = (w.abs().reshape(n, n // 128, 128).amax(-1) / 127.5).contiguous()
+        return w, h, s, torch.zeros_like(s)
+
+    def timed(n, k):
+        w, h, s, z = problem(n, 42)
+        wq.gptq_quantize(w, h, s, z, 128, 8)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(k):
+            r = wq.gptq_quantize(w, h, s, z, 128, 8)
+        e1.record()
+        torch.cuda.synchronize()
+        if wq.device_status() != 0:
+            raise RuntimeError("wq_gptq_quantize reported a device status")
+        return e0.elapsed_time(e1) / k, (w, h, s, z, r)
+
+    n = 8192
+    ms, _ = timed(n, reps)
+    flops = n ** 3 / 3 + n * n * n  # one Cholesky factorisation + the column updates (R C^2)
+    peak = 148 * 128 * 2 * 1.965e9 / 1e12  # fp32 FMA lanes x 2 flop x max SM clock, TFLOP/s
+    out = {"workload": f"W {n}x{n} fp32, H = A A^T + I, symmetric 8-bit, group 128, blocks of 128, "
+                       "percdamp 0.01 (the GPTQ page's benchmark defaults)",
+           "ms": round(ms, 3),
+           "roofline": {"bound": "alu", "achieved": round(flops / (ms * 1e-3) / 1e12, 2), "peak": round(peak, 1),
+                        "unit": "TFLOP/s", "frac": round(flops / (ms * 1e-3) / 1e12 / peak, 4),
+                        "flops": "C^3/3 (one Cholesky) + R C^2 (each column's error times every later column)",
+                        "peak_how": "148 SMs x 128 fp32 FMA lanes x 2 x 1965 MHz"},
+           "page_context": "the page prints 135 ms for its Triton variant (2191 ms eager) on its own, unnamed GPU"}
+    small = 2048
+    ms_small, (w, h, s, z, r) = timed(small, reps)
+    from oracle import gptq as og
+    W, H, S, Z = (t.cpu().numpy() for t in (w, h, s, z))
+    t0 = time.perf_counter()
+    ref = og.quantize_weight(W, H, S, Z, 128, 8)
+    el = time.perf_counter() - t0
+    agree = float(np.mean(r["codes"].cpu().numpy().T.astype(np.int32) - 128 == ref["codes"]))
+    out["small"] = {"workload": f"{small}x{small}, same recipe", "ms": round(ms_small, 3),
+                    "codes_equal_to_oracle": round(agree, 6)}
+    out["cpu_baseline"] = {"ms": round(el * 1e3, 1), "kind": "oracle", "cores": os.cpu_count(),
+                           "sample": f"the whole {small}x{small} problem, NumPy fp32 with its BLAS/LAPACK threads"}
+    del w, h, s, z, r
+    return out
+
+
 # ------------------------------------------------------------------ reference arm
 def run_reference(args):
     """The CPU oracle timed as the reference arm, on the headline config and metric."""
@@ -409,6 +472,21 @@ def run_case(name: str, reps: int) -> int:
     wq_build.build()
     import gemm_wq_gemv_b200 as wq
     dev = torch.device("cuda", 0)
+    if name.startswith("gptq_"):  # GPTQ of an n x n problem of the page's recipe, e.g. gptq_2048
+        n = int(name.split("_")[1])
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(42)
+        w = (torch.rand((n, n), generator=gen, device=dev) * 2 - 1) / float(n) ** 0.5
+        a = torch.randn((n, n), generator=gen, device=dev)
+        torch.backends.cuda.matmul.allow_tf32 = False
+        h = a @ a.T + torch.eye(n, device=dev)
+        s = (w.abs().reshape(n, -1, 128).amax(-1) / 127.5).contiguous()
+        for _ in range(reps):
+            wq.gptq_quantize(w, h, s, torch.zeros_like(s), 128, 8)
+        torch.cuda.synchronize()
+        assert wq.device_status() == 0
+        print(json.dumps({"case": name, "reps": reps, "kernel": "gptq"}))
+        return 0
     wl = wq_inputs.WORKLOADS[name]
     stack = Stack(wq, torch, wl, 1, dev)
     fn = wq.gemv if wl.M <= 16 else wq.gemm
@@ -607,6 +685,12 @@ def main(argv=None):
     if not args.no_secondary:
         mse = mse_bench(wq, torch, dev)
 
+    # ---- GPTQ block quantisation (the step that chooses the codes) on the page's
+    # benchmark problem
+    gq = None
+    if not args.no_secondary:
+        gq = gptq_bench(wq, torch, dev)
+
     # ---- every workload once (rank-local, for the table)
     table = []
     if not args.no_secondary:
@@ -675,6 +759,7 @@ def main(argv=None):
         "gpu_launches": args.steps * L * world,
         "workloads": table,
         "mse_search": mse,
+        "gptq": gq,
         "source": src_digest(),
     }
     if rank == 0 and world == 1:

@@ -46,6 +46,7 @@ STATUS = {
     6: "WQ_ERR_CUDA",
     7: "WQ_ERR_SCRATCH_LIMIT",
     8: "WQ_ERR_CHECK",
+    9: "WQ_ERR_NOT_POSITIVE_DEFINITE",
 }
 WQ_FLAG_PDL = 1
 WQ_FLAG_PDL_INPUTS_READY = 2
@@ -102,6 +103,10 @@ def lib() -> ctypes.CDLL:
         L.wq_gemv_plan_destroy.argtypes = [p]
         L.wq_gemv_plan_destroy.restype = None
         L.wq_checked_build.restype = i
+        L.wq_gptq_workspace_size.argtypes = [i, i]
+        L.wq_gptq_workspace_size.restype = ctypes.c_size_t
+        L.wq_gptq_quantize.argtypes = [p, p, p, p, i, i, i, i, i, ctypes.c_float, p, p, p, p, ctypes.c_size_t, p]
+        L.wq_gptq_quantize.restype = i
         for f in ("wq_pack_kmajor", "wq_unpack_kmajor", "wq_gemv", "wq_gemm", "wq_device_status",
                   "wq_selftest_wait_timeout"):
             getattr(L, f).restype = i
@@ -497,6 +502,48 @@ def mse_search(w, bits: int, group_size: int, maxshrink: float = 0.2, grid: int 
                              float(norm), pat, _ptr(out["scale"]), _ptr(out["zero"]), _ptr(out["step"]),
                              _ptr(out["err"]), _ptr(ws), 4 if ws is not None else 0, _stream())
     _check("wq_mse_search", st)
+    return out
+
+
+def gptq_quantize(W, H, scale, zero, group_size: int, bits: int, blocksize: int = 128,
+                  percdamp: float = 0.01, want_q: bool = True, want_codes: bool = True):
+    """``wq_gptq_quantize``: GPTQ block quantisation of ``W`` (rows, cols) with
+    the Hessian ``H`` (cols, cols), on the current stream, in fp32.
+
+    ``scale`` / ``zero``: (rows, ceil(cols / group_size)) float32, the zero
+    points on the signed scale (0 for symmetric arguments).  Returns a dict:
+    ``Q`` (rows, cols) float32, the fake-quantised W; ``codes`` (cols, rows)
+    uint8, ``q + 2**(bits-1)``, the K-major codes ``pack_kmajor`` takes;
+    ``losses`` (rows,) float32.  A Hessian that is not positive definite shows
+    as ``device_status() == 9`` and NaN outputs."""
+    torch = _torch()
+    _need(W, torch.float32, "W")
+    _need(H, torch.float32, "H")
+    _need(scale, torch.float32, "scale")
+    _need(zero, torch.float32, "zero")
+    _same_device(W, H=H, scale=scale, zero=zero)
+    rows, cols = W.shape
+    if tuple(H.shape) != (cols, cols):
+        raise ValueError(f"H has shape {tuple(H.shape)}, expected {(cols, cols)}")
+    if group_size < 1:
+        raise ValueError("group_size must be at least 1")
+    ng = -(-cols // group_size)
+    for name, t in (("scale", scale), ("zero", zero)):
+        if tuple(t.shape) != (rows, ng):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {(rows, ng)}")
+    dev = W.device
+    out = {"losses": torch.empty(rows, dtype=torch.float32, device=dev)}
+    out["Q"] = torch.empty((rows, cols), dtype=torch.float32, device=dev) if want_q else None
+    out["codes"] = torch.empty((cols, rows), dtype=torch.uint8, device=dev) if want_codes else None
+    nbytes = lib().wq_gptq_workspace_size(rows, cols)
+    if nbytes == 0:
+        raise ValueError(f"unsupported shape ({rows}, {cols})")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    st = lib().wq_gptq_quantize(_ptr(W), _ptr(H), _ptr(scale), _ptr(zero), rows, cols, group_size, bits,
+                                blocksize, float(percdamp), _ptr(out["Q"]), _ptr(out["codes"]),
+                                _ptr(out["losses"]), _ptr(ws), nbytes, _stream())
+    _check("wq_gptq_quantize", st)
+    out["workspace"] = ws  # kept alive until the caller drops the result
     return out
 
 

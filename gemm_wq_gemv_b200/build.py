@@ -25,7 +25,7 @@ LIB = PKG / "libwq.so"
 LIB_CHECKED = PKG / "libwq_checked.so"
 BUILD = ROOT / "_build"
 SOURCES = ["wq_abi.cu", "wq_host.cu", "wq_pack.cu", "wq_gemv.cu", "wq_gemv_lean.cu", "wq_gemm.cu",
-           "wq_noalloc.cu", "wq_mse.cu", "wq_selftest.cu"]
+           "wq_noalloc.cu", "wq_mse.cu", "wq_gptq.cu", "wq_selftest.cu"]
 HEADERS = ["wq_internal.h", "wq_ptx.cuh", "wq_dequant.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

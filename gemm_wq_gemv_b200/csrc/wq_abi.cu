@@ -89,6 +89,7 @@ const char* wq_status_string(wq_status s) {
         case WQ_ERR_CUDA: return "CUDA runtime error";
         case WQ_ERR_SCRATCH_LIMIT: return "shape needs more split-K scratch than the static array holds";
         case WQ_ERR_CHECK: return "a bounds check of the checked build caught an access outside its array";
+        case WQ_ERR_NOT_POSITIVE_DEFINITE: return "the damped Hessian is not positive definite";
     }
     return "unknown status";
 }
@@ -261,6 +262,31 @@ wq_status wq_mse_search(const float* w, int rows, int cols, int group_size, int 
                                  (cudaStream_t)stream);
 }
 
+size_t wq_gptq_workspace_size(int rows, int cols) {
+    if (rows < 1 || cols < 1 || cols > 65536) return 0;
+    return wq::gptq_workspace_bytes(rows, cols);
+}
+
+wq_status wq_gptq_quantize(const float* W, const float* H, const float* scale, const float* zero, int rows,
+                           int cols, int group_size, int bits, int blocksize, float percdamp, float* Q,
+                           uint8_t* codes, float* losses, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+    if (bits < 1 || bits > 8) return WQ_ERR_UNSUPPORTED;
+    if (rows < 1 || cols < 1 || cols > 65536 || group_size < 1 || blocksize < 1 || blocksize > 128)
+        return WQ_ERR_INVALID_ARG;
+    if ((size_t)rows * (size_t)cols > ((size_t)1 << 40)) return WQ_ERR_INVALID_ARG;
+    if (!(percdamp >= 0.0f) || !(percdamp < 1.0e30f)) return WQ_ERR_INVALID_ARG;  // rejects NaN
+    if (!W || !H || !scale || !zero || !losses || !workspace) return WQ_ERR_INVALID_ARG;
+    if (workspace_bytes < wq::gptq_workspace_bytes(rows, cols)) return WQ_ERR_INVALID_ARG;
+    if (!aligned(W, 4) || !aligned(H, 4) || !aligned(scale, 4) || !aligned(zero, 4) || !aligned(losses, 4) ||
+        (Q && !aligned(Q, 4)) || !aligned(workspace, 256))
+        return WQ_ERR_ALIGNMENT;
+    wq_status st = check_device();
+    if (st != WQ_OK) return st;
+    return wq::launch_gptq(W, H, scale, zero, rows, cols, group_size, bits, blocksize, percdamp, Q, codes, losses,
+                           workspace, (cudaStream_t)stream);
+}
+
 int wq_checked_build(void) {
 #ifdef WQ_CHECKS
     return 1;
@@ -273,8 +299,11 @@ wq_status wq_device_status(int reset) {
     const wq_status a = wq::gemm_device_status(reset);
     const wq_status b = wq::gemv_device_status(reset);
     const wq_status c = wq::gemv_lean_device_status(reset);
-    if (a == WQ_ERR_CUDA || b == WQ_ERR_CUDA || c == WQ_ERR_CUDA) return WQ_ERR_CUDA;
-    return (a != WQ_OK) ? a : (b != WQ_OK) ? b : c;
+    const wq_status d = wq::gptq_device_status(reset);
+    if (a == WQ_ERR_CUDA || b == WQ_ERR_CUDA || c == WQ_ERR_CUDA || d == WQ_ERR_CUDA) return WQ_ERR_CUDA;
+    for (const wq_status e : {WQ_ERR_TIMEOUT, WQ_ERR_CHECK})
+        if (a == e || b == e || c == e) return e;
+    return d;
 }
 
 }  // extern "C"

@@ -68,6 +68,13 @@ wq_status launch_mse_search(const float* w, int rows, int cols, int group_size, 
 wq_status gemm_device_status(int reset);
 wq_status gemv_device_status(int reset);
 wq_status gemv_lean_device_status(int reset);
+wq_status gptq_device_status(int reset);
+
+// GPTQ block quantisation (wq_gptq.cu), arguments already validated.
+size_t gptq_workspace_bytes(int R, int C);
+wq_status launch_gptq(const float* W, const float* H, const float* scale, const float* zero, int R, int C, int G,
+                      int bits, int blocksize, float percdamp, float* Q, uint8_t* codes, float* losses,
+                      void* workspace, cudaStream_t s);
 
 // 2-D tiled TMA descriptor for a row-major (outer, inner) array.
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t outer,

@@ -61,8 +61,10 @@ typedef enum {
     WQ_ERR_TIMEOUT = 5,       /* a kernel gave up a bounded wait (see wq_device_status) */
     WQ_ERR_CUDA = 6,          /* the CUDA runtime refused a launch or query */
     WQ_ERR_SCRATCH_LIMIT = 7, /* the shape needs more split-K scratch than wq_gemm_noalloc holds */
-    WQ_ERR_CHECK = 8          /* checked build only: a kernel's bounds check caught an access outside
+    WQ_ERR_CHECK = 8,         /* checked build only: a kernel's bounds check caught an access outside
                                  its array and skipped it (see wq_device_status) */
+    WQ_ERR_NOT_POSITIVE_DEFINITE = 9 /* wq_gptq_quantize: the damped Hessian has a pivot <= 0
+                                        (see wq_device_status) */
 } wq_status;
 
 /*
@@ -294,6 +296,51 @@ wq_status wq_mse_search(const float* w, int rows, int cols, int group_size, int 
                         void* stream);
 
 /*
+ * GPTQ block quantisation ("benchmark GPTQ implementations" page:
+ * _prepare_weight_and_hessian, quantize_weight_eager with the GROUP strategy,
+ * and the fake quantisation of _quantize_block_triton_kernel), in fp32 as the
+ * page fixes it.  The producer of the codes that wq_pack_kmajor packs.
+ *
+ * W (rows x cols, row-major, one row per output channel) and the Hessian H
+ * (cols x cols, symmetric, row-major).  Columns c with H[c][c] == 0 are dead:
+ * H[c][c] = 1 and W[:, c] = 0.  damp = percdamp * mean(diag H) is added to the
+ * diagonal.  Column c takes group g = c / group_size and the fp32 parameters
+ * scale[r][g], zero[r][g] (rows x ceil(cols / group_size), row-major; zero
+ * points on the page's signed scale, 0 for symmetric arguments).  Columns are
+ * quantised from left to right in blocks of `blocksize`:
+ *   q = clamp(rint(w / s) + z, -2^(bits-1), 2^(bits-1) - 1), w_hat = (q - z) s,
+ * with w the column's current value, and the error is spread over the later
+ * columns through the upper Cholesky factor of the inverse damped Hessian.
+ *
+ * Outputs (device, written on `stream`):
+ *   Q      rows x cols fp32, row-major: the fake-quantised W (the page's result),
+ *          or null;
+ *   codes  cols x rows uint8, K-major (the layout wq_pack_kmajor takes with
+ *          K = cols, N = rows): q + 2^(bits-1), so that the product's zero point
+ *          is z + 2^(bits-1); or null;
+ *   losses rows fp32: half the sum of each row's loss terms (the page's
+ *          `losses`; its `loss` is their sum).
+ * workspace: wq_gptq_workspace_size(rows, cols) bytes of device memory, 256-byte
+ *   aligned, owned by the caller, not read before written; it must not be used
+ *   by anything else until the call's work on `stream` is done.
+ *
+ * Arguments: rows, cols >= 1 (cols <= 65536), 1 <= group_size, bits 1..8,
+ * 1 <= blocksize <= 128 (the page's benchmark uses 128; in exact arithmetic
+ * the result does not depend on it), 0 <= percdamp < 1e30 (else
+ * WQ_ERR_INVALID_ARG / WQ_ERR_UNSUPPORTED for bits).  Float arrays 4-byte
+ * aligned (else WQ_ERR_ALIGNMENT).  Scales must be nonzero.
+ *
+ * A damped Hessian that is not positive definite sets the device status read
+ * by wq_device_status (WQ_ERR_NOT_POSITIVE_DEFINITE); the outputs are then
+ * NaN.  Asynchronous on `stream`; H and W are only read.
+ */
+size_t wq_gptq_workspace_size(int rows, int cols);
+wq_status wq_gptq_quantize(const float* W, const float* H, const float* scale, const float* zero, int rows,
+                           int cols, int group_size, int bits, int blocksize, float percdamp, float* Q,
+                           uint8_t* codes, float* losses, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/*
  * A decode product prepared once (the weights bound, x and y per call).  The
  * dashq_kernel.py page's TritonQuantLinear holds the packed weights, scales
  * and zero points as a layer and applies them to each new x; this is that
@@ -325,7 +372,8 @@ void wq_gemv_plan_destroy(wq_gemv_plan* plan);
  * Device-side status of the current device: WQ_OK, or WQ_ERR_TIMEOUT when a
  * kernel on this device gave up a bounded wait since the last reset (its
  * output is then incomplete), or WQ_ERR_CHECK when a bounds check of the
- * checked build fired.  Synchronises the device.  reset != 0 clears it.
+ * checked build fired, or WQ_ERR_NOT_POSITIVE_DEFINITE when a factorisation
+ * of wq_gptq_quantize met a pivot <= 0 (reported in that order).  Synchronises the device.  reset != 0 clears it.
  */
 wq_status wq_device_status(int reset);
 

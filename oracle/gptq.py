@@ -103,8 +103,9 @@ def quantize_weight(W, H, scale, zero, group_size: int, bits: int, blocksize: in
     ``scale`` / ``zero``: (rows, ceil(cols / group_size)); column c uses group
     ``c // group_size``.  Returns a dict: ``loss`` (float), ``losses`` (per
     row, half the sum of its loss terms), ``Q`` (fake-quantised W, rows x cols),
-    ``codes`` (signed integer codes, int32), ``W0`` (W with dead columns
-    zeroed), ``H`` (the damped Hessian) and ``Hinv``."""
+    ``codes`` (signed integer codes, int32), ``ratio`` (each column's current
+    value over its scale, the number that is rounded), ``W0`` (W with dead
+    columns zeroed), ``H`` (the damped Hessian) and ``Hinv``."""
     ft = precision
     W, Hd, Hinv = prepare(W, H, percdamp, ft)
     W0 = W.copy()
@@ -113,6 +114,7 @@ def quantize_weight(W, H, scale, zero, group_size: int, bits: int, blocksize: in
     z_all = np.asarray(zero, ft)
     qmin, qmax = qrange(bits)
     codes = np.zeros((rows, cols), np.int32)
+    ratio = np.zeros((rows, cols), ft)
     losses = np.zeros(rows, ft)
     for i1 in range(0, cols, blocksize):
         i2 = min(i1 + blocksize, cols)
@@ -128,7 +130,9 @@ def quantize_weight(W, H, scale, zero, group_size: int, bits: int, blocksize: in
             g = (i1 + i) // group_size
             s = s_all[:, g]
             zp = z_all[:, g]
-            qi = np.clip(np.rint((w / s).astype(ft)) + zp, ft(qmin), ft(qmax)).astype(ft)
+            t = (w / s).astype(ft)
+            ratio[:, i1 + i] = t
+            qi = np.clip(np.rint(t) + zp, ft(qmin), ft(qmax)).astype(ft)
             q = ((qi - zp).astype(ft) * s).astype(ft)
             codes[:, i1 + i] = qi.astype(np.int32)
             Q1[:, i] = q
@@ -140,7 +144,7 @@ def quantize_weight(W, H, scale, zero, group_size: int, bits: int, blocksize: in
         losses += (np.sum(losses1, axis=1, dtype=ft) / ft(2)).astype(ft)
         W[:, i2:] -= (Err1 @ Hinv[i1:i2, i2:]).astype(ft)
     return {"loss": float(np.sum(losses, dtype=ft)), "losses": losses, "Q": W, "codes": codes,
-            "W0": W0, "H": Hd, "Hinv": Hinv}
+            "ratio": ratio, "W0": W0, "H": Hd, "Hinv": Hinv}
 
 
 def gptq_loss_of(W, Q, Hd):

@@ -31,7 +31,7 @@ def test_every_declared_symbol_is_exported(libwq):
 def test_version_and_strings(libwq):
     L = libwq.lib()
     assert L.wq_abi_version() == 3
-    for s in range(9):
+    for s in range(10):
         assert L.wq_status_string(s) and L.wq_status_string(s) != b"unknown status"
     assert L.wq_checked_build() in (0, 1)
     assert L.wq_status_string(99) == b"unknown status"
@@ -199,6 +199,32 @@ def test_mse_search_argument_checks(libwq):
     if not torch.cuda.is_available():
         assert call() == 6                              # valid: reaches CUDA, which has no device here
         assert call(pat=5, ws=P, ws_bytes=4) == 6
+
+
+def test_gptq_argument_checks(libwq):
+    """wq_gptq_quantize rejects bad shapes, bit widths, block sizes, damping,
+    pointers and short workspaces on the host, before any launch."""
+    L = libwq.lib()
+    f = ctypes.c_float
+    need = L.wq_gptq_workspace_size(16, 256)
+    assert need >= 4 * (256 * 256 + 2 * 256 * 16)
+    assert L.wq_gptq_workspace_size(0, 256) == 0 and L.wq_gptq_workspace_size(16, 65537) == 0
+
+    def call(W=P, H=P, s=P, z=P, rows=16, cols=256, G=128, bits=8, bs=128, damp=0.01, Q=P, codes=P,
+             losses=P, ws=P, ws_bytes=None):
+        return L.wq_gptq_quantize(W, H, s, z, rows, cols, G, bits, bs, f(damp), Q, codes, losses, ws,
+                                  ctypes.c_size_t(need if ws_bytes is None else ws_bytes), None)
+    assert call(bits=0) == 2 and call(bits=9) == 2
+    assert call(rows=0) == 1 and call(cols=0) == 1 and call(cols=65537) == 1 and call(G=0) == 1
+    assert call(bs=0) == 1 and call(bs=129) == 1
+    assert call(damp=-0.1) == 1 and call(damp=float("nan")) == 1 and call(damp=float("inf")) == 1
+    assert call(W=None) == 1 and call(H=None) == 1 and call(s=None) == 1 and call(losses=None) == 1
+    assert call(ws=None) == 1 and call(ws_bytes=need - 1) == 1
+    assert call(W=P + 2) == 3 and call(ws=P + 16) == 3                # floats 4-byte, workspace 256-byte
+    import torch
+    if not torch.cuda.is_available():
+        assert call() == 6                                 # valid: reaches CUDA, which has no device here
+        assert call(Q=None, codes=None) == 6               # both outputs are optional
 
 
 def test_gemv_plan_argument_checks(libwq):

@@ -141,7 +141,7 @@ MUTANTS = {
     "lower_factor": ("quantize_weight", "Err1 @ Hinv[i1:i2, i2:]", "Err1 @ Hinv.T[i1:i2, i2:]"),
     "first_pivot": ("quantize_weight", "d = Hinv1[i, i]", "d = Hinv1[0, 0]"),
     "loss_not_halved": ("quantize_weight", "/ ft(2)", "/ ft(1)"),
-    "floor_not_round": ("quantize_weight", "np.rint((w / s)", "np.floor((w / s)"),
+    "floor_not_round": ("quantize_weight", "np.rint(t)", "np.floor(t)"),
     "group_modulo": ("quantize_weight", "(i1 + i) // group_size", "(i1 + i) % group_size"),
     "error_not_scaled": ("quantize_weight", "err1 = ((w - q) / d)", "err1 = ((w - q) * 1)"),
     "no_damp": ("prepare", "H[idx, idx] += damp", "H[idx, idx] += 0 * damp"),

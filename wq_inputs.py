@@ -129,14 +129,13 @@ def gptq_problem(rows: int, cols: int, seed: int = 42):
     default initialisation, U[-1/sqrt(cols), 1/sqrt(cols)], and the positive
     definite Hessian H = A A^T + I (cols x cols, fp32) with A ~ N(0, 1).
 
-    One ``default_rng(seed)`` stream: W first, then A.  H is formed in fp64
-    and rounded to fp32 once (the page forms it in fp32 on the device; the
-    rounding of the input does not matter to parity, both sides get these
-    bytes)."""
+    One ``default_rng(seed)`` stream: W first, then A.  H is formed in fp32,
+    as on the page (the bytes may differ between BLAS builds in the last
+    place; both sides of a comparison are given the same array)."""
     rng = np.random.default_rng(seed)
     bound = 1.0 / np.sqrt(cols)
     W = rng.uniform(-bound, bound, size=(rows, cols)).astype(np.float32)
-    A = rng.standard_normal((cols, cols)).astype(np.float32).astype(np.float64)
+    A = rng.standard_normal((cols, cols)).astype(np.float32)
     H = A @ A.T
-    H[np.arange(cols), np.arange(cols)] += 1.0
-    return W, H.astype(np.float32)
+    H[np.arange(cols), np.arange(cols)] += np.float32(1.0)
+    return W, H
