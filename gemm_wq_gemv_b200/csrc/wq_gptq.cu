@@ -137,62 +137,89 @@ __global__ void gptq_transpose_kernel(const float* __restrict__ W, const float* 
 // ---- blocked Cholesky of P (lower, in place) -------------------------------
 
 // The diagonal block at k0 (nb <= 64 wide, already updated by the earlier
-// panels): factored in shared memory, column by column, and its lower
-// triangular inverse written to Linv (nb x nb, zeros above the diagonal).
-// Thread t owns the 16 entries (t / 4, t % 4 + 4 u) of both 64 x 64 arrays.
-__global__ void __launch_bounds__(256) chol_diag_kernel(float* __restrict__ P, int C, int k0, int nb,
-                                                        float* __restrict__ Linv) {
+// panels): factored in shared memory and its lower triangular inverse written
+// to Linv (nb x nb, zeros above the diagonal).  Thread t owns row t.  The
+// factorisation eliminates without square roots (after step j, the entries
+// right of column j hold the Schur complement of the leading j + 1 columns),
+// then scales column c by 1 / sqrt(pivot c); the inverse is formed row by row
+// before the division by its diagonal.  One barrier per column; each thread's
+// row updates issue their shared-memory loads eight at a time.
+__global__ void __launch_bounds__(NB) chol_diag_kernel(float* __restrict__ P, int C, int k0, int nb,
+                                                       float* __restrict__ Linv) {
     __shared__ float A[NB][NBP];
-    __shared__ float X[NB][NBP];
-    const int tid = threadIdx.x;
-    const int oi = tid >> 2, oc = tid & 3;  // owned row, first owned column
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-        const int c = oc + 4 * u;
-        A[oi][c] = (oi < nb && c <= oi) ? P[(size_t)(k0 + oi) * C + k0 + c] : 0.0f;
-        X[oi][c] = (oi == c) ? 1.0f : 0.0f;
-    }
-    // right-looking factorisation: scale column j, then update the trailing lower triangle
-    for (int j = 0; j < nb; ++j) {
-        __syncthreads();
-        const float piv = A[j][j];
-        const float d = __fsqrt_rn(piv);  // NaN for a negative pivot
-        __syncthreads();                  // every thread has read the pivot
-        if (tid == 0 && !(piv > 0.0f)) atomicOr(&g_gptq_status, 4u);
-        if (tid < nb) A[tid][j] = (tid == j) ? d : (tid > j ? __fdiv_rn(A[tid][j], d) : A[tid][j]);
-        __syncthreads();
-        const float lij = A[oi][j];
+    __shared__ float Y[NB][NBP];
+    __shared__ float sq[NB];
+    const int t = threadIdx.x;
+    for (int i0 = 0; i0 < NB; i0 += 16) {  // thread t reads column t of 16 rows: 16 loads in flight
+        float v[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
-            const int c = oc + 4 * u;
-            if (c > j && c <= oi && oi < nb) A[oi][c] = fmaf(-lij, A[c][j], A[oi][c]);
+            const int i = i0 + u;
+            v[u] = (i < nb && t <= i) ? P[(size_t)(k0 + i) * C + k0 + t] : 0.0f;
         }
-    }
-    // X = A^-1 by right-looking forward substitution on the identity
-    for (int k = 0; k < nb; ++k) {
-        __syncthreads();
-        const float dk = A[k][k];
-        if (oi == k) {
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int c = oc + 4 * u;
-                if (c <= k) X[k][c] = __fdiv_rn(X[k][c], dk);
-            }
-        }
-        __syncthreads();
-        const float lik = A[oi][k];
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
-            const int c = oc + 4 * u;
-            if (oi > k && oi < nb && c <= k) X[oi][c] = fmaf(-lik, X[k][c], X[oi][c]);
+            A[i0 + u][t] = v[u];
+            Y[i0 + u][t] = (i0 + u == t) ? 1.0f : 0.0f;
         }
     }
     __syncthreads();
+    const bool own = t < nb;
+    for (int j = 0; j < nb; ++j) {
+        if (own && t > j) {
+            const float f = __fdiv_rn(A[t][j], A[j][j]);
+            int c = j + 1;
+            for (; c + 7 <= t; c += 8) {
+                float a[8], r[8];
 #pragma unroll
-    for (int u = 0; u < 16; ++u) {
-        const int c = oc + 4 * u;
-        if (oi < nb && c <= oi) P[(size_t)(k0 + oi) * C + k0 + c] = A[oi][c];
-        if (oi < nb && c < nb) Linv[oi * NB + c] = X[oi][c];
+                for (int u = 0; u < 8; ++u) {
+                    a[u] = A[c + u][j];
+                    r[u] = A[t][c + u];
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) A[t][c + u] = fmaf(-f, a[u], r[u]);
+            }
+            for (; c <= t; ++c) A[t][c] = fmaf(-f, A[c][j], A[t][c]);
+        }
+        __syncthreads();
+    }
+    if (own) {
+        const float piv = A[t][t];
+        if (!(piv > 0.0f)) atomicOr(&g_gptq_status, 4u);
+        sq[t] = __fsqrt_rn(piv);  // NaN for a negative pivot
+    }
+    __syncthreads();
+    if (own) {
+        for (int c = 0; c < t; ++c) A[t][c] = __fdiv_rn(A[t][c], sq[c]);
+        A[t][t] = sq[t];
+    }
+    __syncthreads();
+    // rows of A^-1 before their division by the diagonal: Y_t -= (L_tk / L_kk) Y_k
+    for (int k = 0; k < nb; ++k) {
+        if (own && t > k) {
+            const float f = __fdiv_rn(A[t][k], A[k][k]);
+            int c = 0;
+            for (; c + 7 <= k; c += 8) {
+                float yk[8], yt[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    yk[u] = Y[k][c + u];
+                    yt[u] = Y[t][c + u];
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) Y[t][c + u] = fmaf(-f, yk[u], yt[u]);
+            }
+            for (; c <= k; ++c) Y[t][c] = fmaf(-f, Y[k][c], Y[t][c]);
+        }
+        __syncthreads();
+    }
+    if (own)
+        for (int c = 0; c <= t; ++c) Y[t][c] = __fdiv_rn(Y[t][c], A[t][t]);
+    __syncthreads();
+    for (int idx = t; idx < NB * NB; idx += NB) {
+        const int i = idx / NB, c = idx % NB;
+        if (i < nb && c <= i) P[(size_t)(k0 + i) * C + k0 + c] = A[i][c];
+        if (i < nb && c < nb) Linv[i * NB + c] = (c <= i) ? Y[i][c] : 0.0f;
     }
 }
 
@@ -218,14 +245,24 @@ __global__ void __launch_bounds__(256) chol_tile_kernel(float* __restrict__ P, i
         tj = (int)blockIdx.x - ti * (ti + 1) / 2;
     }
     const int i0 = base + NB * ti, m0 = base + NB * tj;
-    for (int idx = tid; idx < NB * NB; idx += blockDim.x) {
-        const int r = idx / NB, k = idx % NB;
+    {  // 16 rows per thread, both operands: 32 loads in flight before the stores
+        const int k = tid % NB, r0 = tid / NB;  // 256 threads: 4 rows per pass
         const bool kin = k < nb;
-        As[r][k] = (kin && i0 + r < C) ? P[(size_t)(i0 + r) * C + k0 + k] : 0.0f;
-        if (PANEL)
-            Bs[r][k] = (kin && r < nb) ? Linv[r * NB + k] : 0.0f;
-        else
-            Bs[r][k] = (kin && m0 + r < C) ? P[(size_t)(m0 + r) * C + k0 + k] : 0.0f;
+        float va[16], vb[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int r = r0 + 4 * u;
+            va[u] = (kin && i0 + r < C) ? P[(size_t)(i0 + r) * C + k0 + k] : 0.0f;
+            if (PANEL)
+                vb[u] = (kin && r < nb) ? Linv[r * NB + k] : 0.0f;
+            else
+                vb[u] = (kin && m0 + r < C) ? P[(size_t)(m0 + r) * C + k0 + k] : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            As[r0 + 4 * u][k] = va[u];
+            Bs[r0 + 4 * u][k] = vb[u];
+        }
     }
     __syncthreads();
     const int ty = tid / 16, tx = tid % 16;
@@ -301,18 +338,47 @@ __global__ void __launch_bounds__(RT) gptq_block_kernel(const BlockParams p) {
     float* Vs = sm;                        // cnt * cnt
     float* la = Vs + cnt * cnt;            // cnt * RTP: w' of column j for thread t at j * RTP + t
     float* wo = la + cnt * RTP;            // cnt * RTP: original w, then w_hat
+    float* vds = wo + cnt * RTP;           // cnt: V_jj of the block's columns
     const int t = threadIdx.x;
     const int r0 = blockIdx.x * RT, r = r0 + t;
     const bool live = r < p.R;
-    for (int idx = t; idx < cnt * cnt; idx += RT) {
-        const int i = idx / cnt, j = idx % cnt;
-        Vs[idx] = (j > i) ? p.P[(size_t)(p.i1 + i) * p.C + p.i1 + j] : 0.0f;
+    {  // V' of the block: each warp 4 rows per pass, each lane 4 columns: 16 loads in flight
+        const int lane = t & 31, w = t >> 5;
+        for (int ib = w * 4; ib < cnt; ib += 4 * (RT / 32)) {
+            float v[4][4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int i = ib + a, j = lane + 32 * b;
+                    v[a][b] = (i < cnt && j < cnt && j > i) ? p.P[(size_t)(p.i1 + i) * p.C + p.i1 + j] : 0.0f;
+                }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int i = ib + a, j = lane + 32 * b;
+                    if (i < cnt && j < cnt) Vs[i * cnt + j] = v[a][b];
+                }
+        }
     }
-    for (int j = 0; j < cnt; ++j) {
-        const size_t g = (size_t)(p.i1 + j) * p.R + r;
-        const float w = live ? p.Wt[g] : 0.0f;
-        la[j * RTP + t] = live ? w + p.Acc[g] : 0.0f;
-        wo[j * RTP + t] = w;
+    for (int j = t; j < cnt; j += RT) vds[j] = p.vd[p.i1 + j];
+    for (int j0 = 0; j0 < cnt; j0 += 8) {  // the row's values: 16 loads in flight
+        float w[8], a[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const size_t g = (size_t)(p.i1 + j0 + u) * p.R + r;
+            const bool in = live && j0 + u < cnt;
+            w[u] = in ? p.Wt[g] : 0.0f;
+            a[u] = in ? p.Acc[g] : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (j0 + u < cnt) {
+                la[(j0 + u) * RTP + t] = w[u] + a[u];
+                wo[(j0 + u) * RTP + t] = w[u];
+            }
+        }
     }
     __syncthreads();
     float lsum = 0.0f, s = 1.0f, z = 0.0f;
@@ -329,7 +395,7 @@ __global__ void __launch_bounds__(RT) gptq_block_kernel(const BlockParams p) {
         float q = __fadd_rn(rintf(__fdiv_rn(wt, s)), z);  // nearbyint(w / s) + zp
         q = fminf(fmaxf(q, p.qmin), p.qmax);
         const float wh = __fmul_rn(__fsub_rn(q, z), s);
-        const float e = __fmul_rn(__fsub_rn(wt, wh), p.vd[c]);  // (w - w_hat) / U_cc
+        const float e = __fmul_rn(__fsub_rn(wt, wh), vds[i]);  // (w - w_hat) / U_cc
         lsum = fmaf(e, e, lsum);
         const float dl = __fsub_rn(wo[i * RTP + t], wh);
         wo[i * RTP + t] = wh;
@@ -338,8 +404,18 @@ __global__ void __launch_bounds__(RT) gptq_block_kernel(const BlockParams p) {
             if (p.codes) p.codes[(size_t)c * p.R + r] = (uint8_t)(int)(q + p.half);
         }
         const float* vrow = Vs + i * cnt;
-#pragma unroll 4
-        for (int j = i + 1; j < cnt; ++j) la[j * RTP + t] = fmaf(dl, vrow[j], la[j * RTP + t]);
+        int j = i + 1;
+        for (; j + 7 < cnt; j += 8) {  // eight loads in flight, then the eight updates
+            float v[8], a[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                v[u] = vrow[j + u];
+                a[u] = la[(j + u) * RTP + t];
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) la[(j + u) * RTP + t] = fmaf(dl, v[u], a[u]);
+        }
+        for (; j < cnt; ++j) la[j * RTP + t] = fmaf(dl, vrow[j], la[j * RTP + t]);
     }
     if (live) p.losses[r] += 0.5f * lsum;
     __syncthreads();
@@ -356,31 +432,59 @@ __global__ void __launch_bounds__(RT) gptq_block_kernel(const BlockParams p) {
 constexpr int UT = 128;  // output tile (j and r)
 constexpr int UK = 8;    // k chunk
 
+// 256 threads, 8 x 8 outputs each.  The next k chunk is read into registers
+// while the current one is multiplied from shared memory (two buffers, one
+// barrier per chunk).  VEC: C, R and i2 multiples of 4, so every global access
+// is a 16-byte vector.
+template <bool VEC>
 __global__ void __launch_bounds__(256) gptq_update_kernel(const float* __restrict__ P, const float* __restrict__ D,
                                                           float* __restrict__ Acc, int R, int C, int i1, int cnt,
                                                           int i2) {
-    __shared__ __align__(16) float As[UK][UT];
-    __shared__ __align__(16) float Bs[UK][UT];
+    __shared__ __align__(16) float As[2][UK][UT];
+    __shared__ __align__(16) float Bs[2][UK][UT];
     const int tid = threadIdx.x;
     const int j0 = i2 + blockIdx.x * UT, rb = blockIdx.y * UT;
     const int ty = tid / 16, tx = tid % 16;
-    float acc[8][8] = {};
     const int lk = tid / 32, lc = (tid % 32) * 4;  // loader: one k row, four columns
-    for (int k0 = 0; k0 < cnt; k0 += UK) {
+    float acc[8][8] = {};
+    float pa[4], pb[4];
+    auto fetch = [&](int k0) {
         const int k = k0 + lk;
+        const int j = j0 + lc, rr = rb + lc;
+        if (VEC) {
+            const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 a4 = (k < cnt && j < C) ? *reinterpret_cast<const float4*>(P + (size_t)(i1 + k) * C + j) : z4;
+            const float4 b4 = (k < cnt && rr < R) ? *reinterpret_cast<const float4*>(D + (size_t)k * R + rr) : z4;
+            pa[0] = a4.x; pa[1] = a4.y; pa[2] = a4.z; pa[3] = a4.w;
+            pb[0] = b4.x; pb[1] = b4.y; pb[2] = b4.z; pb[3] = b4.w;
+        } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                pa[u] = (k < cnt && j + u < C) ? P[(size_t)(i1 + k) * C + j + u] : 0.0f;
+                pb[u] = (k < cnt && rr + u < R) ? D[(size_t)k * R + rr + u] : 0.0f;
+            }
+        }
+    };
+    auto stash = [&](int buf) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const int j = j0 + lc + u, rr = rb + lc + u;
-            As[lk][lc + u] = (k < cnt && j < C) ? P[(size_t)(i1 + k) * C + j] : 0.0f;
-            Bs[lk][lc + u] = (k < cnt && rr < R) ? D[(size_t)k * R + rr] : 0.0f;
+            As[buf][lk][lc + u] = pa[u];
+            Bs[buf][lk][lc + u] = pb[u];
         }
-        __syncthreads();
+    };
+    const int nchunk = (cnt + UK - 1) / UK;
+    fetch(0);
+    stash(0);
+    __syncthreads();
+    for (int kc = 0; kc < nchunk; ++kc) {
+        const int buf = kc & 1;
+        if (kc + 1 < nchunk) fetch((kc + 1) * UK);
 #pragma unroll
         for (int kk = 0; kk < UK; ++kk) {
-            const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
-            const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][64 + ty * 4]);
-            const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
-            const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][64 + tx * 4]);
+            const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+            const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
+            const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+            const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
             const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
             const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -388,6 +492,7 @@ __global__ void __launch_bounds__(256) gptq_update_kernel(const float* __restric
 #pragma unroll
                 for (int v = 0; v < 8; ++v) acc[u][v] = fmaf(a[u], b[v], acc[u][v]);
         }
+        if (kc + 1 < nchunk) stash(buf ^ 1);
         __syncthreads();
     }
 #pragma unroll
@@ -395,9 +500,23 @@ __global__ void __launch_bounds__(256) gptq_update_kernel(const float* __restric
         const int j = j0 + (u < 4 ? ty * 4 + u : 64 + ty * 4 + u - 4);
         if (j >= C) continue;
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-            const int rr = rb + (v < 4 ? tx * 4 + v : 64 + tx * 4 + v - 4);
-            if (rr < R) Acc[(size_t)j * R + rr] += acc[u][v];
+        for (int h = 0; h < 2; ++h) {
+            const int r4 = rb + h * 64 + tx * 4;
+            float* dst = Acc + (size_t)j * R + r4;
+            if (VEC) {
+                if (r4 < R) {
+                    float4 o = *reinterpret_cast<float4*>(dst);
+                    o.x += acc[u][4 * h + 0];
+                    o.y += acc[u][4 * h + 1];
+                    o.z += acc[u][4 * h + 2];
+                    o.w += acc[u][4 * h + 3];
+                    *reinterpret_cast<float4*>(dst) = o;
+                }
+            } else {
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                    if (r4 + v < R) dst[v] += acc[u][4 * h + v];
+            }
         }
     }
 }
@@ -425,7 +544,7 @@ wq_status launch_gptq(const float* W, const float* H, const float* scale, const 
     gptq_transpose_kernel<<<dim3((C + 31) / 32, (R + 31) / 32), dim3(32, 8), 0, s>>>(W, H, R, C, Wt, Acc);
     for (int k0 = 0; k0 < C; k0 += NB) {
         const int nb = C - k0 < NB ? C - k0 : NB;
-        chol_diag_kernel<<<1, 256, 0, s>>>(P, C, k0, nb, Linv);
+        chol_diag_kernel<<<1, NB, 0, s>>>(P, C, k0, nb, Linv);
         const int rest = C - k0 - nb;
         if (rest > 0) {
             const int T = (rest + NB - 1) / NB;
@@ -437,7 +556,7 @@ wq_status launch_gptq(const float* W, const float* H, const float* scale, const 
     if (cudaGetLastError() != cudaSuccess) return WQ_ERR_CUDA;
 
     const int NG = (C + G - 1) / G;
-    const size_t smem_max = sizeof(float) * ((size_t)BMAX * BMAX + 2 * (size_t)BMAX * RTP);
+    const size_t smem_max = sizeof(float) * ((size_t)BMAX * BMAX + 2 * (size_t)BMAX * RTP + BMAX);
     static std::atomic<uint64_t> attr_ctx[MAX_DEVICES];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return WQ_ERR_CUDA;
@@ -450,12 +569,16 @@ wq_status launch_gptq(const float* W, const float* H, const float* scale, const 
         const int cnt = C - i1 < blocksize ? C - i1 : blocksize;
         bp.i1 = i1;
         bp.cnt = cnt;
-        const size_t smem = sizeof(float) * ((size_t)cnt * cnt + 2 * (size_t)cnt * RTP);
+        const size_t smem = sizeof(float) * ((size_t)cnt * cnt + 2 * (size_t)cnt * RTP + cnt);
         gptq_block_kernel<<<(R + RT - 1) / RT, RT, smem, s>>>(bp);
         const int i2 = i1 + cnt;
-        if (i2 < C)
-            gptq_update_kernel<<<dim3((C - i2 + UT - 1) / UT, (R + UT - 1) / UT), 256, 0, s>>>(P, D, Acc, R, C, i1,
-                                                                                               cnt, i2);
+        if (i2 < C) {
+            const dim3 grid((C - i2 + UT - 1) / UT, (R + UT - 1) / UT);
+            if ((C % 4) == 0 && (R % 4) == 0 && (i2 % 4) == 0)
+                gptq_update_kernel<true><<<grid, 256, 0, s>>>(P, D, Acc, R, C, i1, cnt, i2);
+            else
+                gptq_update_kernel<false><<<grid, 256, 0, s>>>(P, D, Acc, R, C, i1, cnt, i2);
+        }
     }
     return cudaGetLastError() == cudaSuccess ? WQ_OK : WQ_ERR_CUDA;
 }
