@@ -331,7 +331,8 @@ struct BlockParams {
 // One thread per row, RT rows per CTA.  Shared memory: the block's V'
 // (cnt x cnt), the current values w' of the block's columns (column-major by
 // thread, padded) and the original values, which are replaced by w_hat for the
-// coalesced store of Q at the end.
+// coalesced store of Q at the end.  The loop takes the block in sub-blocks of
+// 32 columns held in registers.
 __global__ void __launch_bounds__(RT) gptq_block_kernel(const BlockParams p) {
     extern __shared__ float sm[];
     const int cnt = p.cnt;
@@ -383,39 +384,57 @@ __global__ void __launch_bounds__(RT) gptq_block_kernel(const BlockParams p) {
     __syncthreads();
     float lsum = 0.0f, s = 1.0f, z = 0.0f;
     int gcur = -1;
-    for (int i = 0; i < cnt; ++i) {
-        const int c = p.i1 + i;
-        const int g = c / p.G;
-        if (g != gcur) {
-            gcur = g;
-            s = live ? p.scale[(size_t)r * p.NG + g] : 1.0f;
-            z = live ? p.zero[(size_t)r * p.NG + g] : 0.0f;
-        }
-        const float wt = la[i * RTP + t];
-        float q = __fadd_rn(rintf(__fdiv_rn(wt, s)), z);  // nearbyint(w / s) + zp
-        q = fminf(fmaxf(q, p.qmin), p.qmax);
-        const float wh = __fmul_rn(__fsub_rn(q, z), s);
-        const float e = __fmul_rn(__fsub_rn(wt, wh), vds[i]);  // (w - w_hat) / U_cc
-        lsum = fmaf(e, e, lsum);
-        const float dl = __fsub_rn(wo[i * RTP + t], wh);
-        wo[i * RTP + t] = wh;
-        if (live) {
-            p.D[(size_t)i * p.R + r] = dl;
-            if (p.codes) p.codes[(size_t)c * p.R + r] = (uint8_t)(int)(q + p.half);
-        }
-        const float* vrow = Vs + i * cnt;
-        int j = i + 1;
-        for (; j + 7 < cnt; j += 8) {  // eight loads in flight, then the eight updates
-            float v[8], a[8];
+    // sub-blocks of SB columns: their current values and errors in registers,
+    // their errors then applied to the block's later columns as SB-term sums
+    constexpr int SB = 32;
+    for (int s0 = 0; s0 < cnt; s0 += SB) {
+        float cur[SB], dl[SB];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                v[u] = vrow[j + u];
-                a[u] = la[(j + u) * RTP + t];
+        for (int u = 0; u < SB; ++u) cur[u] = (s0 + u < cnt) ? la[(s0 + u) * RTP + t] : 0.0f;
+#pragma unroll
+        for (int u = 0; u < SB; ++u) {
+            dl[u] = 0.0f;
+            const int i = s0 + u;
+            if (i < cnt) {
+                const int c = p.i1 + i;
+                const int g = c / p.G;
+                if (g != gcur) {
+                    gcur = g;
+                    s = live ? p.scale[(size_t)r * p.NG + g] : 1.0f;
+                    z = live ? p.zero[(size_t)r * p.NG + g] : 0.0f;
+                }
+                const float wt = cur[u];
+                float q = __fadd_rn(rintf(__fdiv_rn(wt, s)), z);  // nearbyint(w / s) + zp
+                q = fminf(fmaxf(q, p.qmin), p.qmax);
+                const float wh = __fmul_rn(__fsub_rn(q, z), s);
+                const float e = __fmul_rn(__fsub_rn(wt, wh), vds[i]);  // (w - w_hat) / U_cc
+                lsum = fmaf(e, e, lsum);
+                dl[u] = __fsub_rn(wo[i * RTP + t], wh);
+                wo[i * RTP + t] = wh;
+                if (live) {
+                    p.D[(size_t)i * p.R + r] = dl[u];
+                    if (p.codes) p.codes[(size_t)c * p.R + r] = (uint8_t)(int)(q + p.half);
+                }
+                const float* vrow = Vs + i * cnt + s0;  // V'[i][s0 + v]
+#pragma unroll
+                for (int v = u + 1; v < SB; ++v) cur[v] = fmaf(dl[u], vrow[v < cnt - s0 ? v : 0], cur[v]);
+            }
+        }
+        // the block's later columns: la[j] += sum_u dl[u] V'[s0 + u][j], four columns at a time
+        for (int j = s0 + SB; j < cnt; j += 4) {
+            float acc4[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc4[k] = (j + k < cnt) ? la[(j + k) * RTP + t] : 0.0f;
+#pragma unroll
+            for (int u = 0; u < SB; ++u) {
+                const float* vrow = Vs + (s0 + u) * cnt + j;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) acc4[k] = fmaf(dl[u], (j + k < cnt) ? vrow[k] : 0.0f, acc4[k]);
             }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) la[(j + u) * RTP + t] = fmaf(dl, v[u], a[u]);
+            for (int k = 0; k < 4; ++k)
+                if (j + k < cnt) la[(j + k) * RTP + t] = acc4[k];
         }
-        for (; j < cnt; ++j) la[j * RTP + t] = fmaf(dl, vrow[j], la[j * RTP + t]);
     }
     if (live) p.losses[r] += 0.5f * lsum;
     __syncthreads();

@@ -379,8 +379,9 @@ wq_status wq_device_status(int reset);
 
 /*
  * 1 if this library is the checked build (compiled with WQ_CHECKS, as
- * libwq_checked.so), else 0.  Host-only.  In the checked build every kernel
- * checks the index of each global and shared-memory access it computes itself
+ * libwq_checked.so), else 0.  Host-only.  In the checked build every kernel of
+ * the products (wq_gemv, wq_gemm and their plans) checks the index of each
+ * global and shared-memory access it computes itself
  * (x, y, the split-K workspace, the s/z rows and the staging buffers; the TMA
  * copies are bounded by their descriptors) against the array it belongs to;
  * an access that fails is skipped and recorded, and wq_device_status then
