@@ -1,5 +1,5 @@
 // wq_gemv_lean.cu -- decode-time product y (M x N) = x (M x K) @ dequant(W_q) for
-// 1 <= M <= 8 and 4- or 8-bit words, with a small shared-memory footprint.
+// 1 <= M <= 16 and 2-, 4- or 8-bit words, with a small shared-memory footprint.
 //
 // What is computed: dashq_kernel.py `_dashq_gemv_kernel` (one token there; up to
 // 8 here): each output column n is sum_k x[k] * (q[k][n] - z[g][n]) * s[g][n],
@@ -21,7 +21,7 @@
 //    whole range, so a CTA's words are all in flight at once.  Slots are
 //    refilled as they are consumed when the range is longer.  One more TMA copy
 //    brings the s and z rows of the CTA's groups.
-//  * x is not staged: each lane reads the 16 (8-bit: 8) bytes of x its word row
+//  * x is not staged: each lane reads the 16 (8-bit: 8, 2-bit: 32) bytes of x its word row
 //    needs straight from global memory (L2-resident: every CTA reads the same
 //    x), a group of quads ahead of their use, and permutes them into the MMA's
 //    k order with PRMT.
@@ -81,21 +81,34 @@ struct LeanParams {
     int late_wait;  // wait for the previous kernel only before writing y
 };
 
-// The 16 (8-bit: 8) bytes of x that word row k0 / EPS needs, token row xr;
-// zeros at and beyond K.
+// The x values of one word row: 16 bytes (4-bit; 8-bit: the first 8), or
+// 32 bytes for the 16 values of a 2-bit word row.
+struct X16 {
+    uint4 a, b;
+};
 template <int EPS>
-__device__ __forceinline__ uint4 ldg_x(const uint16_t* xr, int k0, int K) {
+using XRow = std::conditional_t<(EPS == 16), X16, uint4>;
+
+// The bytes of x that word row k0 / EPS needs, token row xr; zeros at and beyond K.
+template <int EPS>
+__device__ __forceinline__ XRow<EPS> ldg_x(const uint16_t* xr, int k0, int K) {
     const bool in = k0 < K;
     const uint16_t* src = xr + (in ? k0 : 0);  // a row past K reads row 0 and is zeroed below
-    uint4 r;
-    if constexpr (EPS == 8) {
-        r = __ldg(reinterpret_cast<const uint4*>(src));
+    if constexpr (EPS == 16) {
+        X16 r{__ldg(reinterpret_cast<const uint4*>(src)), __ldg(reinterpret_cast<const uint4*>(src) + 1)};
+        if (!in) r = X16{};
+        return r;
     } else {
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(src));
-        r = make_uint4(v.x, v.y, 0u, 0u);
+        uint4 r;
+        if constexpr (EPS == 8) {
+            r = __ldg(reinterpret_cast<const uint4*>(src));
+        } else {
+            const uint2 v = __ldg(reinterpret_cast<const uint2*>(src));
+            r = make_uint4(v.x, v.y, 0u, 0u);
+        }
+        if (!in) r = make_uint4(0u, 0u, 0u, 0u);
+        return r;
     }
-    if (!in) r = make_uint4(0u, 0u, 0u, 0u);
-    return r;
 }
 
 // Conversion constants of a lane's 4 columns for one group, from the group's z
@@ -120,7 +133,15 @@ struct GroupConsts {
                 const uint32_t c0 = hsub2_u32(h2c(0x6000u), r);  // 512 - 1536 - zi = -(1024 + zi)
                 cc[2 * h][0] = prmt(c0, c0, 0x1010u);
                 cc[2 * h + 1][0] = prmt(c0, c0, 0x3232u);
-                if constexpr (NC > 1) {
+                if constexpr (BITS == 2) {  // -(1024 / 4^ci + zi) = (1536 - 1024 / 4^ci) - (1536 + zi), exact
+                    constexpr uint32_t A[4] = {0x6500u, 0x65C0u, 0x65F0u, 0x65FCu};  // 1280, 1472, 1520, 1532
+#pragma unroll
+                    for (int ci = 1; ci < NC; ++ci) {
+                        const uint32_t cx = hsub2_u32(h2c(A[ci - 1]), r);
+                        cc[2 * h][ci] = prmt(cx, cx, 0x1010u);
+                        cc[2 * h + 1][ci] = prmt(cx, cx, 0x3232u);
+                    }
+                } else if constexpr (NC > 1) {
                     const uint32_t c1 = hsub2_u32(h2c(0x65C0u), r);  // 1472 - 1536 - zi = -(64 + zi)
                     cc[2 * h][1] = prmt(c1, c1, 0x1010u);
                     cc[2 * h + 1][1] = prmt(c1, c1, 0x3232u);
@@ -291,9 +312,14 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
             const int kl = kx0 + 4 * EPS * i;
             const bool ok = XS ? (kl - kc0 + EPS <= LWK * p.QW * 4 * EPS && (uint32_t)(kl - kc0 + EPS) * 2u <= p.xs_stride)
                                : (kl + EPS <= p.K);
-            if (!check(ok, &g_gemv_lean_status)) return make_uint4(0u, 0u, 0u, 0u);
+            if (!check(ok, &g_gemv_lean_status)) return XRow<EPS>{};
         }
-        if constexpr (XS) {
+        if constexpr (EPS == 16) {  // 4 word rows = 64 values on per quad
+            if constexpr (XS)
+                return X16{lds128_u32(xs_lane[n] + 128u * i), lds128_u32(xs_lane[n] + 128u * i + 16u)};
+            const uint4* src = reinterpret_cast<const uint4*>(xr[n] + kx0) + 8 * i;
+            return X16{__ldg(src), __ldg(src + 1)};
+        } else if constexpr (XS) {
             if constexpr (EPS == 8) return lds128_u32(xs_lane[n] + 64u * i);
             const uint2 v = lds64_u32(xs_lane[n] + 32u * i);
             return make_uint4(v.x, v.y, 0u, 0u);
@@ -375,25 +401,39 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
             }
         };
         // one quad: the words hv (this lane's 16 bytes) and its x values xa[n]
-        auto quad = [&](const uint4& hv, const uint4 (&xa)[NT]) {
+        auto quad = [&](const uint4& hv, const XRow<EPS> (&xa)[NT]) {
             uint32_t bx[NT][EPS / 2];
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
-                if constexpr (EPS == 8) {  // pairs (0, 4), (1, 5), (2, 6), (3, 7) of the row's 8 values
-                    bx[n][0] = prmt(xa[n].x, xa[n].z, 0x5410u);
-                    bx[n][1] = prmt(xa[n].x, xa[n].z, 0x7632u);
-                    bx[n][2] = prmt(xa[n].y, xa[n].w, 0x5410u);
-                    bx[n][3] = prmt(xa[n].y, xa[n].w, 0x7632u);
-                } else {                   // pairs (0, 2), (1, 3) of the row's 4 values
-                    bx[n][0] = prmt(xa[n].x, xa[n].y, 0x5410u);
-                    bx[n][1] = prmt(xa[n].x, xa[n].y, 0x7632u);
-                }
-                if constexpr (FRAC) {  // this lane's row sum of x (fp32)
-                    const uint32_t xv[4] = {xa[n].x, xa[n].y, xa[n].z, xa[n].w};
+                if constexpr (EPS == 16) {  // pairs (j, j + 8) of the row's 16 values
+                    const uint32_t lo[4] = {xa[n].a.x, xa[n].a.y, xa[n].a.z, xa[n].a.w};
+                    const uint32_t hi[4] = {xa[n].b.x, xa[n].b.y, xa[n].b.z, xa[n].b.w};
 #pragma unroll
-                    for (int u = 0; u < EPS / 2; ++u) {
-                        const float2 f = T16::pair(xv[u]);
-                        xsum[n] += f.x + f.y;
+                    for (int j = 0; j < 8; ++j) bx[n][j] = prmt(lo[j >> 1], hi[j >> 1], (j & 1) ? 0x7632u : 0x5410u);
+                    if constexpr (FRAC) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float2 f = T16::pair(lo[u]), h = T16::pair(hi[u]);
+                            xsum[n] += (f.x + f.y) + (h.x + h.y);
+                        }
+                    }
+                } else {
+                    if constexpr (EPS == 8) {  // pairs (0, 4), (1, 5), (2, 6), (3, 7) of the row's 8 values
+                        bx[n][0] = prmt(xa[n].x, xa[n].z, 0x5410u);
+                        bx[n][1] = prmt(xa[n].x, xa[n].z, 0x7632u);
+                        bx[n][2] = prmt(xa[n].y, xa[n].w, 0x5410u);
+                        bx[n][3] = prmt(xa[n].y, xa[n].w, 0x7632u);
+                    } else {                   // pairs (0, 2), (1, 3) of the row's 4 values
+                        bx[n][0] = prmt(xa[n].x, xa[n].y, 0x5410u);
+                        bx[n][1] = prmt(xa[n].x, xa[n].y, 0x7632u);
+                    }
+                    if constexpr (FRAC) {  // this lane's row sum of x (fp32)
+                        const uint32_t xv[4] = {xa[n].x, xa[n].y, xa[n].z, xa[n].w};
+#pragma unroll
+                        for (int u = 0; u < EPS / 2; ++u) {
+                            const float2 f = T16::pair(xv[u]);
+                            xsum[n] += f.x + f.y;
+                        }
                     }
                 }
             }
@@ -420,7 +460,7 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
             const uint32_t wblk = slot_addr + 512u * (uint32_t)i4;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                uint4 xa[NT];
+                XRow<EPS> xa[NT];
 #pragma unroll
                 for (int n = 0; n < NT; ++n) xa[n] = ldx(i + j, n);
                 quad(lds128_u32(wblk + 512u * j + ((j & 1) ? off_odd : off_even)), xa);
@@ -473,7 +513,7 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             if (i + j < nq) {
-                                uint4 xa[NT];
+                                XRow<EPS> xa[NT];
 #pragma unroll
                                 for (int n = 0; n < NT; ++n) xa[n] = ldx_guarded(i + j, n);
                                 quad(lds128_u32(wblk + 512u * j + ((j & 1) ? off_odd : off_even)), xa);
@@ -895,7 +935,7 @@ wq_status gemv_lean_device_status(int reset) {
 }
 
 bool gemv_lean_takes(const Problem& p) {
-    if (p.bits != 4 && p.bits != 8) return false;
+    if (p.bits != 2 && p.bits != 4 && p.bits != 8) return false;
     if (p.M > 16) return false;
     // x written by the previous kernel on the stream: the staged copy of x is
     // read in 16-byte rows
@@ -907,6 +947,7 @@ bool gemv_lean_takes(const Problem& p) {
 wq_status launch_gemv_lean(const Problem& p, cudaStream_t s, Prepared* prep) {
     const bool bf = (p.flags & WQ_FLAG_BF16) != 0;
     switch (p.bits) {
+        case 2: return bf ? run_lean<2, true>(p, s, prep) : run_lean<2, false>(p, s, prep);
         case 4: return bf ? run_lean<4, true>(p, s, prep) : run_lean<4, false>(p, s, prep);
         case 8: return bf ? run_lean<8, true>(p, s, prep) : run_lean<8, false>(p, s, prep);
         default: return WQ_ERR_UNSUPPORTED;

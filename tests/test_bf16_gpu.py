@@ -57,6 +57,8 @@ GEMV_SHAPES = [
     (1, 1024, 200, 3, 64),
     (12, 2048, 56, 3, 128),
     (4, 8192, 16, 4, 128),
+    (1, 8192, 128, 2, 128),   # 2-bit words on the lean kernel
+    (11, 2048, 72, 2, -1),
 ]
 
 

@@ -56,6 +56,10 @@ SHAPES = [
     (9, 1056, 40, 4, 32),     # 33 quads over 8 warps, G = 32: one group per quad
     (1, 4096, 4104, 4, 128),  # the one-token decode kernel, ragged last column block
     (1, 2048, 4096, 4, 128),  # the one-token decode kernel, 8 quads per warp
+    (1, 8192, 256, 2, 128),   # 2-bit words on the lean kernel: one token, aligned plan
+    (16, 2048, 96, 2, 128),   # 2-bit, two token tiles
+    (4, 4096, 136, 2, -1),    # 2-bit per channel, ragged column block
+    (5, 1088, 40, 2, 64),     # 2-bit, 17 quads over 8 warps (ragged range)
 ]
 
 
@@ -259,6 +263,7 @@ def test_rejected_calls(cuda, libwq):
 # quads per warp (G = 256: two 4-quad blocks per group).  G = -1 is one group
 # across the range.
 ALIGNED = [(3, 16384, 64, 4, 128), (1, 16384, 64, 4, -1), (2, 8192, 64, 8, 128), (1, 4096, 4096, 4, 256),
+           (1, 8192, 512, 2, 128), (6, 8192, 64, 2, 128),
            (1, 4096, 4096, 4, 128), (1, 2048, 2560, 4, 128)]  # the last two: the one-token decode kernel
 
 
@@ -306,9 +311,9 @@ def test_aligned_plan_one_hot_rows_are_exact(cuda, libwq, M, K, N, bits, G):
     assert np.array_equal(y, w.astype(np.float16))
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", [2, 4, 8])
 def test_pdl_chain_at_decode_size(cuda, libwq, orc, bits):
-    """WQ_FLAG_PDL on the 4096 x 4096 decode shape (the staged-x plan of the 4/8-bit
+    """WQ_FLAG_PDL on the 4096 x 4096 decode shape (the staged-x plan of the 2/4/8-bit
     kernel): the first product matches the oracle, and the overlapped chain gives
     the same bits as the same calls run one at a time."""
     import torch
