@@ -1,5 +1,5 @@
 // wq_gemv_lean.cu -- decode-time product y (M x N) = x (M x K) @ dequant(W_q) for
-// 1 <= M <= 16 and 2-, 4- or 8-bit words, with a small shared-memory footprint.
+// 1 <= M <= 16 and 1-, 2-, 4- or 8-bit words, with a small shared-memory footprint.
 //
 // What is computed: dashq_kernel.py `_dashq_gemv_kernel` (one token there; up to
 // 8 here): each output column n is sum_k x[k] * (q[k][n] - z[g][n]) * s[g][n],
@@ -81,20 +81,28 @@ struct LeanParams {
     int late_wait;  // wait for the previous kernel only before writing y
 };
 
-// The x values of one word row: 16 bytes (4-bit; 8-bit: the first 8), or
-// 32 bytes for the 16 values of a 2-bit word row.
+// The x values of one word row: 16 bytes (4-bit; 8-bit: the first 8), 32
+// bytes for the 16 values of a 2-bit word row, 64 for the 32 of a 1-bit one.
 struct X16 {
     uint4 a, b;
 };
+struct X32 {
+    uint4 a, b, c, d;
+};
 template <int EPS>
-using XRow = std::conditional_t<(EPS == 16), X16, uint4>;
+using XRow = std::conditional_t<(EPS == 32), X32, std::conditional_t<(EPS == 16), X16, uint4>>;
 
 // The bytes of x that word row k0 / EPS needs, token row xr; zeros at and beyond K.
 template <int EPS>
 __device__ __forceinline__ XRow<EPS> ldg_x(const uint16_t* xr, int k0, int K) {
     const bool in = k0 < K;
     const uint16_t* src = xr + (in ? k0 : 0);  // a row past K reads row 0 and is zeroed below
-    if constexpr (EPS == 16) {
+    if constexpr (EPS == 32) {
+        const uint4* v = reinterpret_cast<const uint4*>(src);
+        X32 r{__ldg(v), __ldg(v + 1), __ldg(v + 2), __ldg(v + 3)};
+        if (!in) r = X32{};
+        return r;
+    } else if constexpr (EPS == 16) {
         X16 r{__ldg(reinterpret_cast<const uint4*>(src)), __ldg(reinterpret_cast<const uint4*>(src) + 1)};
         if (!in) r = X16{};
         return r;
@@ -133,7 +141,16 @@ struct GroupConsts {
                 const uint32_t c0 = hsub2_u32(h2c(0x6000u), r);  // 512 - 1536 - zi = -(1024 + zi)
                 cc[2 * h][0] = prmt(c0, c0, 0x1010u);
                 cc[2 * h + 1][0] = prmt(c0, c0, 0x3232u);
-                if constexpr (BITS == 2) {  // -(1024 / 4^ci + zi) = (1536 - 1024 / 4^ci) - (1536 + zi), exact
+                if constexpr (BITS == 1) {  // -(1024 / 2^ci + zi) = (1536 - 1024 / 2^ci) - (1536 + zi), exact
+                    constexpr uint32_t A[9] = {0x6400u, 0x6500u, 0x6580u, 0x65C0u, 0x65E0u,
+                                               0x65F0u, 0x65F8u, 0x65FCu, 0x65FEu};  // 1024, 1280, ..., 1534
+#pragma unroll
+                    for (int ci = 1; ci < NC; ++ci) {
+                        const uint32_t cx = hsub2_u32(h2c(A[ci - 1]), r);
+                        cc[2 * h][ci] = prmt(cx, cx, 0x1010u);
+                        cc[2 * h + 1][ci] = prmt(cx, cx, 0x3232u);
+                    }
+                } else if constexpr (BITS == 2) {  // -(1024 / 4^ci + zi) = (1536 - 1024 / 4^ci) - (1536 + zi), exact
                     constexpr uint32_t A[4] = {0x6500u, 0x65C0u, 0x65F0u, 0x65FCu};  // 1280, 1472, 1520, 1532
 #pragma unroll
                     for (int ci = 1; ci < NC; ++ci) {
@@ -167,9 +184,10 @@ struct GroupConsts {
 // not depend on it is issued and waited for first; after the grid dependency
 // wait the CTA copies its slice of x into shared memory in one round trip, and
 // the quads read it from there.
-// TOK: 1 (one token), 8 (M <= 8) or 16 (M <= 16: two 8-token MMA tiles).
+// TOK: 1 (one token), 8 (M <= 8) or 16 (M <= 16: two 8-token MMA tiles; not
+// for 1-bit words, whose ten conversion constants per column leave no room).
 template <int BITS, bool BF, int BQ, int TOK, bool ALIGNED, bool XS>
-__global__ void __launch_bounds__(LWK * 32, TOK > 8 ? 2 : 3)
+__global__ void __launch_bounds__(LWK * 32, (TOK > 8 || BITS == 1) ? 2 : 3)
 gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
                  const __grid_constant__ CUtensorMap tm_z, const LeanParams p) {
     using F = Fmt<BITS>;
@@ -314,7 +332,14 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
                                : (kl + EPS <= p.K);
             if (!check(ok, &g_gemv_lean_status)) return XRow<EPS>{};
         }
-        if constexpr (EPS == 16) {  // 4 word rows = 64 values on per quad
+        if constexpr (EPS == 32) {  // 4 word rows = 128 values on per quad
+            if constexpr (XS) {
+                const uint32_t a = xs_lane[n] + 256u * i;
+                return X32{lds128_u32(a), lds128_u32(a + 16u), lds128_u32(a + 32u), lds128_u32(a + 48u)};
+            }
+            const uint4* src = reinterpret_cast<const uint4*>(xr[n] + kx0) + 16 * i;
+            return X32{__ldg(src), __ldg(src + 1), __ldg(src + 2), __ldg(src + 3)};
+        } else if constexpr (EPS == 16) {  // 4 word rows = 64 values on per quad
             if constexpr (XS)
                 return X16{lds128_u32(xs_lane[n] + 128u * i), lds128_u32(xs_lane[n] + 128u * i + 16u)};
             const uint4* src = reinterpret_cast<const uint4*>(xr[n] + kx0) + 8 * i;
@@ -405,7 +430,21 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
             uint32_t bx[NT][EPS / 2];
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
-                if constexpr (EPS == 16) {  // pairs (j, j + 8) of the row's 16 values
+                if constexpr (EPS == 32) {  // pairs (j, j + 16) of the row's 32 values
+                    const uint32_t lo[8] = {xa[n].a.x, xa[n].a.y, xa[n].a.z, xa[n].a.w,
+                                            xa[n].b.x, xa[n].b.y, xa[n].b.z, xa[n].b.w};
+                    const uint32_t hi[8] = {xa[n].c.x, xa[n].c.y, xa[n].c.z, xa[n].c.w,
+                                            xa[n].d.x, xa[n].d.y, xa[n].d.z, xa[n].d.w};
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) bx[n][j] = prmt(lo[j >> 1], hi[j >> 1], (j & 1) ? 0x7632u : 0x5410u);
+                    if constexpr (FRAC) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const float2 f = T16::pair(lo[u]), h = T16::pair(hi[u]);
+                            xsum[n] += (f.x + f.y) + (h.x + h.y);
+                        }
+                    }
+                } else if constexpr (EPS == 16) {  // pairs (j, j + 8) of the row's 16 values
                     const uint32_t lo[4] = {xa[n].a.x, xa[n].a.y, xa[n].a.z, xa[n].a.w};
                     const uint32_t hi[4] = {xa[n].b.x, xa[n].b.y, xa[n].b.z, xa[n].b.w};
 #pragma unroll
@@ -911,7 +950,8 @@ wq_status run_lean(const Problem& pb, cudaStream_t stream, Prepared* prep) {
             constexpr bool X = decltype(xs_tag)::value;
             if (pb.M == 1) return launch_lean<BITS, BF, B, 1, A, X>(mw, ms, mz, p, smem, pb, stream, prep);
             if (pb.M <= 8) return launch_lean<BITS, BF, B, 8, A, X>(mw, ms, mz, p, smem, pb, stream, prep);
-            return launch_lean<BITS, BF, B, 16, A, X>(mw, ms, mz, p, smem, pb, stream, prep);
+            if constexpr (BITS == 1) return WQ_ERR_UNSUPPORTED;  // two 1-bit token tiles spill: not routed here
+            else return launch_lean<BITS, BF, B, 16, A, X>(mw, ms, mz, p, smem, pb, stream, prep);
         };
         return xs ? tok(std::true_type{}) : tok(std::false_type{});
     };
@@ -935,8 +975,8 @@ wq_status gemv_lean_device_status(int reset) {
 }
 
 bool gemv_lean_takes(const Problem& p) {
-    if (p.bits != 2 && p.bits != 4 && p.bits != 8) return false;
-    if (p.M > 16) return false;
+    if (p.bits == 3) return false;
+    if (p.M > (p.bits == 1 ? 8 : 16)) return false;  // 1-bit with two token tiles would spill registers
     // x written by the previous kernel on the stream: the staged copy of x is
     // read in 16-byte rows
     if ((p.flags & WQ_FLAG_PDL) && !(p.flags & WQ_FLAG_PDL_INPUTS_READY) && p.K % 8 != 0) return false;
@@ -947,6 +987,7 @@ bool gemv_lean_takes(const Problem& p) {
 wq_status launch_gemv_lean(const Problem& p, cudaStream_t s, Prepared* prep) {
     const bool bf = (p.flags & WQ_FLAG_BF16) != 0;
     switch (p.bits) {
+        case 1: return bf ? run_lean<1, true>(p, s, prep) : run_lean<1, false>(p, s, prep);
         case 2: return bf ? run_lean<2, true>(p, s, prep) : run_lean<2, false>(p, s, prep);
         case 4: return bf ? run_lean<4, true>(p, s, prep) : run_lean<4, false>(p, s, prep);
         case 8: return bf ? run_lean<8, true>(p, s, prep) : run_lean<8, false>(p, s, prep);

@@ -53,7 +53,8 @@ struct Prepared {
 // Fill `pr` for problem p (x and y may be null) instead of launching.
 wq_status prepare_gemv(const Problem& p, Prepared& pr);
 wq_status launch_prepared(const Prepared& pr, const void* x, void* y, cudaStream_t s);
-// GEMV with a small shared-memory footprint for 2-, 4- and 8-bit words and M <= 16
+// GEMV with a small shared-memory footprint for 1-, 2-, 4- and 8-bit words and M <= 16
+// (1-bit: M <= 8)
 // (wq_gemv_lean.cu); launch_gemv routes the shapes it takes there.
 bool gemv_lean_takes(const Problem& p);
 wq_status launch_gemv_lean(const Problem& p, cudaStream_t s, Prepared* prep = nullptr);

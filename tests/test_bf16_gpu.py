@@ -59,6 +59,8 @@ GEMV_SHAPES = [
     (4, 8192, 16, 4, 128),
     (1, 8192, 128, 2, 128),   # 2-bit words on the lean kernel
     (11, 2048, 72, 2, -1),
+    (1, 8192, 128, 1, 128),   # 1-bit words on the lean kernel
+    (6, 4096, 64, 1, -1),
 ]
 
 

@@ -60,6 +60,10 @@ SHAPES = [
     (16, 2048, 96, 2, 128),   # 2-bit, two token tiles
     (4, 4096, 136, 2, -1),    # 2-bit per channel, ragged column block
     (5, 1088, 40, 2, 64),     # 2-bit, 17 quads over 8 warps (ragged range)
+    (1, 8192, 512, 1, 128),   # 1-bit words on the lean kernel
+    (8, 4096, 72, 1, -1),     # 1-bit per channel, 8 tokens, ragged column block
+    (3, 2176, 40, 1, 128),    # 1-bit, 17 quads (ragged range)
+    (12, 2048, 64, 1, 128),   # 1-bit with 12 tokens: the table kernel
 ]
 
 
@@ -263,7 +267,7 @@ def test_rejected_calls(cuda, libwq):
 # quads per warp (G = 256: two 4-quad blocks per group).  G = -1 is one group
 # across the range.
 ALIGNED = [(3, 16384, 64, 4, 128), (1, 16384, 64, 4, -1), (2, 8192, 64, 8, 128), (1, 4096, 4096, 4, 256),
-           (1, 8192, 512, 2, 128), (6, 8192, 64, 2, 128),
+           (1, 8192, 512, 2, 128), (6, 8192, 64, 2, 128), (1, 8192, 512, 1, 128), (4, 16384, 64, 1, 128),
            (1, 4096, 4096, 4, 128), (1, 2048, 2560, 4, 128)]  # the last two: the one-token decode kernel
 
 
@@ -311,9 +315,9 @@ def test_aligned_plan_one_hot_rows_are_exact(cuda, libwq, M, K, N, bits, G):
     assert np.array_equal(y, w.astype(np.float16))
 
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", [1, 2, 4, 8])
 def test_pdl_chain_at_decode_size(cuda, libwq, orc, bits):
-    """WQ_FLAG_PDL on the 4096 x 4096 decode shape (the staged-x plan of the 2/4/8-bit
+    """WQ_FLAG_PDL on the 4096 x 4096 decode shape (the staged-x plan of the lean
     kernel): the first product matches the oracle, and the overlapped chain gives
     the same bits as the same calls run one at a time."""
     import torch
