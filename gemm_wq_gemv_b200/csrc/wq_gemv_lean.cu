@@ -178,8 +178,9 @@ struct GroupConsts {
 };
 
 // ALIGNED: one box holds each warp's whole range (QW == BQ quads, all inside K)
-// and groups start on the range's 4-quad blocks, so the main loop runs group by
-// group without per-quad bookkeeping.
+// and groups start on the range's 4-quad blocks or hold 1 or 2 quads (1- and
+// 2-bit words at group 128), so the main loop runs group by group without
+// per-quad bookkeeping.
 // XS: x is written by the previous kernel on the stream.  Every load that does
 // not depend on it is issued and waited for first; after the grid dependency
 // wait the CTA copies its slice of x into shared memory in one round trip, and
@@ -505,6 +506,17 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
                 quad(lds128_u32(wblk + 512u * j + ((j & 1) ? off_odd : off_even)), xa);
             }
         };
+        // CNT (1 or 2) quads from quad i of the slot (a group of 1- or 2-bit words)
+        auto block_short = [&](auto cnt_tag, uint32_t slot_addr, int i) {
+            constexpr int CNT = decltype(cnt_tag)::value;
+#pragma unroll
+            for (int j = 0; j < CNT; ++j) {
+                XRow<EPS> xa[NT];
+#pragma unroll
+                for (int n = 0; n < NT; ++n) xa[n] = ldx(i + j, n);
+                quad(lds128_u32(slot_addr + 512u * (uint32_t)(i + j) + (((i + j) & 1) ? off_odd : off_even)), xa);
+            }
+        };
 
         if constexpr (ALIGNED) {
             if (ok_all && nq > 0) {
@@ -517,8 +529,14 @@ gemv_lean_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
 #pragma unroll 1
             for (int q0 = 0; q0 < BQ; q0 += seg) {
                 if (q0 > 0) consts(gcur);
+                if (seg >= 4) {
 #pragma unroll 1
-                for (int i = q0; i < q0 + seg; i += 4) block(ring0, i, i);
+                    for (int i = q0; i < q0 + seg; i += 4) block(ring0, i, i);
+                } else if (seg == 2) {
+                    block_short(std::integral_constant<int, 2>{}, ring0, q0);
+                } else {
+                    block_short(std::integral_constant<int, 1>{}, ring0, q0);
+                }
                 fold();
                 ++gcur;
             }
@@ -941,7 +959,7 @@ wq_status run_lean(const Problem& pb, cudaStream_t stream, Prepared* prep) {
     // ALIGNED: one box per warp covering its QW quads, every warp of every rank
     // full and inside K, and groups starting on 4-quad blocks of the ranges
     const bool aligned = p.S == 1 && p.QW == BQ && p.Q == KS * LWK * p.QW && p.Kw == 4 * p.Q &&
-                         ((p.qpg <= p.QW && p.QW % p.qpg == 0 && p.qpg % 4 == 0) ||
+                         ((p.qpg <= p.QW && p.QW % p.qpg == 0 && (p.qpg % 4 == 0 || p.qpg <= 2)) ||
                           (p.qpg > p.QW && (p.qpg % p.QW == 0 || p.qpg >= p.Q)));
     auto go = [&](auto bq, auto a) {
         constexpr int B = decltype(bq)::value;

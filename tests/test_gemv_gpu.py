@@ -268,6 +268,7 @@ def test_rejected_calls(cuda, libwq):
 # across the range.
 ALIGNED = [(3, 16384, 64, 4, 128), (1, 16384, 64, 4, -1), (2, 8192, 64, 8, 128), (1, 4096, 4096, 4, 256),
            (1, 8192, 512, 2, 128), (6, 8192, 64, 2, 128), (1, 8192, 512, 1, 128), (4, 16384, 64, 1, 128),
+           (1, 4096, 4096, 4, 64), (1, 8192, 8192, 2, 128),
            (1, 4096, 4096, 4, 128), (1, 2048, 2560, 4, 128)]  # the last two: the one-token decode kernel
 
 
