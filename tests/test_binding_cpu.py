@@ -50,3 +50,16 @@ def test_status_names(libwq):
     assert "scratch" in libwq.describe(7)
     err = libwq.WQError("wq_gemv", 3)
     assert err.status == 3 and "WQ_ERR_ALIGNMENT" in str(err)
+
+
+def test_gptq_refuses_cpu_tensors(libwq):
+    W = torch.zeros((4, 64), dtype=torch.float32)
+    H = torch.eye(64, dtype=torch.float32)
+    s = torch.ones((4, 1), dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        libwq.gptq_quantize(W, H, s, s * 0, 64, 8)
+
+
+def test_gptq_status_name(libwq):
+    assert libwq.STATUS[9] == "WQ_ERR_NOT_POSITIVE_DEFINITE"
+    assert "positive definite" in libwq.describe(9)

@@ -37,3 +37,17 @@ def test_deterministic_and_in_range():
         assert a.codes.max() <= (1 << wl.bits) - 1, name
         assert a.scales.min() >= np.float16(wl.s_lo) and a.scales.max() <= np.float16(wl.s_hi), name
         assert a.scales.shape == (wl.groups, wl.N) and a.x.shape == (wl.M, wl.K), name
+
+
+def test_gptq_problem_recipe():
+    """The GPTQ benchmark's problem: W inside +-1/sqrt(cols), H = A A^T + I
+    symmetric with every eigenvalue at least 1 (up to fp32 rounding), the same
+    bytes for the same seed."""
+    W, H = wq_inputs.gptq_problem(16, 96, seed=3)
+    assert W.dtype == np.float32 and H.dtype == np.float32
+    assert W.shape == (16, 96) and H.shape == (96, 96)
+    assert np.abs(W).max() <= 1 / np.sqrt(96)
+    np.testing.assert_allclose(H, H.T, rtol=1e-6, atol=1e-4)
+    assert np.linalg.eigvalsh(H.astype(np.float64)).min() > 1 - 1e-3
+    W2, H2 = wq_inputs.gptq_problem(16, 96, seed=3)
+    assert np.array_equal(W, W2) and np.array_equal(H, H2)
